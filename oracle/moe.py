@@ -1,0 +1,345 @@
+"""Plain float64 oracle of the routed MoE FFN: route, permute, FFN, combine.
+
+TEST INFRASTRUCTURE ONLY (see the package docstring).
+
+Notation: M tokens, H = hidden, I = intermediate_hidden, E = num_experts,
+k = num_topk.  A routed *slot* is the pair (token t, position j < k), with the
+flat slot index s = t*k + j.
+
+What is computed, per token t (the definition this file restates):
+
+    for every slot j with e = topk_idx[t, j] >= 0:
+        x^     = decode(x[t])                             activation decode
+        g, u   = gate / up projections of x^ by expert e  (L1, "gate_up")
+        h      = min(g, c) * sigmoid(min(g, c)) * clamp(u, -c, c)
+        h^     = decode(requant(h))                       L1 epilogue re-quant
+        y      = down projection of h^ by expert e        (L2, "down")
+    out[t] = bf16( sum_j topk_weights[t, j] * y )         the combine
+
+Sources, by page and section:
+
+* Struct_mega_ffn_ep_combine_send, Args: ``gate_up_weight`` (E, N1, K1//2),
+  ``down_weight`` (E, N2, moe_dim//2), ``gate_up_expert_scales`` (L1
+  per-expert output scaling), ``down_expert_scales`` (L2 per-expert output
+  scaling), ``c_input_scales`` (per-expert input scale of the NVFP4
+  re-quant), ``expert_start_indices`` (per-expert prefix-sum offsets),
+  ``expert_ids`` (-1 = masked), ``a_scale_offsets`` (per-expert scale-block
+  offsets), ``src_info`` (per-row metadata that leads back to the source).
+  Parameters: ``clamp_activation`` (the clamped L1 activation).
+* flashinfer.megamoe.MegaMoESymmBuffer, Parameters: ``activation_clamp`` (the
+  SwiGLU clamp value, 10.0 by default); staging views: E4M3 x with FP32
+  [.., hidden // 128] scales, INT64 topk_idx, FP32 topk_weights.
+* flashinfer.fused_moe.MoEActivationPack: NVFP4 activations (packed uint8
+  [M, H/2] + float8_e4m3fn [M, H/16] block scales); ``FromLogits`` routing
+  with a ``routing_bias`` for bias-aware methods.
+* DistributedEPCombine, Args: ``router_weights`` scale each expert's
+  contribution; the combine reduces the expert rows back to their tokens.
+
+Readings taken where the pages are silent (each one is listed with its
+reasoning in the design notes of the repository):
+
+* Routing: select on score = fp32(logit + bias), descending, ties to the lower
+  expert index, NaN scores last; the weights are the softmax of the
+  *unbiased* logits over the chosen k.
+* Permutation: stable in the flat slot index; ``src_info[row] = t*k + j``.
+* ``topk_idx == -1`` is a skipped slot (the masked-id convention of
+  ``expert_ids``); duplicates within a token are independent slots.
+* Activation: h = min(g,c) * sigmoid(min(g,c)) * clamp(u,-c,c); c = +inf is
+  the textbook SwiGLU.  Gate rows are W13[e, :I], up rows are W13[e, I:].
+* Re-quant of h (computed in float64, then held in float32 as the kernel
+  holds it): NVFP4 per 16 values along I with an E4M3 block scale and the
+  per-expert FP32 ``c_input_scales`` G as the dequant multiplier; FP8 per 128
+  values with an FP32 scale amax/448; BF16 by round-to-nearest-even.  The
+  FP32 steps of the quantisers are fixed (see ``requant``) so that a code is
+  decided in the same precision on both sides.
+* NVFP4 GEMMs: the MMA sums products of (e2m1 x e4m3 block scale) operands,
+  then the per-expert scale (``gate_up_expert_scales`` or
+  ``down_expert_scales``) multiplies the sum.  FP8 GEMMs: every operand is
+  its E4M3 code times its FP32 block scale.
+* The output is BF16, rounded once from the float64 sum (via float32).
+"""
+
+import numpy as np
+
+from . import formats as F
+
+FORMATS = ("bf16", "fp8", "nvfp4")
+
+
+# ----------------------------------------------------------------------------
+# Routing (flashinfer.fused_moe.MoEActivationPack, routing_input_mode FromLogits)
+# ----------------------------------------------------------------------------
+
+def route(logits, bias, k):
+    """Top-k expert selection from router logits, bias used for selection only.
+
+    Returns (topk_idx int64 [M, k], topk_weights float64 [M, k]).
+    Slots are ordered by selection score, highest first.
+    """
+    l32 = np.asarray(logits, dtype=np.float32)
+    M, E = l32.shape
+    if not (1 <= k <= E):
+        raise ValueError("num_topk must be in [1, num_experts]")
+    b32 = np.zeros(E, np.float32) if bias is None else np.asarray(bias, np.float32)
+    score = l32 + b32[None, :]                      # one IEEE float32 add
+    nan = np.isnan(score)
+    key = np.where(nan, -np.inf, score).astype(np.float64)
+    ids = np.broadcast_to(np.arange(E), (M, E))
+    # lexsort: the last key is the primary one.
+    order = np.lexsort((ids, -key, nan), axis=-1)
+    topk_idx = order[:, :k].astype(np.int64)
+    chosen = np.take_along_axis(l32, topk_idx, axis=1).astype(np.float64)
+    z = np.exp(chosen - chosen.max(axis=1, keepdims=True))
+    topk_weights = z / z.sum(axis=1, keepdims=True)
+    return topk_idx, topk_weights
+
+
+# ----------------------------------------------------------------------------
+# Permutation (Struct_mega_ffn_ep_combine_send: expert_start_indices, expert_ids,
+# a_scale_offsets, src_info, num_active_experts)
+# ----------------------------------------------------------------------------
+
+def check_indices(topk_idx, num_experts):
+    idx = np.asarray(topk_idx)
+    if idx.size and (idx.min() < -1 or idx.max() >= num_experts):
+        raise ValueError("topk_idx out of range [-1, num_experts)")
+
+
+def permute(topk_idx, num_experts, scale_block_rows=128):
+    """Group the routed slots by expert, stably in the flat slot index.
+
+    Returns a dict of int64 arrays:
+      expert_counts [E]          valid slots per expert
+      expert_start_indices [E+1] exclusive prefix sum of the counts
+      src_info [R_valid]         flat slot index s = t*k + j of each row
+      slot_to_row [M*k]          row of each slot, -1 for a skipped slot
+      expert_ids [E]             active experts ascending, -1 padded
+      num_active                 number of experts with at least one slot
+      a_scale_offsets [E+1]      prefix sum of counts rounded up to 128 rows
+    """
+    check_indices(topk_idx, num_experts)
+    flat = np.asarray(topk_idx, dtype=np.int64).reshape(-1)
+    E = num_experts
+    counts = np.zeros(E, np.int64)
+    for e in range(E):
+        counts[e] = np.count_nonzero(flat == e)
+    starts = np.zeros(E + 1, np.int64)
+    starts[1:] = np.cumsum(counts)
+    src_info = np.zeros(int(starts[-1]), np.int64)
+    slot_to_row = np.full(flat.shape[0], -1, np.int64)
+    for e in range(E):
+        slots = np.nonzero(flat == e)[0]            # ascending slot index
+        rows = starts[e] + np.arange(slots.shape[0])
+        src_info[rows] = slots
+        slot_to_row[slots] = rows
+    active = np.nonzero(counts > 0)[0]
+    expert_ids = np.full(E, -1, np.int64)
+    expert_ids[: active.shape[0]] = active
+    padded = -(-counts // scale_block_rows) * scale_block_rows
+    a_scale_offsets = np.zeros(E + 1, np.int64)
+    a_scale_offsets[1:] = np.cumsum(padded)
+    return dict(expert_counts=counts, expert_start_indices=starts,
+                src_info=src_info, slot_to_row=slot_to_row,
+                expert_ids=expert_ids, num_active=int(active.shape[0]),
+                a_scale_offsets=a_scale_offsets)
+
+
+# ----------------------------------------------------------------------------
+# Decoding of activations and expert weights
+# ----------------------------------------------------------------------------
+
+def decode_x(fmt, x, x_scale, H, rows=None):
+    """Activations [M, H] -> float64.
+
+    fp8: E4M3 codes times the FP32 per-128 block scale of the token.
+    nvfp4: e2m1 codes times the E4M3 per-16 block scale (no global scale; the
+    per-expert L1 output scaling carries it).
+    """
+    x = np.asarray(x)
+    if rows is not None:
+        x = x[rows]
+        x_scale = None if x_scale is None else np.asarray(x_scale)[rows]
+    if fmt == "bf16":
+        return F.bf16_decode(x)
+    if fmt == "fp8":
+        s = np.asarray(x_scale, np.float32).astype(np.float64)
+        return F.e4m3_decode(x) * np.repeat(s, 128, axis=1)
+    if fmt == "nvfp4":
+        codes = F.fp4_unpack(x, H)
+        s = F.e4m3_decode(x_scale)
+        return F.e2m1_decode(codes) * np.repeat(s, 16, axis=1)
+    raise ValueError(fmt)
+
+
+def decode_weight(fmt, w, w_scale, e, n_rows, k_cols):
+    """Expert e's weight [n_rows, k_cols] (K-major, as stored) -> float64.
+
+    fp8 scales are per 128 x 128 block; nvfp4 scales per 1 x 16 block.
+    """
+    if fmt == "bf16":
+        return F.bf16_decode(np.asarray(w)[e])
+    if fmt == "fp8":
+        s = np.asarray(w_scale, np.float32)[e].astype(np.float64)
+        full = np.repeat(np.repeat(s, 128, axis=0), 128, axis=1)
+        return F.e4m3_decode(np.asarray(w)[e]) * full
+    if fmt == "nvfp4":
+        codes = F.fp4_unpack(np.asarray(w)[e], k_cols)
+        s = F.e4m3_decode(np.asarray(w_scale)[e])
+        return F.e2m1_decode(codes) * np.repeat(s, 16, axis=1)
+    raise ValueError(fmt)
+
+
+# ----------------------------------------------------------------------------
+# The expert FFN
+# ----------------------------------------------------------------------------
+
+def clamped_swiglu(g, u, clamp):
+    """h = min(g, c) * sigmoid(min(g, c)) * clamp(u, -c, c), in float64.
+
+    flashinfer.megamoe.MegaMoESymmBuffer, ``activation_clamp``: the SwiGLU
+    clamp value; Struct_mega_ffn_ep_combine_send, ``clamp_activation``.
+    The gate is clamped from above only, the up branch on both sides.
+    """
+    c = float(clamp)
+    g = np.minimum(g, c)
+    u = np.clip(u, -c, c)
+    return g / (1.0 + np.exp(-g)) * u
+
+
+def gate_up(fmt, xhat, w13hat, alpha1, I):
+    """L1: g = x^ W1^T, u = x^ W3^T with W1 = W13[:I], W3 = W13[I:]; NVFP4 scaled by alpha1."""
+    acc = xhat @ w13hat.T
+    if fmt == "nvfp4":
+        acc = acc * float(np.float32(alpha1))
+    return acc[:, :I], acc[:, I:]
+
+
+def requant(fmt, h32, G=None):
+    """Re-quantise the FP32 intermediate h [rows, I] to the L2 input format.
+
+    Returns dict(codes, scales, hhat) with hhat float64 = the dequantised value
+    the down GEMM sees (for NVFP4 without the global G, which the L2 output
+    scaling carries).
+
+    nvfp4, per block of 16 along I (all steps FP32, round to nearest):
+        sf   = e4m3_satfinite(amax / (6 * G))
+        q    = e2m1_satfinite(h * (1 / (sf * G)))      (q = 0 where sf == 0)
+    fp8, per block of 128 along I:
+        s    = amax / 448
+        q    = e4m3_satfinite(h * (1 / s))             (q = 0, s = 0 where amax == 0)
+    bf16:  q = bf16_rn(h)
+    """
+    h32 = np.asarray(h32, np.float32)
+    rows, I = h32.shape
+    if fmt == "bf16":
+        codes = F.bf16_encode(h32)
+        return dict(codes=codes, scales=None, hhat=F.bf16_decode(codes))
+    if fmt == "fp8":
+        blk = h32.reshape(rows, I // 128, 128)
+        amax = np.max(np.abs(blk), axis=2)                          # float32
+        s = (amax / np.float32(448.0)).astype(np.float32)
+        with np.errstate(divide="ignore"):
+            inv = (np.float32(1.0) / s).astype(np.float32)
+        v = (blk * inv[:, :, None]).astype(np.float32)
+        codes = F.e4m3_encode(v)
+        codes = np.where((s == 0)[:, :, None], np.uint8(0), codes).reshape(rows, I)
+        hhat = F.e4m3_decode(codes).reshape(rows, I // 128, 128) * s[:, :, None].astype(np.float64)
+        return dict(codes=codes, scales=s, hhat=hhat.reshape(rows, I))
+    if fmt == "nvfp4":
+        G32 = np.float32(G)
+        blk = h32.reshape(rows, I // 16, 16)
+        amax = np.max(np.abs(blk), axis=2)
+        denom = np.float32(np.float32(6.0) * G32)
+        sf_code = F.e4m3_encode((amax / denom).astype(np.float32))
+        sf = F.e4m3_decode(sf_code).astype(np.float32)
+        sg = (sf * G32).astype(np.float32)
+        with np.errstate(divide="ignore"):
+            inv = (np.float32(1.0) / sg).astype(np.float32)
+        v = (blk * inv[:, :, None]).astype(np.float32)
+        q = F.e2m1_encode(v)
+        q = np.where((sf == 0)[:, :, None], np.uint8(0), q).reshape(rows, I)
+        hhat = (F.e2m1_decode(q).reshape(rows, I // 16, 16)
+                * sf[:, :, None].astype(np.float64)).reshape(rows, I)
+        return dict(codes=F.fp4_pack(q), scales=sf_code, hhat=hhat)
+    raise ValueError(fmt)
+
+
+def dequant_intermediate(fmt, codes, scales, I):
+    """Decode re-quantised intermediate rows (as ``requant`` returns them) to float64."""
+    if fmt == "bf16":
+        return F.bf16_decode(codes)
+    if fmt == "fp8":
+        s = np.asarray(scales, np.float32).astype(np.float64)
+        return F.e4m3_decode(codes) * np.repeat(s, 128, axis=1)
+    if fmt == "nvfp4":
+        q = F.fp4_unpack(codes, I)
+        return F.e2m1_decode(q) * np.repeat(F.e4m3_decode(scales), 16, axis=1)
+    raise ValueError(fmt)
+
+
+def down(fmt, hhat, w2hat, alpha2):
+    """L2: y = h^ W2^T; NVFP4 scaled by alpha2 (``down_expert_scales``)."""
+    y = hhat @ w2hat.T
+    if fmt == "nvfp4":
+        y = y * float(np.float32(alpha2))
+    return y
+
+
+def _expert_scale(inputs, name, e):
+    arr = inputs.get(name)
+    return None if arr is None else np.asarray(arr, np.float32)[e]
+
+
+def moe_forward(problem, inputs, topk_idx, topk_weights, tokens=None,
+                keep_intermediate=False, hhat_override=None):
+    """The routed MoE FFN by its per-token definition.
+
+    problem: dict(hidden, intermediate_hidden, num_experts, num_topk,
+                  activation_clamp, format)
+    inputs:  dict(x, x_scale, w13, w13_scale, w2, w2_scale,
+                  gate_up_expert_scales, down_expert_scales, c_input_scales)
+    tokens:  optional subset of token indices (every quantity here is per
+             token, so a subset is computed exactly as in the full problem).
+    hhat_override: optional callable (e, t_array, j_array) -> float64 rows
+             that replaces the oracle's own re-quantised intermediate (used to
+             recompute L2 and the combine from another implementation's codes).
+
+    Returns dict(out_f64 [T, H], out_bf16 uint16 [T, H], and, when
+    keep_intermediate, per-slot h32 / codes / scales keyed by (t, j)).
+    """
+    fmt = problem["format"]
+    H = problem["hidden"]
+    I = problem["intermediate_hidden"]
+    E = problem["num_experts"]
+    clamp = problem.get("activation_clamp", 10.0)
+    idx = np.asarray(topk_idx, np.int64)
+    w = np.asarray(topk_weights, np.float32).astype(np.float64)
+    check_indices(idx, E)
+    tok = np.arange(idx.shape[0]) if tokens is None else np.asarray(tokens, np.int64)
+    idx_t = idx[tok]
+    w_t = w[tok]
+    xhat = decode_x(fmt, inputs["x"], inputs.get("x_scale"), H, rows=tok)
+    out = np.zeros((tok.shape[0], H), np.float64)
+    inter = {} if keep_intermediate else None
+    for e in range(E):
+        ti, sj = np.nonzero(idx_t == e)             # ascending (token, slot)
+        if ti.shape[0] == 0:
+            continue
+        w13hat = decode_weight(fmt, inputs["w13"], inputs.get("w13_scale"), e, 2 * I, H)
+        w2hat = decode_weight(fmt, inputs["w2"], inputs.get("w2_scale"), e, H, I)
+        g, u = gate_up(fmt, xhat[ti], w13hat, _expert_scale(inputs, "gate_up_expert_scales", e), I)
+        h32 = clamped_swiglu(g, u, clamp).astype(np.float32)
+        rq = requant(fmt, h32, _expert_scale(inputs, "c_input_scales", e))
+        hhat = rq["hhat"] if hhat_override is None else hhat_override(e, tok[ti], sj)
+        y = down(fmt, hhat, w2hat, _expert_scale(inputs, "down_expert_scales", e))
+        np.add.at(out, ti, w_t[ti, sj][:, None] * y)
+        if keep_intermediate:
+            for n in range(ti.shape[0]):
+                key = (int(tok[ti[n]]), int(sj[n]))
+                inter[key] = dict(expert=e, h32=h32[n],
+                                  codes=rq["codes"][n],
+                                  scales=None if rq["scales"] is None else rq["scales"][n])
+    res = dict(out_f64=out, out_bf16=F.bf16_encode(out.astype(np.float32)))
+    if keep_intermediate:
+        res["intermediate"] = inter
+    return res
