@@ -1,0 +1,461 @@
+#!/usr/bin/env python
+"""Throughput of the routed MoE FFN layer (moe_fused) on B200 GPUs.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one moe_fused call -- routing (when the workload routes from
+logits), permutation, the two grouped GEMMs with their fused epilogues and the
+BF16 finalise -- over one batch of synthetic inputs resident in HBM.  The L2
+is flushed (a 512 MiB write) before every timed step, outside the step's
+CUDA-event interval.  With N > 1 (one process per GPU, launched by torchrun)
+every rank runs its own batch with its own copy of the experts (data
+parallel, no collective on the data path; weak scaling); the time is the
+maximum over ranks.
+
+Rank 0 prints one JSON line.  `value` is routed tokens (token, expert slot
+pairs) per second summed over ranks; `e2e` is the same through the public API
+with the inputs copied from pinned host memory and the output read back every
+step; `roofline` is the dominant kernel's algorithmic throughput against the
+measured peak; `cpu_baseline` times the float64 CPU oracle on a bounded sample.
+`--impl reference` times that oracle alone (the reference arm).
+"""
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+DEFAULT_WORKLOAD = "fp8_block"
+FLUSH_BYTES = 512 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FMT_TENSOR_RATIO = {"bf16": 1.0, "fp8": 2.0, "nvfp4": 4.0}   # nominal dense ratio to bf16
+ELEM_BYTES = {"bf16": 2.0, "fp8": 1.0, "nvfp4": 0.5}
+BOUND = {"tiny_bf16": "hbm", "fp8_block": "hbm", "nvfp4_decode": "hbm",
+         "nvfp4_prefill": "tensor", "fp8_prefill_routed": "tensor"}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# --------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            cmd = ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits", "-lms", "200"]
+            if self.gpu_id is not None:
+                cmd += ["-i", str(self.gpu_id)]
+            self.proc = subprocess.Popen(cmd, stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), power=float(parts[3]),
+                                 hw=parts[5], hwt=parts[6], swt=parts[7], pcap=parts[8]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        reasons = set()
+        for r in rows:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in rows),
+                "sm_max_mhz": max(r["smax"] for r in rows),
+                "power_w_max": max(r["power"] for r in rows),
+                "samples": len(rows), "reasons": sorted(reasons)}
+
+
+# --------------------------------------------------------------------------- work model
+
+def work_model(p, num_active):
+    """Algorithmic FLOPs and bytes of the layer and of its two GEMM kernels."""
+    M, H, I, E, k = (p["num_tokens"], p["hidden"], p["intermediate_hidden"], p["num_experts"],
+                     p["num_topk"])
+    fmt = p["format"]
+    R = M * k
+    eb = ELEM_BYTES[fmt]
+    if fmt == "fp8":
+        w13_sc = (2 * I // 128) * (H // 128) * 4
+        w2_sc = (H // 128) * (I // 128) * 4
+        x_sc, h_sc = H // 128 * 4, I // 128 * 4
+    elif fmt == "nvfp4":
+        w13_sc, w2_sc = 2 * I * H // 16, H * I // 16
+        x_sc, h_sc = H // 16, I // 16
+    else:
+        w13_sc = w2_sc = x_sc = h_sc = 0
+    w13 = num_active * (2 * I * H * eb + w13_sc)
+    w2 = num_active * (H * I * eb + w2_sc)
+    x = M * (H * eb + x_sc)
+    out = M * H * 2
+    gemm1 = dict(flops=4.0 * R * H * I, bytes=w13 + R * (H * eb + x_sc) + R * (I * eb + h_sc))
+    gemm2 = dict(flops=2.0 * R * H * I, bytes=w2 + R * (I * eb + h_sc) + M * H * 4)
+    layer = dict(flops=6.0 * R * H * I, bytes=w13 + w2 + x + out + (M * E * 4 if p["routing"] == "logits" else 0))
+    return dict(gemm1=gemm1, gemm2=gemm2, layer=layer)
+
+
+# --------------------------------------------------------------------------- our arm
+
+def run_ours(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from mixture_experts_routed_03_b200 import api, layer, workloads
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    p = workloads.problem(args.workload)
+    d = workloads.make_inputs(p, seed=args.seed + rank, device=dev)
+    wts = {k: d.get(k) for k in ("w13", "w13_scale", "w2", "w2_scale", "gate_up_expert_scales",
+                                 "down_expert_scales", "c_input_scales")}
+    L = layer.MoELayer(p, wts, device=dev)
+    routed = p["routing"] == "logits"
+    M, k = p["num_tokens"], p["num_topk"]
+    R = M * k
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    out = torch.empty((M, p["hidden"]), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        if routed:
+            L.forward(d["x"], d["x_scale"], logits=d["logits"], bias=d["bias"], out=out)
+        else:
+            L.forward(d["x"], d["x_scale"], topk_idx=d["topk_idx"], topk_weights=d["topk_weights"], out=out)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+    L.check_status()
+
+    # ---- device-resident timed region
+    api.timing_enable(True, max(args.steps, 1))
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    gpu_id = None
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        gpu_id = local_rank
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(gpu_id) as clocks:
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    per_step = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    kern = api.timing_read()
+    api.timing_enable(False, 0)
+    L.check_status()
+    t_ms = sum(per_step)
+    launches = sum(n for _, n in kern.values())
+
+    # ---- end to end through the public API, inputs from pinned host memory
+    names = ["x"] + (["x_scale"] if d["x_scale"] is not None else []) + \
+            (["logits", "bias"] if routed else ["topk_idx", "topk_weights"])
+    host_in = {n: d[n].cpu().pin_memory() for n in names}
+    dev_in = {n: torch.empty_like(d[n]) for n in names}
+    host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = host_out.numel() * host_out.element_size()
+    e_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e_ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+
+    def e2e_step(i):
+        for n in names:
+            dev_in[n].copy_(host_in[n], non_blocking=True)
+        if routed:
+            L.forward(dev_in["x"], dev_in.get("x_scale"), logits=dev_in["logits"], bias=dev_in["bias"], out=out)
+        else:
+            L.forward(dev_in["x"], dev_in.get("x_scale"), topk_idx=dev_in["topk_idx"],
+                      topk_weights=dev_in["topk_weights"], out=out)
+        host_out.copy_(out, non_blocking=True)
+
+    for i in range(min(args.warmup, 3)):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    barrier()
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        e_starts[i].record(stream)
+        e2e_step(i)
+        e_ends[i].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = sum(s.elapsed_time(e) for s, e in zip(e_starts, e_ends))
+    L.check_status()
+
+    # ---- active experts of this batch (for the algorithmic byte counts)
+    if routed:
+        idx, _ = L.route(d["logits"], d["bias"])
+    else:
+        idx = d["topk_idx"]
+    num_active = int(torch.unique(idx[idx >= 0]).numel())
+
+    # ---- max over ranks
+    if world > 1:
+        tt = torch.tensor([t_ms, e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_ms, e2e_ms = float(tt[0]), float(tt[1])
+    return dict(p=p, t_ms=t_ms, per_step=per_step, kern=kern, launches=launches, e2e_ms=e2e_ms,
+                h2d=h2d, d2h=d2h, num_active=num_active, clocks=clocks.summary(), R=R, M=M,
+                host_inputs=(d, L) if rank == 0 else None)
+
+
+def cpu_baseline(p, d, seconds):
+    """The oracle, as it stands, on a bounded sample of this workload's tokens."""
+    import numpy as np
+    from mixture_experts_routed_03_b200 import workloads
+    from oracle import moe as O
+
+    host = workloads.to_numpy({k: v for k, v in d.items()})
+    if p["routing"] == "logits":
+        host["topk_idx"], host["topk_weights"] = O.route(host["logits"], host["bias"], p["num_topk"])
+        host["topk_weights"] = host["topk_weights"].astype(np.float32)
+    M, k = p["num_tokens"], p["num_topk"]
+    rng = np.random.default_rng(0)
+    order = rng.permutation(M)
+    n, done, t_total = 1, 0, 0.0
+    while True:
+        toks = np.sort(order[done: done + n])
+        if toks.size == 0:
+            break
+        t0 = time.perf_counter()
+        if p["routing"] == "logits":
+            O.route(host["logits"][toks], host["bias"], k)
+        O.moe_forward(p, host, host["topk_idx"], host["topk_weights"], tokens=toks)
+        dt = time.perf_counter() - t0
+        t_total += dt
+        done += toks.size
+        if t_total >= seconds or done >= M:
+            break
+        n = min(M - done, max(1, int(n * 2)))
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([int(i.get("num_threads", 1)) for i in threadpool_info()] or [1])
+    except Exception:
+        cores = os.cpu_count()
+    return dict(value=done * k / t_total, unit="routed_tokens/s", cores=cores, kind="oracle",
+                sample=f"{done} of {M} tokens ({done * k} routed slots), float64 numpy oracle incl. "
+                       f"per-expert weight decode, {t_total:.1f} s")
+
+
+def main_ours(args):
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        dist.init_process_group("nccl", device_id=torch.device("cuda", local_rank))
+    r = run_ours(args, rank, world, local_rank)
+    p = r["p"]
+    peaks, peak_src = load_peaks()
+    units = r["R"] * world * args.steps
+    value = units / (r["t_ms"] / 1e3)
+    e2e_value = units / (r["e2e_ms"] / 1e3)
+    wm = work_model(p, r["num_active"])
+    kern = r["kern"]
+    step_ms = r["t_ms"] / args.steps
+    # dominant kernel of the step
+    slot = max(("gemm1", "gemm2"), key=lambda s: kern[s][0])
+    k_ms = kern[slot][0] / max(kern[slot][1], 1)
+    bound = BOUND.get(args.workload, "hbm")
+    if bound == "tensor":
+        peak = peaks["bf16_tflops"] * FMT_TENSOR_RATIO[p["format"]]
+        achieved = wm[slot]["flops"] / (k_ms / 1e3) / 1e12
+        unit = "TFLOP/s"
+    else:
+        peak = peaks["hbm_gbs"]
+        achieved = wm[slot]["bytes"] / (k_ms / 1e3) / 1e9
+        unit = "GB/s"
+    total_k = sum(v[0] for v in kern.values()) or 1.0
+    line = {
+        "metric": "routed tokens/sec per MoE layer (moe_fused), 1 B200 per rank",
+        "value": value,
+        "unit": "routed_tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": step_ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": {"bf16": "bf16", "fp8": "e4m3+f32 scales (f32 accumulate)",
+                  "nvfp4": "e2m1+e4m3 scales (f32 accumulate)"}[p["format"]],
+        "data": "synthetic (seeded torch generators; random-init experts of the workload's shapes)",
+        "config": {"workload": args.workload, "num_tokens": p["num_tokens"], "hidden": p["hidden"],
+                   "intermediate_hidden": p["intermediate_hidden"], "num_experts": p["num_experts"],
+                   "num_topk": p["num_topk"], "format": p["format"], "routing": p["routing"],
+                   "active_experts": r["num_active"], "parallelism": f"dp{world} (replicas)",
+                   "l2": "flushed (512 MiB write) before every timed step, outside the step interval"},
+        "tokens_per_s": p["num_tokens"] * world * args.steps / (r["t_ms"] / 1e3),
+        "layer_tflops": wm["layer"]["flops"] / (step_ms / 1e3) / 1e12,
+        "layer_gbs": wm["layer"]["bytes"] / (step_ms / 1e3) / 1e9,
+        "roofline": {"kernel": slot, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                     "frac": achieved / peak, "traffic": None,
+                     "peak_source": f"{peak_src} ({'bf16 burst x nominal ' + p['format'] + ' ratio' if bound == 'tensor' else 'hbm copy'})",
+                     "kernel_ms": k_ms},
+        "kernels_ms": {s: v[0] / max(v[1], 1) for s, v in kern.items() if v[1]},
+        "kernel_share": {s: v[0] / total_k for s, v in kern.items() if v[1]},
+        "gpu_launches": r["launches"],
+        "e2e": {"value": e2e_value, "unit": "routed_tokens/s", "h2d_bytes_per_step": r["h2d"],
+                "d2h_bytes_per_step": r["d2h"], "ms_per_step": r["e2e_ms"] / args.steps},
+        "clocks": r["clocks"],
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        d, _ = r["host_inputs"]
+        line["cpu_baseline"] = cpu_baseline(p, d, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# --------------------------------------------------------------------------- reference arm
+
+def main_reference(args):
+    """The CPU oracle timed on the host cores, on this workload (rank 0 only)."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import numpy as np
+    import torch
+
+    from mixture_experts_routed_03_b200 import workloads
+    from oracle import moe as O
+
+    p = workloads.problem(args.workload)
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    host = workloads.to_numpy(workloads.make_inputs(p, seed=args.seed, device=dev))
+    M, k = p["num_tokens"], p["num_topk"]
+    if p["routing"] == "logits":
+        idx_all, w_all = O.route(host["logits"], host["bias"], k)
+    else:
+        idx_all, w_all = host["topk_idx"], host["topk_weights"]
+    rng = np.random.default_rng(0)
+    # size one step to about 4 s of oracle work
+    n = 1
+    while True:
+        toks = np.sort(rng.choice(M, size=n, replace=False))
+        t0 = time.perf_counter()
+        O.moe_forward(p, host, idx_all, w_all.astype(np.float32), tokens=toks)
+        dt = time.perf_counter() - t0
+        if dt >= 1.0 or n >= M:
+            break
+        n = min(M, n * 4)
+    n = int(min(M, max(1, n * 4.0 / max(dt, 1e-3))))
+    times = []
+    for i in range(args.warmup + args.steps):
+        toks = np.sort(rng.choice(M, size=n, replace=False))
+        t0 = time.perf_counter()
+        if p["routing"] == "logits":
+            O.route(host["logits"][toks], host["bias"], k)
+        O.moe_forward(p, host, idx_all, w_all.astype(np.float32), tokens=toks)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    t = sum(times)
+    value = n * k * args.steps / t
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([int(i.get("num_threads", 1)) for i in threadpool_info()] or [1])
+    except Exception:
+        cores = os.cpu_count()
+    sample = f"{n} of {M} tokens per step ({n * k} routed slots), float64 numpy oracle"
+    line = {
+        "impl": "reference",
+        "metric": "routed tokens/sec per MoE layer (moe_fused), 1 B200 per rank",
+        "value": value, "unit": "routed_tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded torch generators)",
+        "config": {"workload": args.workload, "num_tokens": M, "hidden": p["hidden"],
+                   "intermediate_hidden": p["intermediate_hidden"], "num_experts": p["num_experts"],
+                   "num_topk": k, "format": p["format"], "routing": p["routing"]},
+        "cpu_baseline": {"value": value, "unit": "routed_tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "routed_tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        main_reference(args)
+    else:
+        main_ours(args)
+
+
+if __name__ == "__main__":
+    main()

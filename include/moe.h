@@ -1,0 +1,276 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) routed Mixture-of-Experts FFN.
+ *
+ * One layer, on one GPU:
+ *
+ *   route    top-k expert selection from router logits, the bias used for the
+ *            selection only (flashinfer.fused_moe.MoEActivationPack,
+ *            routing_input_mode FromLogits)
+ *   permute  stable counting sort of the routed slots into expert-contiguous
+ *            rows (Struct_mega_ffn_ep_combine_send, Args: expert_start_indices,
+ *            expert_ids, a_scale_offsets, src_info, num_active_experts)
+ *   ffn      grouped gate_up GEMM with the clamped-SwiGLU + re-quant epilogue,
+ *            then the grouped down GEMM whose epilogue scatter-reduces every
+ *            row, weighted by its router weight, into the token-ordered output
+ *            (Struct_mega_ffn_ep_combine_send: gate_up_weight, down_weight,
+ *            gate_up_expert_scales, down_expert_scales, c_input_scales;
+ *            flashinfer.megamoe.MegaMoESymmBuffer: activation_clamp)
+ *   combine  the router-weighted reduction back to token order, finalised to
+ *            BF16 (DistributedEPCombine, Args: router_weights)
+ *   fused    all of the above on one stream, from one call
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every pointer argument named as a device buffer is a CUDA device address
+ *    on the current device.  The caller owns all memory, including the
+ *    workspace; the library allocates nothing per call and keeps no per-call
+ *    state on the host.
+ *  - `stream` is a cudaStream_t passed as void*; NULL is the legacy default
+ *    stream.  Every call except moe_read_status only enqueues work.
+ *  - Host-side validation runs before any launch.  A failed check returns an
+ *    error and launches nothing.  Unsupported combinations return
+ *    MOE_ERR_UNSUPPORTED; nothing falls back silently (EPConfig,
+ *    fuse_ffn_combine_send: incompatible options raise rather than degrade).
+ *  - Errors found on the device (an expert id >= num_experts or < -1, a
+ *    bounded wait that ran out) are recorded in a sticky status word at the
+ *    start of the workspace; the affected outputs are unspecified.  Read it
+ *    with moe_read_status.  No kernel traps or asserts.
+ *  - topk_idx == -1 marks a skipped slot (the -1 = masked convention of
+ *    expert_ids): it is not counted and contributes nothing.
+ *  - num_tokens == 0 is a no-op that returns MOE_OK.
+ *
+ * Layouts (row-major; K-major weights as the pages give them)
+ * ----------------------------------------------------------
+ *  M = num_tokens, H = hidden, I = intermediate_hidden, E = num_experts,
+ *  k = num_topk, R = M*k routed slots.
+ *
+ *  format BF16      x  bf16 [M, H]
+ *                   w13 bf16 [E, 2I, H]   rows [0, I) gate (W1), [I, 2I) up (W3)
+ *                   w2  bf16 [E, H, I]
+ *  format FP8       x  e4m3 [M, H], x_scale fp32 [M, H/128] (token-major)
+ *                   w13 e4m3 [E, 2I, H], w13_scale fp32 [E, 2I/128, H/128]
+ *                   w2  e4m3 [E, H, I],  w2_scale  fp32 [E, H/128, I/128]
+ *  format NVFP4     x  packed e2m1 uint8 [M, H/2] (element 2i in the low
+ *                   nibble), x_scale e4m3 [M, H/16]
+ *                   w13 uint8 [E, 2I, H/2], w13_scale e4m3 [E, 2I, H/16]
+ *                   w2  uint8 [E, H, I/2],  w2_scale  e4m3 [E, H, I/16]
+ *                   gate_up_expert_scales fp32 [E]  L1 output multiplier
+ *                   down_expert_scales    fp32 [E]  L2 output multiplier
+ *                   c_input_scales        fp32 [E]  re-quant dequant multiplier G
+ *  topk_idx int64 [M, k]; topk_weights fp32 [M, k]; output bf16 [M, H].
+ *
+ *  Geometry (flashinfer.megamoe.MegaMoESymmBuffer, Parameters): hidden is a
+ *  multiple of 256 and intermediate_hidden a multiple of 128; NVFP4 also needs
+ *  intermediate_hidden % 256 == 0 (one 128-byte K stage of the down GEMM).
+ *  1 <= num_topk <= num_experts <= 1024.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,  /* a null pointer, a bad size, a bad enum value */
+  MOE_ERR_UNSUPPORTED = 2,  /* a valid but unserved combination */
+  MOE_ERR_WORKSPACE = 3,    /* workspace smaller than moe_get_workspace_size */
+  MOE_ERR_CUDA = 4,         /* a CUDA runtime call failed (launch, attribute) */
+  MOE_ERR_BAD_INDEX = 5,    /* device: topk_idx outside [-1, num_experts) */
+  MOE_ERR_TIMEOUT = 6       /* device: a bounded wait gave up */
+} moe_status_t;
+
+typedef enum {
+  MOE_FMT_BF16 = 0,
+  MOE_FMT_FP8_E4M3_B128 = 1,  /* E4M3 with FP32 per-128 block scales */
+  MOE_FMT_NVFP4 = 2           /* e2m1 with E4M3 per-16 block scales + per-expert FP32 */
+} moe_format_t;
+
+/* The problem statement, after flashinfer.megamoe.MegaMoESymmBuffer
+ * (num_experts, num_topk, hidden, intermediate_hidden, activation_clamp,
+ * fast_math). */
+typedef struct {
+  int64_t num_tokens;           /* M >= 0 */
+  int32_t hidden;               /* H, multiple of 256 */
+  int32_t intermediate_hidden;  /* I, multiple of 128 */
+  int32_t num_experts;          /* E */
+  int32_t num_topk;             /* k */
+  float activation_clamp;       /* c of the clamped SwiGLU; +inf disables the clamp */
+  int32_t format;               /* moe_format_t */
+  int32_t fast_math;            /* nonzero: the SiLU uses the fast exponential */
+} moe_problem_t;
+
+/* Activations (device).  x_scale is NULL for BF16. */
+typedef struct {
+  const void* x;
+  const void* x_scale;
+} moe_act_t;
+
+/* Expert weights (device), in the layouts listed above.  For NVFP4 the
+ * w13_scale / w2_scale pointers must be the PREPARED scale tiles written by
+ * moe_prepare_weights (Struct_mega_ffn_ep_combine_send: "pre-permuted W13
+ * scale tile", "W2 scale tile"); the three per-expert FP32 arrays are used
+ * by NVFP4 only and may be NULL otherwise. */
+typedef struct {
+  const void* w13;
+  const void* w13_scale;
+  const void* w2;
+  const void* w2_scale;
+  const float* gate_up_expert_scales;
+  const float* down_expert_scales;
+  const float* c_input_scales;
+} moe_weights_t;
+
+/* The expert-contiguous layout that moe_permute writes (device int32 arrays,
+ * caller-owned):
+ *   expert_counts [E]          valid slots per expert
+ *   expert_start_indices [E+1] exclusive prefix sum of the counts; the last
+ *                              entry is the number of valid slots R'
+ *   src_info [R]               row r holds the flat slot s = t*k + j (rows
+ *                              >= R' are unspecified)
+ *   slot_to_row [R]            inverse of src_info; -1 for a skipped slot
+ *   expert_ids [E]             active experts ascending, then -1
+ *   num_active [1]             number of active experts
+ *   a_scale_offsets [E+1]      first padded scale row of each expert: the
+ *                              prefix sum of the counts rounded up to 128
+ *   tile_offsets [E+1]         prefix sum over the active experts of their
+ *                              128-row tile counts (the GEMM scheduler table)
+ * Within an expert the rows ascend in flat slot index (a stable sort). */
+typedef struct {
+  int32_t* expert_counts;
+  int32_t* expert_start_indices;
+  int32_t* src_info;
+  int32_t* slot_to_row;
+  int32_t* expert_ids;
+  int32_t* num_active;
+  int32_t* a_scale_offsets;
+  int32_t* tile_offsets;
+} moe_layout_t;
+
+/* moe_ffn output modes. */
+#define MOE_OUT_ACCUMULATE 0  /* out: fp32 [M, H], zeroed by the call, then += w * y per slot */
+#define MOE_OUT_STAGED 1      /* out: fp32 [R, H], row r = y of row r (no router weight) */
+
+/* moe_combine input modes. */
+#define MOE_IN_ACCUMULATED 0  /* in: fp32 [M, H] from MOE_OUT_ACCUMULATE; round to BF16 */
+#define MOE_IN_STAGED 1       /* in: fp32 [R, H] from MOE_OUT_STAGED; weighted gather */
+
+/* Sets the kernels' shared-memory attributes on `device` (the current device
+ * is not changed).  Call once per device before capturing any call into a
+ * CUDA graph (flashinfer.megamoe.MegaMoESymmBuffer, prewarm: build every
+ * module the fused op can select before capture).  Idempotent. */
+moe_status_t moe_init(int device);
+
+/* Bytes of device workspace that every call with this problem needs
+ * (256-byte aligned base required).  Valid for any num_tokens up to
+ * problem->num_tokens. */
+moe_status_t moe_get_workspace_size(const moe_problem_t* problem, size_t* bytes);
+
+/* Zeroes the workspace header (the sticky status word).  Call once after
+ * allocating a workspace and after moe_read_status reported an error. */
+moe_status_t moe_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
+
+/* Prepares NVFP4 weight scales for the kernels (one time, per weight set):
+ * rewrites w13_scale [E, 2I, H/16] and w2_scale [E, H, I/16] into 128-row x
+ * 4-block tiles (512 bytes each, the order the tensor-core scale copy reads).
+ * out_w13_scale and out_w2_scale are device buffers of the same byte sizes as
+ * the inputs.  BF16 and FP8 weights need no preparation (returns
+ * MOE_ERR_UNSUPPORTED for them). */
+moe_status_t moe_prepare_weights(const moe_problem_t* problem, const void* w13_scale,
+                                 const void* w2_scale, void* out_w13_scale,
+                                 void* out_w2_scale, void* stream);
+
+/* Routing from logits (flashinfer.fused_moe.MoEActivationPack, FromLogits).
+ * logits fp32 [M, E]; bias fp32 [E] or NULL (used for the selection only).
+ * Per token: score_e = logit_e + bias_e (one FP32 add); the k highest scores
+ * in descending order, ties to the lower expert index, NaN scores last;
+ * topk_weights = softmax over the chosen k of the UNBIASED logits.
+ * Writes topk_idx int64 [M, k] and topk_weights fp32 [M, k]. */
+moe_status_t moe_route(const moe_problem_t* problem, const float* logits, const float* bias,
+                       int64_t* topk_idx, float* topk_weights, void* stream);
+
+/* Expert-contiguous layout of the routed slots (see moe_layout_t).
+ * topk_idx int64 [M, k], values in [-1, E).  Out-of-range ids set
+ * MOE_ERR_BAD_INDEX in the workspace status word and are skipped. */
+moe_status_t moe_permute(const moe_problem_t* problem, const int64_t* topk_idx,
+                         const moe_layout_t* layout, void* workspace, size_t workspace_bytes,
+                         void* stream);
+
+/* The expert FFN over a layout from moe_permute: gathers the activation rows
+ * into expert order, runs the grouped gate_up GEMM with the clamped-SwiGLU
+ * and re-quant epilogue, then the grouped down GEMM whose epilogue either
+ * scatter-reduces w * y into `out` (MOE_OUT_ACCUMULATE) or stores y per row
+ * (MOE_OUT_STAGED).  topk_weights fp32 [M, k] (read in accumulate mode).
+ * If `intermediate` is not NULL the re-quantised intermediate is ALSO kept
+ * there for inspection: codes [R, I] (BF16: 2 bytes, FP8: 1, NVFP4: 1/2
+ * byte per element) at byte 0, followed at byte offset
+ * moe_intermediate_scale_offset() by its scales (FP8: fp32 [I/128][P];
+ * NVFP4: 512-byte tiles [P/128][I/64]; P = padded rows, a_scale_offsets[E]).
+ * Size it with moe_get_intermediate_size. */
+moe_status_t moe_ffn(const moe_problem_t* problem, const moe_act_t* act,
+                     const moe_weights_t* weights, const moe_layout_t* layout,
+                     const float* topk_weights, int32_t out_mode, void* out,
+                     void* intermediate, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes needed for moe_ffn's optional `intermediate` buffer, and the byte
+ * offset of its scales. */
+moe_status_t moe_get_intermediate_size(const moe_problem_t* problem, size_t* bytes,
+                                       size_t* scale_offset);
+
+/* Combine back to token order, BF16 out [M, H] (DistributedEPCombine).
+ * MOE_IN_ACCUMULATED: out = bf16_rn(in[t]).  MOE_IN_STAGED: out[t] =
+ * bf16_rn(sum_{j<k, slot valid} w[t,j] * in[slot_to_row[t*k+j]]), summed in
+ * FP32 in ascending j (deterministic).  `layout` and `topk_weights` are read
+ * in staged mode only. */
+moe_status_t moe_combine(const moe_problem_t* problem, const moe_layout_t* layout,
+                         const float* topk_weights, const void* in, int32_t in_mode,
+                         void* out_bf16, void* stream);
+
+/* The whole layer from one call: route (when `logits` is given, else the
+ * caller's topk_idx / topk_weights are used), permute, the FFN with the
+ * scatter-reduce epilogue, and the BF16 finalise, enqueued on `stream`
+ * without any host synchronisation.  Exactly one of (topk_idx and
+ * topk_weights) or logits must be non-NULL.  The routing chosen in-kernel
+ * is written into the workspace and is not returned. */
+moe_status_t moe_fused(const moe_problem_t* problem, const moe_act_t* act,
+                       const moe_weights_t* weights, const int64_t* topk_idx,
+                       const float* topk_weights, const float* logits, const float* bias,
+                       void* out_bf16, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Per-kernel timing, for measurement.  moe_timing_enable(1, max_calls)
+ * creates CUDA events for up to max_calls calls (once, on the current
+ * device); from then on every moe_fused / moe_ffn / moe_permute / moe_route /
+ * moe_combine call records an event pair around each kernel it launches, on
+ * the call's stream (the calls then must not be captured into a CUDA graph).
+ * moe_timing_read waits for the recorded events and returns, per kernel slot,
+ * the summed milliseconds and the number of launches timed, then starts a
+ * new window.  moe_timing_enable(0, 0) stops recording (events are kept).
+ * Slots: MOE_SLOT_* below. */
+#define MOE_SLOT_ROUTE 0
+#define MOE_SLOT_PERMUTE 1
+#define MOE_SLOT_GATHER 2
+#define MOE_SLOT_GEMM1 3
+#define MOE_SLOT_ZERO 4
+#define MOE_SLOT_GEMM2 5
+#define MOE_SLOT_FINALIZE 6
+#define MOE_SLOT_COMBINE 7
+#define MOE_NUM_SLOTS 8
+moe_status_t moe_timing_enable(int enable, int max_calls);
+moe_status_t moe_timing_read(float* ms /* [MOE_NUM_SLOTS] */, int* launches /* [MOE_NUM_SLOTS] */);
+
+/* Synchronises `stream` and returns the sticky device status recorded in the
+ * workspace (MOE_OK if no device error was seen). */
+moe_status_t moe_read_status(const void* workspace, void* stream);
+
+/* A static, human-readable name for a status code. */
+const char* moe_status_string(moe_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

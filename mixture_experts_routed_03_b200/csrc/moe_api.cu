@@ -1,0 +1,650 @@
+// moe_api.cu -- the C ABI of include/moe.h: argument validation, workspace
+// carving, TMA descriptor set-up and kernel launches.  No memory is
+// allocated here; every buffer is the caller's.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "aux_kernels.cuh"
+#include "gemm.cuh"
+
+using namespace moe;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// ---------------------------------------------------------------- validation
+int x_row_bytes(int fmt, int H) { return fmt == FMT_BF16 ? 2 * H : (fmt == FMT_FP8 ? H : H / 2); }
+int h_row_bytes(int fmt, int I) { return fmt == FMT_BF16 ? 2 * I : (fmt == FMT_FP8 ? I : I / 2); }
+
+moe_status_t check_problem(const moe_problem_t* p) {
+  if (!p) return MOE_ERR_INVALID_ARG;
+  if (p->num_tokens < 0) return MOE_ERR_INVALID_ARG;
+  if (p->format < MOE_FMT_BF16 || p->format > MOE_FMT_NVFP4) return MOE_ERR_INVALID_ARG;
+  if (p->hidden <= 0 || p->hidden % 256 != 0) return MOE_ERR_INVALID_ARG;
+  if (p->intermediate_hidden <= 0 || p->intermediate_hidden % 128 != 0) return MOE_ERR_INVALID_ARG;
+  if (p->num_experts < 1 || p->num_topk < 1 || p->num_topk > p->num_experts) return MOE_ERR_INVALID_ARG;
+  if (p->num_experts > 1024) return MOE_ERR_UNSUPPORTED;
+  if (std::isnan(p->activation_clamp) || !(p->activation_clamp > 0.0f)) return MOE_ERR_INVALID_ARG;
+  if (p->format == MOE_FMT_NVFP4 && p->intermediate_hidden % 256 != 0) return MOE_ERR_UNSUPPORTED;
+  const int64_t R = p->num_tokens * p->num_topk;
+  if (R > (int64_t(1) << 30)) return MOE_ERR_UNSUPPORTED;
+  // expert weight row indices are 32-bit in the TMA coordinates
+  if (int64_t(p->num_experts) * 2 * p->intermediate_hidden >= (int64_t(1) << 31) ||
+      int64_t(p->num_experts) * p->hidden >= (int64_t(1) << 31))
+    return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+// ---------------------------------------------------------------- workspace
+struct WsLayout {
+  int64_t M, R, P;   // tokens, routed rows, padded scale rows
+  int nblk;          // permute chunks
+  size_t header, route_idx, route_w;
+  size_t counts, starts, src_info, slot_to_row, expert_ids, num_active, a_scale_offsets, tile_offsets;
+  size_t block_counts;
+  size_t x_perm, x_sf;
+  size_t h, h_sf;
+  size_t acc;
+  size_t total;
+  size_t h_bytes, h_sf_bytes;
+};
+
+WsLayout make_layout(const moe_problem_t* p) {
+  WsLayout L{};
+  const int E = p->num_experts, H = p->hidden, I = p->intermediate_hidden, fmt = p->format;
+  L.M = p->num_tokens;
+  L.R = L.M * p->num_topk;
+  L.P = int64_t(align_up(size_t(L.R), 128)) + 128 * std::min<int64_t>(E, L.R);
+  L.nblk = int((L.R + kPermChunk - 1) / kPermChunk);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + std::max<size_t>(bytes, 1), kAlign);
+    return o;
+  };
+  L.header = take(sizeof(WsHeader));
+  L.route_idx = take(size_t(L.R) * 8);
+  L.route_w = take(size_t(L.R) * 4);
+  L.counts = take(size_t(E) * 4);
+  L.starts = take(size_t(E + 1) * 4);
+  L.src_info = take(size_t(L.R) * 4);
+  L.slot_to_row = take(size_t(L.R) * 4);
+  L.expert_ids = take(size_t(E) * 4);
+  L.num_active = take(4);
+  L.a_scale_offsets = take(size_t(E + 1) * 4);
+  L.tile_offsets = take(size_t(E + 1) * 4);
+  L.block_counts = take(size_t(L.nblk) * E * 4);
+  L.x_perm = take(size_t(L.R) * x_row_bytes(fmt, H));
+  L.x_sf = take(fmt == FMT_FP8 ? size_t(H / 128) * L.P * 4 : (fmt == FMT_NVFP4 ? size_t(L.P) * (H / 16) : 0));
+  L.h_bytes = size_t(L.R) * h_row_bytes(fmt, I);
+  L.h_sf_bytes = fmt == FMT_FP8 ? size_t(I / 128) * L.P * 4 : (fmt == FMT_NVFP4 ? size_t(L.P) * (I / 16) : 0);
+  L.h = take(L.h_bytes);
+  L.h_sf = take(L.h_sf_bytes);
+  L.acc = take(size_t(L.M) * H * 4);
+  L.total = off;
+  return L;
+}
+
+// ---------------------------------------------------------------- TMA maps
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                              const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                              CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                              CUtensorMapFloatOOBfill);
+
+EncodeFn get_encode() {
+  static EncodeFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeFn>(ptr);
+  });
+  return fn;
+}
+
+// 2-D byte tensor [rows][row_bytes], boxes of 128 bytes x box_rows, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows, uint32_t box_rows) {
+  EncodeFn enc = get_encode();
+  if (!enc) return false;
+  if ((reinterpret_cast<uintptr_t>(base) & 15) || (row_bytes & 15) || rows == 0) return false;
+  cuuint64_t dims[2] = {row_bytes, rows};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {128, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------- timing
+struct Timing {
+  bool on = false;
+  int cap = 0;            // event pairs per slot
+  int used[MOE_NUM_SLOTS] = {0};
+  cudaEvent_t* ev = nullptr;  // [MOE_NUM_SLOTS][cap][2]
+  std::mutex mu;
+};
+Timing g_tim;
+
+// Records the start event of `slot` on `st`; returns the pair index or -1.
+int tim_begin(int slot, cudaStream_t st) {
+  if (!g_tim.on) return -1;
+  std::lock_guard<std::mutex> lk(g_tim.mu);
+  const int i = g_tim.used[slot];
+  if (i >= g_tim.cap) return -1;
+  g_tim.used[slot] = i + 1;
+  cudaEventRecord(g_tim.ev[(size_t(slot) * g_tim.cap + i) * 2], st);
+  return i;
+}
+
+void tim_end(int slot, int i, cudaStream_t st) {
+  if (i < 0) return;
+  cudaEventRecord(g_tim.ev[(size_t(slot) * g_tim.cap + i) * 2 + 1], st);
+}
+
+struct TimScope {
+  int slot, i;
+  cudaStream_t st;
+  TimScope(int s, cudaStream_t stream) : slot(s), i(tim_begin(s, stream)), st(stream) {}
+  ~TimScope() { tim_end(slot, i, st); }
+};
+
+// ---------------------------------------------------------------- launches
+int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+template <int FMT, int EPI>
+cudaError_t set_gemm_attr() {
+  return cudaFuncSetAttribute(moe_gemm_kernel<FMT, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              GemmCfg<FMT>::kSmemBytes);
+}
+
+template <int FMT>
+cudaError_t set_attrs_fmt() {
+  cudaError_t e;
+  if ((e = set_gemm_attr<FMT, EPI_L1>()) != cudaSuccess) return e;
+  if ((e = set_gemm_attr<FMT, EPI_L2_ACC>()) != cudaSuccess) return e;
+  return set_gemm_attr<FMT, EPI_L2_STAGED>();
+}
+
+cudaError_t set_all_attrs() {
+  cudaError_t e;
+  if ((e = set_attrs_fmt<FMT_BF16>()) != cudaSuccess) return e;
+  if ((e = set_attrs_fmt<FMT_FP8>()) != cudaSuccess) return e;
+  return set_attrs_fmt<FMT_NVFP4>();
+}
+
+bool ensure_init() {
+  static int inited_mask[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (dev >= 0 && dev < 64 && inited_mask[dev]) return true;
+  if (set_all_attrs() != cudaSuccess) return false;
+  if (dev >= 0 && dev < 64) inited_mask[dev] = 1;
+  return true;
+}
+
+template <int FMT, int EPI>
+cudaError_t launch_gemm(const GemmArgs& a, const CUtensorMap& ta, const CUtensorMap& tb, int grid,
+                        cudaStream_t st) {
+  moe_gemm_kernel<FMT, EPI><<<grid, GemmCfg<FMT>::kThreads, GemmCfg<FMT>::kSmemBytes, st>>>(a, ta, tb);
+  return cudaGetLastError();
+}
+
+template <int EPI>
+cudaError_t launch_gemm_fmt(int fmt, const GemmArgs& a, const CUtensorMap& ta, const CUtensorMap& tb,
+                            int grid, cudaStream_t st) {
+  switch (fmt) {
+    case FMT_BF16: return launch_gemm<FMT_BF16, EPI>(a, ta, tb, grid, st);
+    case FMT_FP8: return launch_gemm<FMT_FP8, EPI>(a, ta, tb, grid, st);
+    default: return launch_gemm<FMT_NVFP4, EPI>(a, ta, tb, grid, st);
+  }
+}
+
+int grid_for(int64_t n, int threads, int cap = 148 * 16) {
+  int64_t g = (n + threads - 1) / threads;
+  if (g < 1) g = 1;
+  if (g > cap) g = cap;
+  return int(g);
+}
+
+cudaError_t launch_route(const moe_problem_t* p, const float* logits, const float* bias, int64_t* idx,
+                         float* w, cudaStream_t st) {
+  const int E = p->num_experts;
+  const int64_t M = p->num_tokens;
+  const int grid = int((M * 32 + 255) / 256);
+  const int per = (E + 31) / 32;
+  TimScope ts(MOE_SLOT_ROUTE, st);
+#define MOE_ROUTE(PER) route_kernel<PER><<<grid, 256, 0, st>>>(logits, bias, M, E, p->num_topk, idx, w)
+  if (per <= 1) MOE_ROUTE(1);
+  else if (per <= 2) MOE_ROUTE(2);
+  else if (per <= 4) MOE_ROUTE(4);
+  else if (per <= 8) MOE_ROUTE(8);
+  else if (per <= 16) MOE_ROUTE(16);
+  else MOE_ROUTE(32);
+#undef MOE_ROUTE
+  return cudaGetLastError();
+}
+
+cudaError_t launch_permute(const moe_problem_t* p, const int64_t* idx, const PermOut& o, int* block_counts,
+                           int nblk, int* status, cudaStream_t st) {
+  const int E = p->num_experts;
+  const int64_t R = p->num_tokens * p->num_topk;
+  TimScope ts(MOE_SLOT_PERMUTE, st);
+  perm_count_kernel<<<nblk, 256, E * sizeof(int), st>>>(idx, R, E, block_counts, status);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  perm_scatter_kernel<<<nblk, 256, (5 * E + 3) * sizeof(int), st>>>(idx, R, E, nblk, block_counts, o);
+  return cudaGetLastError();
+}
+
+struct FfnBuffers {
+  // layout
+  const int *counts, *starts, *src_info, *slot_to_row, *expert_ids, *num_active, *a_scale_offsets, *tile_offsets;
+  // scratch
+  uint8_t *x_perm, *x_sf, *h, *h_sf;
+  int64_t P;
+  int* status;
+};
+
+moe_status_t run_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_weights_t* w,
+                     const FfnBuffers& b, const float* topk_weights,
+                     int out_mode, float* out, cudaStream_t st) {
+  const int fmt = p->format, H = p->hidden, I = p->intermediate_hidden, E = p->num_experts, k = p->num_topk;
+  const int64_t M = p->num_tokens, R = M * k;
+  const int nsm = sm_count();
+
+  // gather
+  GatherArgs g{};
+  g.x = static_cast<const uint8_t*>(act->x);
+  g.x_scale = act->x_scale;
+  g.src_info = b.src_info;
+  g.starts = b.starts;
+  g.a_scale_offsets = b.a_scale_offsets;
+  g.R = R;
+  g.row_bytes = x_row_bytes(fmt, H);
+  g.topk = k;
+  g.H = H;
+  g.fmt = fmt;
+  g.x_perm = b.x_perm;
+  g.sa_t = reinterpret_cast<float*>(b.x_sf);
+  g.sfa = b.x_sf;
+  g.ld = int(b.P);
+  {
+    TimScope ts(MOE_SLOT_GATHER, st);
+    gather_kernel<<<grid_for(R * 32, 256, 1 << 30), 256, 0, st>>>(g, E);
+  }
+  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+
+  // L1: gate_up
+  CUtensorMap ta{}, tb{};
+  const uint32_t l1_box = (fmt == FMT_FP8) ? 64 : 128;
+  if (!make_map(&ta, b.x_perm, x_row_bytes(fmt, H), uint64_t(R), 128)) return MOE_ERR_CUDA;
+  if (!make_map(&tb, w->w13, x_row_bytes(fmt, H), uint64_t(E) * 2 * I, l1_box)) return MOE_ERR_CUDA;
+  GemmArgs a{};
+  a.k_stages = x_row_bytes(fmt, H) / 128;
+  a.w_rows = 2 * I;
+  a.n_tiles = I / 128;
+  a.I = I;
+  a.H = H;
+  a.topk = k;
+  a.clamp = p->activation_clamp;
+  a.fast_math = p->fast_math;
+  a.expert_ids = b.expert_ids;
+  a.num_active = b.num_active;
+  a.starts = b.starts;
+  a.a_scale_offsets = b.a_scale_offsets;
+  a.tile_offsets = b.tile_offsets;
+  a.src_info = b.src_info;
+  a.topk_weights = topk_weights;
+  a.sfa = b.x_sf;
+  a.sfa_kc = H / 64;
+  a.sfb = static_cast<const uint8_t*>(w->w13_scale);
+  a.sfb_kc = H / 64;
+  a.sa_t = reinterpret_cast<const float*>(b.x_sf);
+  a.sa_ld = int(b.P);
+  a.sb = static_cast<const float*>(w->w13_scale);
+  a.sb_nb = 2 * I / 128;
+  a.sb_kb = H / 128;
+  a.alpha = w->gate_up_expert_scales;
+  a.c_in = w->c_input_scales;
+  a.h_out = b.h;
+  a.h_row_bytes = h_row_bytes(fmt, I);
+  a.h_sf = b.h_sf;
+  a.h_sf_kc = I / 64;
+  a.h_scale_t = reinterpret_cast<float*>(b.h_sf);
+  a.h_scale_ld = int(b.P);
+  a.status = b.status;
+  const int64_t mtiles_bound = (R + 127) / 128 + std::min<int64_t>(E, R);
+  int grid1 = int(std::min<int64_t>(nsm, mtiles_bound * a.n_tiles));
+  {
+    TimScope ts(MOE_SLOT_GEMM1, st);
+    if (launch_gemm_fmt<EPI_L1>(fmt, a, ta, tb, std::max(grid1, 1), st) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+
+  // L2: down
+  if (out_mode == MOE_OUT_ACCUMULATE) {
+    TimScope ts(MOE_SLOT_ZERO, st);
+    zero_kernel<<<grid_for(M * H / 4, 256), 256, 0, st>>>(reinterpret_cast<float4*>(out), M * H / 4);
+    if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  CUtensorMap ta2{}, tb2{};
+  if (!make_map(&ta2, b.h, h_row_bytes(fmt, I), uint64_t(R), 128)) return MOE_ERR_CUDA;
+  if (!make_map(&tb2, w->w2, h_row_bytes(fmt, I), uint64_t(E) * H, 256)) return MOE_ERR_CUDA;
+  GemmArgs a2 = a;
+  a2.k_stages = h_row_bytes(fmt, I) / 128;
+  a2.w_rows = H;
+  a2.n_tiles = H / 256;
+  a2.sfa = b.h_sf;
+  a2.sfa_kc = I / 64;
+  a2.sfb = static_cast<const uint8_t*>(w->w2_scale);
+  a2.sfb_kc = I / 64;
+  a2.sa_t = reinterpret_cast<const float*>(b.h_sf);
+  a2.sb = static_cast<const float*>(w->w2_scale);
+  a2.sb_nb = H / 128;
+  a2.sb_kb = I / 128;
+  a2.alpha = w->down_expert_scales;
+  a2.out = out;
+  int grid2 = int(std::min<int64_t>(nsm, mtiles_bound * a2.n_tiles));
+  TimScope ts2(MOE_SLOT_GEMM2, st);
+  cudaError_t e = (out_mode == MOE_OUT_ACCUMULATE)
+                      ? launch_gemm_fmt<EPI_L2_ACC>(fmt, a2, ta2, tb2, std::max(grid2, 1), st)
+                      : launch_gemm_fmt<EPI_L2_STAGED>(fmt, a2, ta2, tb2, std::max(grid2, 1), st);
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; }
+
+moe_status_t check_act_weights(const moe_problem_t* p, const moe_act_t* act, const moe_weights_t* w) {
+  if (!act || !w || !act->x || !w->w13 || !w->w2) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(act->x) || !aligned16(w->w13) || !aligned16(w->w2)) return MOE_ERR_INVALID_ARG;
+  if (p->format != MOE_FMT_BF16 && (!act->x_scale || !w->w13_scale || !w->w2_scale)) return MOE_ERR_INVALID_ARG;
+  if (p->format == MOE_FMT_NVFP4 &&
+      (!w->gate_up_expert_scales || !w->down_expert_scales || !w->c_input_scales))
+    return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+bool layout_ok(const moe_layout_t* l) {
+  return l && l->expert_counts && l->expert_start_indices && l->src_info && l->slot_to_row && l->expert_ids &&
+         l->num_active && l->a_scale_offsets && l->tile_offsets;
+}
+
+}  // namespace
+
+// =============================================================== C ABI
+extern "C" {
+
+const char* moe_status_string(moe_status_t s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_BAD_INDEX: return "MOE_ERR_BAD_INDEX";
+    case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT";
+  }
+  return "MOE_ERR_UNKNOWN";
+}
+
+moe_status_t moe_init(int device) {
+  int prev = 0;
+  if (cudaGetDevice(&prev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaSetDevice(device) != cudaSuccess) return MOE_ERR_CUDA;
+  const bool ok = ensure_init() && get_encode() != nullptr;
+  cudaSetDevice(prev);
+  return ok ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status_t moe_get_workspace_size(const moe_problem_t* p, size_t* bytes) {
+  moe_status_t s = check_problem(p);
+  if (s != MOE_OK) return s;
+  if (!bytes) return MOE_ERR_INVALID_ARG;
+  *bytes = make_layout(p).total;
+  return MOE_OK;
+}
+
+moe_status_t moe_get_intermediate_size(const moe_problem_t* p, size_t* bytes, size_t* scale_offset) {
+  moe_status_t s = check_problem(p);
+  if (s != MOE_OK) return s;
+  if (!bytes || !scale_offset) return MOE_ERR_INVALID_ARG;
+  const WsLayout L = make_layout(p);
+  *scale_offset = align_up(std::max<size_t>(L.h_bytes, 1), kAlign);
+  *bytes = *scale_offset + align_up(std::max<size_t>(L.h_sf_bytes, 1), kAlign);
+  return MOE_OK;
+}
+
+moe_status_t moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+  if (!ws || ws_bytes < sizeof(WsHeader)) return MOE_ERR_INVALID_ARG;
+  zero_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<float4*>(ws),
+                                                               int64_t(sizeof(WsHeader) / 16));
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status_t moe_prepare_weights(const moe_problem_t* p, const void* w13_scale, const void* w2_scale,
+                                 void* out_w13_scale, void* out_w2_scale, void* stream) {
+  moe_status_t s = check_problem(p);
+  if (s != MOE_OK) return s;
+  if (p->format != MOE_FMT_NVFP4) return MOE_ERR_UNSUPPORTED;
+  if (!w13_scale || !w2_scale || !out_w13_scale || !out_w2_scale) return MOE_ERR_INVALID_ARG;
+  if (!ensure_init()) return MOE_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t E = p->num_experts, H = p->hidden, I = p->intermediate_hidden;
+  const int64_t n13 = E * 2 * I * (H / 16), n2 = E * H * (I / 16);
+  prepare_sf_kernel<<<grid_for(n13, 256), 256, 0, st>>>(static_cast<const uint8_t*>(w13_scale),
+                                                       static_cast<uint8_t*>(out_w13_scale), E * 2 * I,
+                                                       int(H / 16));
+  prepare_sf_kernel<<<grid_for(n2, 256), 256, 0, st>>>(static_cast<const uint8_t*>(w2_scale),
+                                                      static_cast<uint8_t*>(out_w2_scale), E * H,
+                                                      int(I / 16));
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status_t moe_route(const moe_problem_t* p, const float* logits, const float* bias, int64_t* topk_idx,
+                       float* topk_weights, void* stream) {
+  moe_status_t s = check_problem(p);
+  if (s != MOE_OK) return s;
+  if (p->num_topk > 32) return MOE_ERR_UNSUPPORTED;
+  if (p->num_tokens == 0) return MOE_OK;
+  if (!logits || !topk_idx || !topk_weights) return MOE_ERR_INVALID_ARG;
+  return launch_route(p, logits, bias, topk_idx, topk_weights, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
+}
+
+moe_status_t moe_permute(const moe_problem_t* p, const int64_t* topk_idx, const moe_layout_t* layout, void* ws,
+                         size_t ws_bytes, void* stream) {
+  moe_status_t s = check_problem(p);
+  if (s != MOE_OK) return s;
+  if (p->num_tokens == 0) return MOE_OK;
+  if (!topk_idx || !layout_ok(layout) || !ws) return MOE_ERR_INVALID_ARG;
+  const WsLayout L = make_layout(p);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  PermOut o{layout->expert_counts, layout->expert_start_indices, layout->src_info, layout->slot_to_row,
+            layout->expert_ids,    layout->num_active,           layout->a_scale_offsets, layout->tile_offsets};
+  return launch_permute(p, topk_idx, o, reinterpret_cast<int*>(base + L.block_counts), L.nblk,
+                        reinterpret_cast<int*>(base + L.header), static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
+}
+
+moe_status_t moe_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_weights_t* w,
+                     const moe_layout_t* layout, const float* topk_weights, int32_t out_mode, void* out,
+                     void* intermediate, void* ws, size_t ws_bytes, void* stream) {
+  moe_status_t s = check_problem(p);
+  if (s != MOE_OK) return s;
+  if (out_mode != MOE_OUT_ACCUMULATE && out_mode != MOE_OUT_STAGED) return MOE_ERR_INVALID_ARG;
+  if (p->num_tokens == 0) return MOE_OK;
+  if ((s = check_act_weights(p, act, w)) != MOE_OK) return s;
+  if (!layout_ok(layout) || !out || !ws || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  if (out_mode == MOE_OUT_ACCUMULATE && !topk_weights) return MOE_ERR_INVALID_ARG;
+  const WsLayout L = make_layout(p);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  if (!ensure_init()) return MOE_ERR_CUDA;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  FfnBuffers b{};
+  b.counts = layout->expert_counts;
+  b.starts = layout->expert_start_indices;
+  b.src_info = layout->src_info;
+  b.slot_to_row = layout->slot_to_row;
+  b.expert_ids = layout->expert_ids;
+  b.num_active = layout->num_active;
+  b.a_scale_offsets = layout->a_scale_offsets;
+  b.tile_offsets = layout->tile_offsets;
+  b.x_perm = base + L.x_perm;
+  b.x_sf = base + L.x_sf;
+  size_t so = 0, isz = 0;
+  moe_get_intermediate_size(p, &isz, &so);
+  b.h = intermediate ? static_cast<uint8_t*>(intermediate) : base + L.h;
+  b.h_sf = intermediate ? static_cast<uint8_t*>(intermediate) + so : base + L.h_sf;
+  b.P = L.P;
+  b.status = reinterpret_cast<int*>(base + L.header);
+  return run_ffn(p, act, w, b, topk_weights, out_mode, static_cast<float*>(out),
+                 static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_combine(const moe_problem_t* p, const moe_layout_t* layout, const float* topk_weights,
+                         const void* in, int32_t in_mode, void* out_bf16, void* stream) {
+  moe_status_t s = check_problem(p);
+  if (s != MOE_OK) return s;
+  if (in_mode != MOE_IN_ACCUMULATED && in_mode != MOE_IN_STAGED) return MOE_ERR_INVALID_ARG;
+  if (p->num_tokens == 0) return MOE_OK;
+  if (!in || !out_bf16 || !aligned16(in) || !aligned16(out_bf16)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t M = p->num_tokens, H = p->hidden;
+  TimScope ts(in_mode == MOE_IN_ACCUMULATED ? MOE_SLOT_FINALIZE : MOE_SLOT_COMBINE, st);
+  if (in_mode == MOE_IN_ACCUMULATED) {
+    finalize_kernel<<<grid_for(M * H / 8, 256), 256, 0, st>>>(static_cast<const float4*>(in),
+                                                             static_cast<uint4*>(out_bf16), M * H / 8);
+  } else {
+    if (!layout || !layout->slot_to_row || !topk_weights) return MOE_ERR_INVALID_ARG;
+    combine_staged_kernel<<<grid_for(M * H / 8, 256), 256, 0, st>>>(
+        static_cast<const float*>(in), layout->slot_to_row, topk_weights, M, int(H), p->num_topk,
+        static_cast<uint4*>(out_bf16));
+  }
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status_t moe_fused(const moe_problem_t* p, const moe_act_t* act, const moe_weights_t* w,
+                       const int64_t* topk_idx, const float* topk_weights, const float* logits,
+                       const float* bias, void* out_bf16, void* ws, size_t ws_bytes, void* stream) {
+  moe_status_t s = check_problem(p);
+  if (s != MOE_OK) return s;
+  if (p->num_tokens == 0) return MOE_OK;
+  if ((s = check_act_weights(p, act, w)) != MOE_OK) return s;
+  const bool pre = topk_idx != nullptr && topk_weights != nullptr;
+  const bool from_logits = logits != nullptr;
+  if (pre == from_logits || (!pre && (topk_idx || topk_weights))) return MOE_ERR_INVALID_ARG;
+  if (from_logits && p->num_topk > 32) return MOE_ERR_UNSUPPORTED;
+  if (!out_bf16 || !aligned16(out_bf16) || !ws) return MOE_ERR_INVALID_ARG;
+  const WsLayout L = make_layout(p);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  if (!ensure_init()) return MOE_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  int* status = reinterpret_cast<int*>(base + L.header);
+  const int64_t* idx = topk_idx;
+  const float* wts = topk_weights;
+  if (from_logits) {
+    int64_t* ridx = reinterpret_cast<int64_t*>(base + L.route_idx);
+    float* rw = reinterpret_cast<float*>(base + L.route_w);
+    if (launch_route(p, logits, bias, ridx, rw, st) != cudaSuccess) return MOE_ERR_CUDA;
+    idx = ridx;
+    wts = rw;
+  }
+  PermOut o{reinterpret_cast<int*>(base + L.counts),     reinterpret_cast<int*>(base + L.starts),
+            reinterpret_cast<int*>(base + L.src_info),   reinterpret_cast<int*>(base + L.slot_to_row),
+            reinterpret_cast<int*>(base + L.expert_ids), reinterpret_cast<int*>(base + L.num_active),
+            reinterpret_cast<int*>(base + L.a_scale_offsets), reinterpret_cast<int*>(base + L.tile_offsets)};
+  if (launch_permute(p, idx, o, reinterpret_cast<int*>(base + L.block_counts), L.nblk, status, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  FfnBuffers b{};
+  b.counts = o.expert_counts;
+  b.starts = o.expert_start_indices;
+  b.src_info = o.src_info;
+  b.slot_to_row = o.slot_to_row;
+  b.expert_ids = o.expert_ids;
+  b.num_active = o.num_active;
+  b.a_scale_offsets = o.a_scale_offsets;
+  b.tile_offsets = o.tile_offsets;
+  b.x_perm = base + L.x_perm;
+  b.x_sf = base + L.x_sf;
+  b.h = base + L.h;
+  b.h_sf = base + L.h_sf;
+  b.P = L.P;
+  b.status = status;
+  float* acc = reinterpret_cast<float*>(base + L.acc);
+  if ((s = run_ffn(p, act, w, b, wts, MOE_OUT_ACCUMULATE, acc, st)) != MOE_OK) return s;
+  const int64_t M = p->num_tokens, H = p->hidden;
+  TimScope ts(MOE_SLOT_FINALIZE, st);
+  finalize_kernel<<<grid_for(M * H / 8, 256), 256, 0, st>>>(reinterpret_cast<const float4*>(acc),
+                                                           static_cast<uint4*>(out_bf16), M * H / 8);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status_t moe_timing_enable(int enable, int max_calls) {
+  std::lock_guard<std::mutex> lk(g_tim.mu);
+  if (!enable) {
+    g_tim.on = false;
+    return MOE_OK;
+  }
+  if (max_calls < 1) return MOE_ERR_INVALID_ARG;
+  if (!g_tim.ev || g_tim.cap < max_calls) {
+    if (g_tim.ev) {
+      for (int i = 0; i < MOE_NUM_SLOTS * g_tim.cap * 2; ++i) cudaEventDestroy(g_tim.ev[i]);
+      delete[] g_tim.ev;
+      g_tim.ev = nullptr;
+    }
+    g_tim.ev = new cudaEvent_t[size_t(MOE_NUM_SLOTS) * max_calls * 2];
+    for (int i = 0; i < MOE_NUM_SLOTS * max_calls * 2; ++i)
+      if (cudaEventCreate(&g_tim.ev[i]) != cudaSuccess) return MOE_ERR_CUDA;
+    g_tim.cap = max_calls;
+  }
+  for (int s = 0; s < MOE_NUM_SLOTS; ++s) g_tim.used[s] = 0;
+  g_tim.on = true;
+  return MOE_OK;
+}
+
+moe_status_t moe_timing_read(float* ms, int* launches) {
+  if (!ms || !launches) return MOE_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_tim.mu);
+  for (int s = 0; s < MOE_NUM_SLOTS; ++s) {
+    ms[s] = 0.0f;
+    launches[s] = g_tim.used[s];
+    for (int i = 0; i < g_tim.used[s]; ++i) {
+      cudaEvent_t a = g_tim.ev[(size_t(s) * g_tim.cap + i) * 2];
+      cudaEvent_t b = g_tim.ev[(size_t(s) * g_tim.cap + i) * 2 + 1];
+      if (cudaEventSynchronize(b) != cudaSuccess) return MOE_ERR_CUDA;
+      float t = 0.0f;
+      if (cudaEventElapsedTime(&t, a, b) != cudaSuccess) return MOE_ERR_CUDA;
+      ms[s] += t;
+    }
+    g_tim.used[s] = 0;
+  }
+  return MOE_OK;
+}
+
+moe_status_t moe_read_status(const void* ws, void* stream) {
+  if (!ws) return MOE_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  return static_cast<moe_status_t>(v);
+}
+
+}  // extern "C"
