@@ -25,7 +25,6 @@ import json
 import math
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -52,7 +51,18 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--set", action="append", default=[], metavar="KEY=VALUE",
+                    help="override a workload field (a smaller case for profiling)")
     return ap.parse_args()
+
+
+def workload(args):
+    from mixture_experts_routed_03_b200 import workloads
+    over = {}
+    for kv in args.set:
+        k, v = kv.split("=", 1)
+        over[k] = type(workloads.WORKLOADS[args.workload].get(k, 0))(v) if k in workloads.WORKLOADS[args.workload] else float(v)
+    return workloads.problem(args.workload, **over)
 
 
 def load_peaks():
@@ -68,61 +78,66 @@ def load_peaks():
 # --------------------------------------------------------------------------- clocks
 
 class ClockSampler:
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and throttle reasons of one GPU, sampled through NVML while
+    the timed steps execute (the host polls until the last step's event has
+    completed)."""
 
-    def __init__(self, gpu_id):
-        self.gpu_id = gpu_id
-        self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+    REASONS = (("hw_slowdown", 0x8), ("sw_thermal_slowdown", 0x20),
+               ("hw_thermal_slowdown", 0x40), ("sw_power_cap", 0x4))
 
-    def __enter__(self):
+    def __init__(self, torch_device):
+        self.samples = []
+        self.handle = None
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.f = open(self.path, "w")
-            cmd = ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits", "-lms", "200"]
-            if self.gpu_id is not None:
-                cmd += ["-i", str(self.gpu_id)]
-            self.proc = subprocess.Popen(cmd, stdout=self.f, stderr=subprocess.DEVNULL)
-        except Exception:
-            self.proc = None
-        return self
-
-    def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            import torch
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(torch_device).uuid)
             try:
-                self.proc.wait(timeout=5)
+                self.handle = pynvml.nvmlDeviceGetHandleByUUID(uuid)
             except Exception:
-                self.proc.kill()
-            self.f.close()
+                self.handle = pynvml.nvmlDeviceGetHandleByIndex(torch_device.index or 0)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.handle = None
+
+    def sample(self):
+        if self.handle is None:
+            return
+        nv = self.nv
+        try:
+            sm = nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)
+            try:
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+            except Exception:
+                rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.handle)
+            pw = nv.nvmlDeviceGetPowerUsage(self.handle) / 1000.0
+            self.samples.append((sm, rs, pw))
+        except Exception:
+            pass
+
+    def poll_until(self, event, min_samples=3):
+        """Sample while `event` (the last timed step) has not completed."""
+        import time as _t
+        while not event.query() or len(self.samples) < min_samples:
+            self.sample()
+            if event.query() and len(self.samples) >= min_samples:
+                break
+            _t.sleep(0.0005)
 
     def summary(self):
-        if self.proc is None:
+        if self.handle is None or not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        rows = []
-        for line in open(self.path):
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), power=float(parts[3]),
-                                 hw=parts[5], hwt=parts[6], swt=parts[7], pcap=parts[8]))
-            except ValueError:
-                continue
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
         reasons = set()
-        for r in rows:
-            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
-                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
-                if r[key].lower().startswith("active"):
+        for _, rs, _ in self.samples:
+            for name, bit in self.REASONS:
+                if rs & bit:
                     reasons.add(name)
-        return {"sm_mhz": statistics.median(r["sm"] for r in rows),
-                "sm_max_mhz": max(r["smax"] for r in rows),
-                "power_w_max": max(r["power"] for r in rows),
-                "samples": len(rows), "reasons": sorted(reasons)}
+        return {"sm_mhz": statistics.median(s for s, _, _ in self.samples),
+                "sm_max_mhz": self.max_mhz,
+                "power_w_max": max(p for _, _, p in self.samples),
+                "samples": len(self.samples), "reasons": sorted(reasons)}
 
 
 # --------------------------------------------------------------------------- work model
@@ -164,7 +179,7 @@ def run_ours(args, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    p = workloads.problem(args.workload)
+    p = workload(args)
     d = workloads.make_inputs(p, seed=args.seed + rank, device=dev)
     wts = {k: d.get(k) for k in ("w13", "w13_scale", "w2", "w2_scale", "gate_up_expert_scales",
                                  "down_expert_scales", "c_input_scales")}
@@ -196,21 +211,18 @@ def run_ours(args, rank, world, local_rank):
     api.timing_enable(True, max(args.steps, 1))
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    gpu_id = None
-    try:
-        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
-    except Exception:
-        gpu_id = local_rank
+    clocks = ClockSampler(dev)
     barrier()
     torch.cuda.synchronize()
-    with ClockSampler(gpu_id) as clocks:
-        for i in range(args.steps):
-            flush.fill_(i & 0xFF)
-            starts[i].record(stream)
-            step()
-            ends[i].record(stream)
-        torch.cuda.synchronize()
-        barrier()
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+        clocks.sample()
+    clocks.poll_until(ends[-1])
+    torch.cuda.synchronize()
+    barrier()
     per_step = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     kern = api.timing_read()
     api.timing_enable(False, 0)
@@ -352,7 +364,8 @@ def main_ours(args):
         "dtype": {"bf16": "bf16", "fp8": "e4m3+f32 scales (f32 accumulate)",
                   "nvfp4": "e2m1+e4m3 scales (f32 accumulate)"}[p["format"]],
         "data": "synthetic (seeded torch generators; random-init experts of the workload's shapes)",
-        "config": {"workload": args.workload, "num_tokens": p["num_tokens"], "hidden": p["hidden"],
+        "config": {"workload": args.workload + ("" if not args.set else " (" + ",".join(args.set) + ")"),
+                   "num_tokens": p["num_tokens"], "hidden": p["hidden"],
                    "intermediate_hidden": p["intermediate_hidden"], "num_experts": p["num_experts"],
                    "num_topk": p["num_topk"], "format": p["format"], "routing": p["routing"],
                    "active_experts": r["num_active"], "parallelism": f"dp{world} (replicas)",
@@ -395,7 +408,7 @@ def main_reference(args):
     from mixture_experts_routed_03_b200 import workloads
     from oracle import moe as O
 
-    p = workloads.problem(args.workload)
+    p = workload(args)
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     host = workloads.to_numpy(workloads.make_inputs(p, seed=args.seed, device=dev))
     M, k = p["num_tokens"], p["num_topk"]

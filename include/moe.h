@@ -110,11 +110,14 @@ typedef struct {
   const void* x_scale;
 } moe_act_t;
 
-/* Expert weights (device), in the layouts listed above.  For NVFP4 the
- * w13_scale / w2_scale pointers must be the PREPARED scale tiles written by
- * moe_prepare_weights (Struct_mega_ffn_ep_combine_send: "pre-permuted W13
- * scale tile", "W2 scale tile"); the three per-expert FP32 arrays are used
- * by NVFP4 only and may be NULL otherwise. */
+/* Expert weights (device).  moe_prepare_weights takes them in the logical
+ * layouts listed above.  Every other call takes w13 and w2 as the PREPARED
+ * blobs that moe_prepare_weights wrote (Struct_mega_ffn_ep_combine_send:
+ * "pre-permuted gate/up weights", "pre-permuted W13 scale tile"); for NVFP4
+ * the block scales are inside those blobs and w13_scale / w2_scale are
+ * ignored; for FP8 w13_scale / w2_scale are the logical FP32 block scales.
+ * The three per-expert FP32 arrays are used by NVFP4 only and may be NULL
+ * otherwise. */
 typedef struct {
   const void* w13;
   const void* w13_scale;
@@ -174,15 +177,22 @@ moe_status_t moe_get_workspace_size(const moe_problem_t* problem, size_t* bytes)
  * allocating a workspace and after moe_read_status reported an error. */
 moe_status_t moe_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
 
-/* Prepares NVFP4 weight scales for the kernels (one time, per weight set):
- * rewrites w13_scale [E, 2I, H/16] and w2_scale [E, H, I/16] into 128-row x
- * 4-block tiles (512 bytes each, the order the tensor-core scale copy reads).
- * out_w13_scale and out_w2_scale are device buffers of the same byte sizes as
- * the inputs.  BF16 and FP8 weights need no preparation (returns
- * MOE_ERR_UNSUPPORTED for them). */
-moe_status_t moe_prepare_weights(const moe_problem_t* problem, const void* w13_scale,
-                                 const void* w2_scale, void* out_w13_scale,
-                                 void* out_w2_scale, void* stream);
+/* Bytes of the prepared gate_up and down weight blobs. */
+moe_status_t moe_get_prepared_weights_size(const moe_problem_t* problem, size_t* w13_bytes,
+                                           size_t* w2_bytes);
+
+/* One-time re-layout of the expert weights for the GEMM kernels (per weight
+ * set; "pre-permuted" weights of Struct_mega_ffn_ep_combine_send).  Reads
+ * `logical` (w13 / w2 and, for NVFP4, w13_scale / w2_scale in the logical
+ * layouts above) and writes out_w13 / out_w2 (device, sizes from
+ * moe_get_prepared_weights_size, 16-byte aligned).  The blobs hold, for
+ * every (expert, n tile, 128-byte K slice), the 256 weight rows the tile
+ * multiplies (gate_up tiles: 64 gate rows, the 64 matching up rows, then
+ * the next 64 of each) in the 128-byte-swizzled order the tensor cores read,
+ * followed for NVFP4 by the slice's E4M3 scales in 512-byte tiles, so each
+ * pipeline stage streams one contiguous block. */
+moe_status_t moe_prepare_weights(const moe_problem_t* problem, const moe_weights_t* logical,
+                                 void* out_w13, void* out_w2, void* stream);
 
 /* Routing from logits (flashinfer.fused_moe.MoEActivationPack, FromLogits).
  * logits fp32 [M, E]; bias fp32 [E] or NULL (used for the selection only).

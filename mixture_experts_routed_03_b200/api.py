@@ -36,6 +36,7 @@ MOE_IN_STAGED = 1
 # Every entry point declared in include/moe.h.
 EXPORTS = (
     "moe_init", "moe_get_workspace_size", "moe_workspace_init", "moe_prepare_weights",
+    "moe_get_prepared_weights_size",
     "moe_route", "moe_permute", "moe_ffn", "moe_get_intermediate_size", "moe_combine",
     "moe_fused", "moe_read_status", "moe_status_string", "moe_timing_enable", "moe_timing_read",
 )
@@ -99,7 +100,8 @@ def lib():
             "moe_init": [ctypes.c_int],
             "moe_get_workspace_size": [P, ctypes.POINTER(sz)],
             "moe_workspace_init": [vp, sz, vp],
-            "moe_prepare_weights": [P, vp, vp, vp, vp, vp],
+            "moe_prepare_weights": [P, ctypes.POINTER(Weights), vp, vp, vp],
+            "moe_get_prepared_weights_size": [P, ctypes.POINTER(sz), ctypes.POINTER(sz)],
             "moe_route": [P, vp, vp, vp, vp, vp],
             "moe_permute": [P, vp, ctypes.POINTER(Layout), vp, sz, vp],
             "moe_ffn": [P, ctypes.POINTER(Act), ctypes.POINTER(Weights), ctypes.POINTER(Layout),
@@ -203,10 +205,16 @@ def workspace_init(ws, nbytes, stream=None):
     _check("moe_workspace_init", lib().moe_workspace_init(_ptr(ws), int(nbytes), _stream(stream)))
 
 
-def prepare_weights(prob, w13_scale, w2_scale, out_w13_scale, out_w2_scale, stream=None):
+def prepared_weights_size(prob):
+    a, b = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    _check("moe_get_prepared_weights_size",
+           lib().moe_get_prepared_weights_size(ctypes.byref(prob), ctypes.byref(a), ctypes.byref(b)))
+    return a.value, b.value
+
+
+def prepare_weights(prob, logical, out_w13, out_w2, stream=None):
     _check("moe_prepare_weights", lib().moe_prepare_weights(
-        ctypes.byref(prob), _ptr(w13_scale), _ptr(w2_scale), _ptr(out_w13_scale),
-        _ptr(out_w2_scale), _stream(stream)))
+        ctypes.byref(prob), ctypes.byref(logical), _ptr(out_w13), _ptr(out_w2), _stream(stream)))
 
 
 def route(prob, logits, bias, topk_idx, topk_weights, stream=None):

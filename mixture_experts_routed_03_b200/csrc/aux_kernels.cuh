@@ -153,6 +153,17 @@ __global__ void __launch_bounds__(256) perm_scatter_kernel(const int64_t* __rest
   int* cursor = start + E + 1;     // [E]
   int* tmp = cursor + E;           // [E+1]
   int* tmp2 = tmp + E + 1;         // [E+1]
+  int* sidx = tmp2 + E + 1;        // [kPermChunk] this chunk's expert ids
+  const int64_t base = static_cast<int64_t>(blockIdx.x) * kPermChunk;
+  for (int i = threadIdx.x; i < kPermChunk; i += blockDim.x) {
+    const int64_t s = base + i;
+    int v = -1;
+    if (s < R) {
+      const int64_t x = idx[s];
+      v = (x >= 0 && x < E) ? static_cast<int>(x) : -1;
+    }
+    sidx[i] = v;
+  }
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     int tot = 0, before = 0;
     for (int b = 0; b < nblk; ++b) {
@@ -202,14 +213,13 @@ __global__ void __launch_bounds__(256) perm_scatter_kernel(const int64_t* __rest
 
   if (threadIdx.x < 32) {
     const int lane = threadIdx.x;
-    const int64_t base = static_cast<int64_t>(blockIdx.x) * kPermChunk;
     const unsigned lt = (1u << lane) - 1u;
     for (int rnd = 0; rnd < kPermChunk / 32; ++rnd) {
       const int64_t s = base + rnd * 32 + lane;
       if (base + rnd * 32 >= R) break;
-      const int64_t v = (s < R) ? idx[s] : -1;
-      const bool valid = v >= 0 && v < E;
-      const int key = valid ? static_cast<int>(v) : (E + lane);
+      const int v = sidx[rnd * 32 + lane];
+      const bool valid = v >= 0;
+      const int key = valid ? v : (E + lane);
       const unsigned peers = __match_any_sync(0xFFFFFFFFu, key);
       int row = -1;
       if (valid) {
@@ -322,26 +332,6 @@ __global__ void __launch_bounds__(256) combine_staged_kernel(const float* __rest
     }
     out[i] = make_uint4(pack_bf16x2(s[0], s[1]), pack_bf16x2(s[2], s[3]),
                         pack_bf16x2(s[4], s[5]), pack_bf16x2(s[6], s[7]));
-  }
-}
-
-// NVFP4 weight scales [rows][K/16] (rows a multiple of 128) -> 512-byte
-// tiles [rows/128][K/64]: tile byte 16*i + 4*m + b holds row 32*m + i of the
-// block, scale column 4*tile_k + b.  One thread per output byte.
-__global__ void __launch_bounds__(256) prepare_sf_kernel(const uint8_t* __restrict__ in,
-                                                         uint8_t* __restrict__ out, int64_t rows,
-                                                         int kcols) {
-  const int kc = kcols / 4;
-  const int64_t n = rows * kcols;
-  for (int64_t o = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; o < n;
-       o += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t tile = o / 512;
-    const int b = static_cast<int>(o - tile * 512);
-    const int64_t rb = tile / kc;
-    const int tk = static_cast<int>(tile - rb * kc);
-    const int64_t row = rb * 128 + ((b & 15) >> 2) * 32 + (b >> 4);
-    const int col = tk * 4 + (b & 3);
-    out[o] = in[row * kcols + col];
   }
 }
 

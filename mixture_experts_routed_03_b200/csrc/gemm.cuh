@@ -13,25 +13,35 @@
 //          it, partial * (a_scale[row, kb] * b_scale[n_blk, kb]), into FP32
 //          registers (the per-128 FP32 block scales have no hardware form)
 //
-// Roles: warp 0 lane 0 issues TMA loads of 128 x 128-byte A rows and
-// 256 x 128-byte B rows per stage (+ the NVFP4 scale tiles as bulk copies)
-// into a STAGES-deep ring guarded by mbarriers; warp 1 lane 0 issues the
-// MMAs (M = 128, N = 256, four K steps of 32 bytes per stage) and commits
-// them to the ring and to the accumulator barriers; the remaining warps are
-// the epilogue, one TMEM lane (= one output row) per thread.
+// Operands.  A (routed rows in expert order) comes by TMA, 128 rows x 128
+// bytes per stage, 128-byte swizzle.  B (expert weights) is PREPARED once
+// (moe_prepare_weights, the "pre-permuted" weights of mega_ffn_ep_combine_
+// send): every (expert, n tile, K stage) block of 256 rows x 128 bytes is
+// stored contiguously, already in the 128-byte-swizzled order the MMA reads
+// (16-byte chunk c of row r at chunk c ^ (r mod 8)), followed for NVFP4 by its
+// 4 KB of scale tiles, so one bulk copy per stage streams it sequentially
+// from HBM.  L1 B tiles interleave gate and up rows as [gate j0..j0+63 |
+// up j0..j0+63 | gate j0+64..j0+127 | up j0+64..j0+127], so each 128-column
+// half of the accumulator holds matching gate and up columns.
+//
+// Roles (320 threads): warp 0 lane 0 issues the copies into a 4-stage ring
+// guarded by mbarriers; warp 1 lane 0 issues the MMAs (M = 128, N = 256, four
+// 32-byte K steps per stage) and commits them; warps 2..9 are the epilogue,
+// two warps per 32-lane TMEM quarter, one per 128-column half, one row per
+// thread.
 //
 // Tiles are (active expert, n tile, 128-row m tile), expert-major, m
-// fastest, handed out round-robin over a grid of at most one CTA per SM.
+// fastest, handed out round-robin over at most one CTA per SM.
 //
-// L1 epilogue: g and u of the same intermediate column j sit in one tile
-// (gate rows of W13 first, up rows I further down); h = min(g,c) *
-// sigmoid(min(g,c)) * clamp(u,-c,c) is re-quantised in registers (BF16 by
+// L1 epilogue: h = min(g,c) * sigmoid(min(g,c)) * clamp(u,-c,c) is formed in
+// registers, the accumulator is released, then h is re-quantised (BF16 by
 // rounding; FP8 per 128 columns with scale amax/448; NVFP4 per 16 columns
 // with an E4M3 scale against the per-expert c_input_scales) and stored in
 // expert order for L2.
-// L2 epilogue: every finished row is multiplied by its router weight and
-// red-added (float4 atomics) into the token-ordered FP32 accumulator -- no
-// (M*k, H) staging buffer -- or, in staged mode, stored per row.
+// L2 epilogue: the row is read into registers, the accumulator released, and
+// the row, times its router weight, red-added (float4 atomics) into the
+// token-ordered FP32 accumulator -- no (M*k, H) staging buffer -- or, in
+// staged mode, stored per row.
 //
 // Every wait is bounded; a wait that runs out records MOE_ERR_TIMEOUT in the
 // workspace status word, raises a CTA-wide abort flag, drains the copies and
@@ -56,23 +66,38 @@ constexpr int kSFBStage = 2 * 4 * kSFTile;    // 2 row blocks x 4 K-steps
 constexpr int kTmemCols = 512;
 constexpr int kSFACol = 256;                  // NVFP4: TMEM columns of the A scales
 constexpr int kSFBCol = 256 + 16;             // NVFP4: TMEM columns of the B scales
+constexpr int kEpiWarps = 8;
 
-template <int FMT>
+// Bytes of one prepared B block (one stage of one tile).
+__host__ __device__ constexpr int b_block_bytes(int fmt) {
+  return kBStage + (fmt == FMT_NVFP4 ? kSFBStage : 0);
+}
+
+// Logical weight row held by row r (0..255) of L1 tile nt: gate and up rows
+// of intermediate columns 128*nt .. 128*nt+127 in 64-row groups.
+__host__ __device__ inline int l1_tile_row(int nt, int r, int I) {
+  const int g = r >> 6, o = r & 63;
+  const int col = 128 * nt + ((g >> 1) << 6) + o;
+  return (g & 1) ? I + col : col;
+}
+
+template <int FMT, int EPI>
 struct GemmCfg {
-  static constexpr int kStages = 4;
-  static constexpr int kEpiWarps = (FMT == FMT_FP8) ? 8 : 4;
+  // L2 gives 36 KB of shared memory to the epilogue's transpose buffers
+  static constexpr int kStages = (EPI == EPI_L1) ? 4 : 3;
   // accumulator (BF16/NVFP4) or partial (FP8) buffers of 256 TMEM columns
   static constexpr int kAccBufs = (FMT == FMT_NVFP4) ? 1 : 2;
   static constexpr int kStageBytes =
-      kAStage + kBStage + ((FMT == FMT_NVFP4) ? (kSFAStage + kSFBStage) : 0);
+      kAStage + kBStage + ((FMT == FMT_NVFP4) ? (kSFBStage + kSFAStage) : 0);
   static constexpr int kThreads = (2 + kEpiWarps) * 32;
   static constexpr int kBarrierBytes = 4096;
-  static constexpr int kSmemBytes = 1024 /*align*/ + kStages * kStageBytes + kBarrierBytes;
+  static constexpr int kXposeStride = 36;   // floats per row of a 32 x 32 transpose buffer
+  static constexpr int kXposeBytes = (EPI == EPI_L1) ? 0 : kEpiWarps * 32 * kXposeStride * 4;
+  static constexpr int kSmemBytes = 1024 /*align*/ + kStages * kStageBytes + kBarrierBytes + kXposeBytes;
 };
 
 struct GemmArgs {
   int k_stages;       // K bytes / 128
-  int w_rows;         // rows of B per expert: 2I (L1) or H (L2)
   int n_tiles;        // tiles along N: I/128 (L1, 128 h columns per tile) or H/256 (L2)
   int I, H, topk;
   float clamp;
@@ -85,11 +110,11 @@ struct GemmArgs {
   const int* tile_offsets;
   const int* src_info;
   const float* topk_weights;
-  // NVFP4 scales: 512-byte tiles [row block][K/64]
+  // prepared weights: [E][n_tiles][k_stages] blocks of b_block_bytes(FMT)
+  const uint8_t* wB;
+  // NVFP4 A scales: 512-byte tiles [row block][K/64]
   const uint8_t* sfa;
   int sfa_kc;
-  const uint8_t* sfb;
-  int sfb_kc;
   // FP8 scales: A transposed [K/128][sa_ld] (padded rows), B [E][N/128][K/128]
   const float* sa_t;
   int sa_ld;
@@ -149,8 +174,8 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
 __device__ __forceinline__ float clamped_swiglu(float g, float u, float c, int fast) {
   const float gc = fminf(g, c);
   const float uc = fminf(fmaxf(u, -c), c);
-  const float ex = fast ? __expf(-gc) : expf(-gc);
-  return __fmul_rn(__fdiv_rn(gc, 1.0f + ex), uc);
+  if (fast) return __fmul_rn(__fdividef(gc, 1.0f + __expf(-gc)), uc);
+  return __fmul_rn(__fdiv_rn(gc, 1.0f + expf(-gc)), uc);
 }
 
 // Byte offset of (padded row pr, scale column j) inside the 512-byte scale
@@ -161,15 +186,22 @@ __device__ __forceinline__ size_t sf_tile_offset(int pr, int j, int kc) {
          ((pr >> 5) & 3) * 4 + (j & 3);
 }
 
+// Packed FP32 pair FMA: (d0, d1) += (a0, a1) * (b0, b1).
+__device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 a, b, c;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+      "mov.b64 c, {%0, %1};\n\tfma.rn.f32x2 c, a, b, c;\n\tmov.b64 {%0, %1}, c;\n\t}"
+      : "+f"(d0), "+f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
 template <int FMT, int EPI>
-__global__ void __launch_bounds__(GemmCfg<FMT>::kThreads, 1)
-    moe_gemm_kernel(const __grid_constant__ GemmArgs p, const __grid_constant__ CUtensorMap tmA,
-                    const __grid_constant__ CUtensorMap tmB) {
-  using Cfg = GemmCfg<FMT>;
+__global__ void __launch_bounds__(GemmCfg<FMT, EPI>::kThreads, 1)
+    moe_gemm_kernel(const __grid_constant__ GemmArgs p, const __grid_constant__ CUtensorMap tmA) {
+  using Cfg = GemmCfg<FMT, EPI>;
   constexpr int S = Cfg::kStages;
   constexpr int NACC = Cfg::kAccBufs;
-  constexpr int NEPI = Cfg::kEpiWarps;
   constexpr int SB = Cfg::kStageBytes;
+  constexpr int BB = b_block_bytes(FMT);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -183,6 +215,7 @@ __global__ void __launch_bounds__(GemmCfg<FMT>::kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S * SB + 512);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* xbuf = reinterpret_cast<float*>(smem + S * SB + 1024);  // FP8 L1: [2][2][128] amax
+  float* xpose = reinterpret_cast<float*>(smem + S * SB + Cfg::kBarrierBytes);  // L2: per-warp 32 x 32
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -194,17 +227,14 @@ __global__ void __launch_bounds__(GemmCfg<FMT>::kThreads, 1)
     }
     for (int b = 0; b < NACC; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], NEPI);
+      mbar_init(&acc_empty[b], kEpiWarps);
     }
     mbar_init(final_bar, 1);
     for (int i = 0; i < 4; ++i) mbar_init(&xbar[i], 64);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) {
-    prefetch_tensormap(&tmA);
-    prefetch_tensormap(&tmB);
-  }
+  if (warp == 0 && lane == 0) prefetch_tensormap(&tmA);
   if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
   tc_fence_before();
   __syncthreads();
@@ -223,49 +253,19 @@ __global__ void __launch_bounds__(GemmCfg<FMT>::kThreads, 1)
       for (int T = blockIdx.x; T < total; T += gridDim.x) {
         TileInfo t;
         decode_tile(p, na, T, t);
-        const int wrow = t.e * p.w_rows;
+        const uint8_t* wb =
+            p.wB + (static_cast<size_t>(t.e) * p.n_tiles + t.n_tile) * p.k_stages * BB;
         for (int ks = 0; ks < p.k_stages; ++ks) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status, 1)) goto producer_done;
           uint8_t* sa = smem + stage * SB;
           uint8_t* sbp = sa + kAStage;
           mbar_arrive_expect_tx(&full[stage], SB);
-          const int kx = ks * kBK;
-          tma_load_2d(sa, &tmA, &full[stage], kx, t.row0);
-          if (EPI == EPI_L1) {
-            const int j0 = t.n_tile * 128;
-            if (FMT == FMT_FP8) {
-              // [gate j0..+63 | up j0..+63 | gate j0+64..+127 | up j0+64..+127]
-              tma_load_2d(sbp, &tmB, &full[stage], kx, wrow + j0);
-              tma_load_2d(sbp + 64 * kBK, &tmB, &full[stage], kx, wrow + p.I + j0);
-              tma_load_2d(sbp + 128 * kBK, &tmB, &full[stage], kx, wrow + j0 + 64);
-              tma_load_2d(sbp + 192 * kBK, &tmB, &full[stage], kx, wrow + p.I + j0 + 64);
-            } else {
-              // [gate j0..+127 | up j0..+127]
-              tma_load_2d(sbp, &tmB, &full[stage], kx, wrow + j0);
-              tma_load_2d(sbp + 128 * kBK, &tmB, &full[stage], kx, wrow + p.I + j0);
-            }
-          } else {
-            tma_load_2d(sbp, &tmB, &full[stage], kx, wrow + t.n_tile * kBN);
-          }
+          tma_load_2d(sa, &tmA, &full[stage], ks * kBK, t.row0);
+          bulk_load(sbp, wb + static_cast<size_t>(ks) * BB, BB, &full[stage]);
           if (FMT == FMT_NVFP4) {
-            uint8_t* sfa_s = sbp + kBStage;
-            uint8_t* sfb_s = sfa_s + kSFAStage;
-            bulk_load(sfa_s,
+            bulk_load(sbp + BB,
                       p.sfa + (static_cast<size_t>(t.srow0 >> 7) * p.sfa_kc + ks * 4) * kSFTile,
                       kSFAStage, &full[stage]);
-            int rb0, rb1;
-            if (EPI == EPI_L1) {
-              rb0 = (wrow + t.n_tile * 128) >> 7;
-              rb1 = (wrow + p.I + t.n_tile * 128) >> 7;
-            } else {
-              rb0 = (wrow + t.n_tile * kBN) >> 7;
-              rb1 = rb0 + 1;
-            }
-            bulk_load(sfb_s, p.sfb + (static_cast<size_t>(rb0) * p.sfb_kc + ks * 4) * kSFTile,
-                      4 * kSFTile, &full[stage]);
-            bulk_load(sfb_s + 4 * kSFTile,
-                      p.sfb + (static_cast<size_t>(rb1) * p.sfb_kc + ks * 4) * kSFTile,
-                      4 * kSFTile, &full[stage]);
           }
           ++issued;
           if (++stage == S) {
@@ -323,8 +323,8 @@ __global__ void __launch_bounds__(GemmCfg<FMT>::kThreads, 1)
           const uint64_t adesc = sdesc_sw128(smem_u32(sa));
           const uint64_t bdesc = sdesc_sw128(smem_u32(sbp));
           if (FMT == FMT_NVFP4) {
-            const uint32_t sfa_s = smem_u32(sbp + kBStage);
-            const uint32_t sfb_s = sfa_s + kSFAStage;
+            const uint32_t sfb_s = smem_u32(sbp + kBStage);
+            const uint32_t sfa_s = sfb_s + kSFBStage;
 #pragma unroll
             for (int kc = 0; kc < 4; ++kc) {
               tmem_copy_sf(tmem + kSFACol + 4 * kc, sdesc_sf_tile(sfa_s + kc * kSFTile));
@@ -371,7 +371,7 @@ __global__ void __launch_bounds__(GemmCfg<FMT>::kThreads, 1)
     // ------------------------------------------------------------ epilogue
     const int ew = warp - 2;
     const int q = warp & 3;               // TMEM lane quarter this warp may access
-    const int half = (NEPI == 8) ? (ew >> 2) : 0;
+    const int half = ew >> 2;             // 128-column half of the accumulator
     const int row_local = q * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     int ab = 0;
@@ -384,15 +384,17 @@ __global__ void __launch_bounds__(GemmCfg<FMT>::kThreads, 1)
       const int r = t.row0 + row_local;
       const int pr = t.srow0 + row_local;
 
+      // acc[0..127]: this thread's row, columns 128*half .. 128*half+127 of
+      // the tile (L1: 64 gate then 64 up; L2: output columns)
+      float acc[128];
       if constexpr (FMT == FMT_FP8) {
-        float acc[128];
 #pragma unroll
         for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
         const float* sbe = p.sb + static_cast<size_t>(t.e) * p.sb_nb * p.sb_kb;
         int nb_lo, nb_hi;  // weight blocks of acc[0..63] and acc[64..127]
         if (EPI == EPI_L1) {
-          nb_lo = (t.n_tile * 128) >> 7;
-          nb_hi = (p.I + t.n_tile * 128) >> 7;
+          nb_lo = t.n_tile;
+          nb_hi = (p.I >> 7) + t.n_tile;
         } else {
           nb_lo = nb_hi = (t.n_tile * kBN + half * 128) >> 7;
         }
@@ -408,13 +410,13 @@ __global__ void __launch_bounds__(GemmCfg<FMT>::kThreads, 1)
           const float s_hi = sa * __ldg(sbe + nb_hi * p.sb_kb + ks);
           const uint32_t base = tmem + ab * kBN + half * 128 + lane_off;
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            float v[32];
+          for (int c = 0; c < 8; ++c) {
+            float v[16];
             __syncwarp();
-            tmem_ld32(base + 32 * c, v);
-            const float s = (c < 2) ? s_lo : s_hi;
+            tmem_ld16(base + 16 * c, v);
+            const float s = (c < 4) ? s_lo : s_hi;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) acc[32 * c + i] = fmaf(v[i], s, acc[32 * c + i]);
+            for (int i = 0; i < 8; ++i) ffma2(acc[16 * c + 2 * i], acc[16 * c + 2 * i + 1], v[2 * i], v[2 * i + 1], s, s);
           }
           tc_fence_before();
           __syncwarp();
@@ -425,15 +427,44 @@ __global__ void __launch_bounds__(GemmCfg<FMT>::kThreads, 1)
           }
         }
         if (!ok) break;
-        if (EPI == EPI_L1) {
-          // h for intermediate columns j0 + 64*half + i, i < 64
-          float h[64];
+      } else {
+        // BF16 / NVFP4: the whole K sum is in TMEM; read it, release it.
+        if (!mbar_wait(&acc_full[ab], aphase, abort_flag, p.status, 6)) break;
+        tc_fence_after();
+        const uint32_t base = tmem + ab * kBN + half * 128 + lane_off;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float v[32];
+          __syncwarp();
+          tmem_ld32(base + 32 * c, v);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) acc[32 * c + i] = v[i];
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[ab]);
+        if (++ab == NACC) {
+          ab = 0;
+          aphase ^= 1u;
+        }
+        if (FMT == FMT_NVFP4) {
+          const float alpha = __ldg(p.alpha + t.e);
+#pragma unroll
+          for (int i = 0; i < 128; ++i) acc[i] = __fmul_rn(acc[i], alpha);
+        }
+      }
+
+      if (EPI == EPI_L1) {
+        // h for intermediate columns j0 + 64*half + i, i < 64
+        const int hcol0 = t.n_tile * 128 + half * 64;
+        float h[64];
+#pragma unroll
+        for (int i = 0; i < 64; ++i) h[i] = clamped_swiglu(acc[i], acc[64 + i], p.clamp, p.fast_math);
+        uint8_t* hrow = p.h_out + static_cast<size_t>(r) * p.h_row_bytes;
+        if constexpr (FMT == FMT_FP8) {
           float amax = 0.0f;
 #pragma unroll
-          for (int i = 0; i < 64; ++i) {
-            h[i] = clamped_swiglu(acc[i], acc[64 + i], p.clamp, p.fast_math);
-            amax = fmaxf(amax, fabsf(h[i]));
-          }
+          for (int i = 0; i < 64; ++i) amax = fmaxf(amax, fabsf(h[i]));
           // One FP8 scale covers the tile's 128 columns: combine the two
           // halves held by warps (q, 0) and (q, 1).  The buffer alternates
           // between tiles, so one barrier phase per tile suffices.
@@ -454,122 +485,90 @@ __global__ void __launch_bounds__(GemmCfg<FMT>::kThreads, 1)
                   cvt_e4m3x2(__fmul_rn(h[4 * i + 2], inv), __fmul_rn(h[4 * i + 3], inv));
               w[i] = (s != 0.0f) ? (lo | (hi << 16)) : 0u;
             }
-            uint4* dst = reinterpret_cast<uint4*>(p.h_out + static_cast<size_t>(r) * p.h_row_bytes +
-                                                  t.n_tile * 128 + half * 64);
+            uint4* dst = reinterpret_cast<uint4*>(hrow + hcol0);
 #pragma unroll
             for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
             if (half == 0) p.h_scale_t[static_cast<size_t>(t.n_tile) * p.h_scale_ld + pr] = s;
           }
-        } else if (valid) {
-          const int n0 = t.n_tile * kBN + half * 128;
-          if (EPI == EPI_L2_ACC) {
-            const int s_flat = __ldg(p.src_info + r);
-            const int tok = s_flat / p.topk;
-            const float wgt = __ldg(p.topk_weights + s_flat);
-            float* dst = p.out + static_cast<size_t>(tok) * p.H + n0;
+        } else if constexpr (FMT == FMT_BF16) {
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(hrow + hcol0 * 2);
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-              atomicAdd(reinterpret_cast<float4*>(dst) + i,
-                        make_float4(acc[4 * i] * wgt, acc[4 * i + 1] * wgt, acc[4 * i + 2] * wgt,
-                                    acc[4 * i + 3] * wgt));
-          } else {
-            float4* dst = reinterpret_cast<float4*>(p.out + static_cast<size_t>(r) * p.H + n0);
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_uint4(pack_bf16x2(h[8 * i], h[8 * i + 1]), pack_bf16x2(h[8 * i + 2], h[8 * i + 3]),
+                                  pack_bf16x2(h[8 * i + 4], h[8 * i + 5]), pack_bf16x2(h[8 * i + 6], h[8 * i + 7]));
+          }
+        } else {
+          const float G = __ldg(p.c_in + t.e);
+          const float denom6 = __fmul_rn(6.0f, G);
+          uint32_t codes[8];
+          uint32_t sfw = 0;
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-              dst[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
+          for (int b = 0; b < 4; ++b) {
+            float amax = 0.0f;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(h[16 * b + j]));
+            const uint32_t sf_code = cvt_e4m3x2(__fdiv_rn(amax, denom6), 0.0f) & 0xFFu;
+            const float sf = e4m3_to_f32(sf_code);
+            uint32_t w0 = 0, w1 = 0;
+            if (sf != 0.0f) {
+              const float inv = __frcp_rn(__fmul_rn(sf, G));
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                w0 |= cvt_e2m1x2(__fmul_rn(h[16 * b + 2 * j], inv), __fmul_rn(h[16 * b + 2 * j + 1], inv)) << (8 * j);
+                w1 |= cvt_e2m1x2(__fmul_rn(h[16 * b + 8 + 2 * j], inv), __fmul_rn(h[16 * b + 9 + 2 * j], inv))
+                      << (8 * j);
+              }
+            }
+            codes[2 * b] = w0;
+            codes[2 * b + 1] = w1;
+            sfw |= sf_code << (8 * b);
+          }
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(hrow + hcol0 / 2);
+            dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+            dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+            // the 4 scale bytes of columns hcol0/16 .. +3 are contiguous in one tile
+            *reinterpret_cast<uint32_t*>(p.h_sf + sf_tile_offset(pr, hcol0 >> 4, p.h_sf_kc)) = sfw;
           }
         }
       } else {
-        // BF16 / NVFP4: the whole K sum is in TMEM.
-        if (!mbar_wait(&acc_full[ab], aphase, abort_flag, p.status, 6)) break;
-        tc_fence_after();
-        const uint32_t base = tmem + ab * kBN + lane_off;
-        const float alpha = (FMT == FMT_NVFP4) ? __ldg(p.alpha + t.e) : 1.0f;
-        if (EPI == EPI_L1) {
-          const int j0 = t.n_tile * 128;
-          const float G = (FMT == FMT_NVFP4) ? __ldg(p.c_in + t.e) : 1.0f;
-          const float denom6 = __fmul_rn(6.0f, G);
-#pragma unroll 1
-          for (int i = 0; i < 8; ++i) {
-            float g[16], u[16];
-            __syncwarp();
-            tmem_ld16(base + 16 * i, g);
-            tmem_ld16(base + 128 + 16 * i, u);
-            float h[16];
-            float amax = 0.0f;
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              float gg = g[j], uu = u[j];
-              if (FMT == FMT_NVFP4) {
-                gg = __fmul_rn(gg, alpha);
-                uu = __fmul_rn(uu, alpha);
-              }
-              h[j] = clamped_swiglu(gg, uu, p.clamp, p.fast_math);
-              amax = fmaxf(amax, fabsf(h[j]));
-            }
-            if (!valid) continue;
-            if (FMT == FMT_BF16) {
-              uint32_t w[8];
-#pragma unroll
-              for (int j = 0; j < 8; ++j) w[j] = pack_bf16x2(h[2 * j], h[2 * j + 1]);
-              uint4* dst = reinterpret_cast<uint4*>(p.h_out + static_cast<size_t>(r) * p.h_row_bytes +
-                                                    (j0 + 16 * i) * 2);
-              dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-              dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-            } else {
-              const uint32_t sf_code = cvt_e4m3x2(__fdiv_rn(amax, denom6), 0.0f) & 0xFFu;
-              const float sf = e4m3_to_f32(sf_code);
-              uint32_t w0 = 0, w1 = 0;
-              if (sf != 0.0f) {
-                const float inv = __frcp_rn(__fmul_rn(sf, G));
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                  w0 |= cvt_e2m1x2(__fmul_rn(h[2 * j], inv), __fmul_rn(h[2 * j + 1], inv)) << (8 * j);
-                  w1 |= cvt_e2m1x2(__fmul_rn(h[8 + 2 * j], inv), __fmul_rn(h[9 + 2 * j], inv)) << (8 * j);
-                }
-              }
-              *reinterpret_cast<uint2*>(p.h_out + static_cast<size_t>(r) * p.h_row_bytes +
-                                        (j0 + 16 * i) / 2) = make_uint2(w0, w1);
-              p.h_sf[sf_tile_offset(pr, (j0 >> 4) + i, p.h_sf_kc)] = static_cast<uint8_t>(sf_code);
-            }
-          }
-        } else {
-          int tok = 0;
-          float wgt = alpha;
-          if (valid && EPI == EPI_L2_ACC) {
-            const int s_flat = __ldg(p.src_info + r);
-            tok = s_flat / p.topk;
-            wgt = alpha * __ldg(p.topk_weights + s_flat);
-          }
-          const int n0 = t.n_tile * kBN;
-#pragma unroll 1
-          for (int c = 0; c < 8; ++c) {
-            float v[32];
-            __syncwarp();
-            tmem_ld32(base + 32 * c, v);
-            if (!valid) continue;
-            if (EPI == EPI_L2_ACC) {
-              float* dst = p.out + static_cast<size_t>(tok) * p.H + n0 + 32 * c;
-#pragma unroll
-              for (int i = 0; i < 8; ++i)
-                atomicAdd(reinterpret_cast<float4*>(dst) + i,
-                          make_float4(v[4 * i] * wgt, v[4 * i + 1] * wgt, v[4 * i + 2] * wgt,
-                                      v[4 * i + 3] * wgt));
-            } else {
-              float4* dst = reinterpret_cast<float4*>(p.out + static_cast<size_t>(r) * p.H + n0 + 32 * c);
-#pragma unroll
-              for (int i = 0; i < 8; ++i)
-                dst[i] = make_float4(v[4 * i] * wgt, v[4 * i + 1] * wgt, v[4 * i + 2] * wgt,
-                                     v[4 * i + 3] * wgt);
-            }
-          }
+        // L2: write the rows through a per-warp 32 x 32 transpose so that one
+        // warp instruction covers four whole 128-byte row segments (8 lanes
+        // per row) instead of 32 scattered 16-byte pieces.
+        const int n0 = t.n_tile * kBN + half * 128;
+        int tok = r;
+        float wgt = 1.0f;
+        if (valid && EPI == EPI_L2_ACC) {
+          const int s_flat = __ldg(p.src_info + r);
+          tok = s_flat / p.topk;
+          wgt = __ldg(p.topk_weights + s_flat);
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[ab]);
-        if (++ab == NACC) {
-          ab = 0;
-          aphase ^= 1u;
+        float* xb = xpose + ew * (32 * Cfg::kXposeStride);
+        const int rows_here = t.rows - q * 32;   // valid rows of this warp's quarter
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float4* wrow = reinterpret_cast<float4*>(xb + lane * Cfg::kXposeStride);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            wrow[i] = make_float4(acc[32 * c + 4 * i], acc[32 * c + 4 * i + 1], acc[32 * c + 4 * i + 2],
+                                  acc[32 * c + 4 * i + 3]);
+          __syncwarp();
+#pragma unroll
+          for (int it = 0; it < 8; ++it) {
+            const int row = it * 4 + (lane >> 3);
+            const int c4 = lane & 7;
+            const int rtok = __shfl_sync(0xFFFFFFFFu, tok, row);
+            const float rw = __shfl_sync(0xFFFFFFFFu, wgt, row);
+            const float4 v = *reinterpret_cast<const float4*>(xb + row * Cfg::kXposeStride + 4 * c4);
+            if (row < rows_here) {
+              float4* dst = reinterpret_cast<float4*>(p.out + static_cast<size_t>(rtok) * p.H + n0 + 32 * c) + c4;
+              const float4 o = make_float4(v.x * rw, v.y * rw, v.z * rw, v.w * rw);
+              if (EPI == EPI_L2_ACC) atomicAdd(dst, o);
+              else *dst = o;
+            }
+          }
+          __syncwarp();
         }
       }
     }
@@ -579,6 +578,63 @@ __global__ void __launch_bounds__(GemmCfg<FMT>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
+// ---------------------------------------------------------------------------
+// Weight preparation: logical K-major weights [E][N][Kb] (+ NVFP4 scales
+// [E][N][K/16]) -> blocks [E][n_tiles][k_stages] of b_block_bytes(fmt).
+// One thread per 16-byte chunk of block data; the NVFP4 scale tiles follow.
+// ---------------------------------------------------------------------------
+struct PrepArgs {
+  const uint8_t* w;        // logical weights
+  const uint8_t* sf;       // NVFP4 logical scales, else null
+  uint8_t* out;
+  int E, N, Kb;            // experts, rows per expert, bytes per row
+  int ksf;                 // NVFP4 scale columns per row (K/16)
+  int n_tiles, k_stages;
+  int l1;                  // 1: gate/up interleaved L1 tiles (N = 2I)
+  int fmt;
+};
+
+__device__ __forceinline__ int prep_row(const PrepArgs& a, int nt, int r) {
+  return a.l1 ? l1_tile_row(nt, r, a.N / 2) : nt * kBN + r;
+}
+
+__global__ void __launch_bounds__(256) prepare_weights_kernel(PrepArgs a) {
+  const int bb = b_block_bytes(a.fmt);
+  const int64_t blocks = static_cast<int64_t>(a.E) * a.n_tiles * a.k_stages;
+  const int64_t n16 = blocks * (kBStage / 16);
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n16;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t blk = i / (kBStage / 16);
+    const int within = static_cast<int>(i - blk * (kBStage / 16));
+    const int r = within >> 3, cpos = within & 7;
+    const int ks = static_cast<int>(blk % a.k_stages);
+    const int64_t et = blk / a.k_stages;
+    const int nt = static_cast<int>(et % a.n_tiles);
+    const int e = static_cast<int>(et / a.n_tiles);
+    const int row = prep_row(a, nt, r);
+    const int c = cpos ^ (r & 7);
+    const uint4* src = reinterpret_cast<const uint4*>(
+        a.w + (static_cast<size_t>(e) * a.N + row) * a.Kb + static_cast<size_t>(ks) * kBK + 16 * c);
+    *reinterpret_cast<uint4*>(a.out + blk * bb + within * 16) = *src;
+  }
+  if (a.fmt != FMT_NVFP4) return;
+  const int64_t nsf = blocks * kSFBStage;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nsf;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t blk = i / kSFBStage;
+    const int o = static_cast<int>(i - blk * kSFBStage);
+    const int rb = o / (4 * kSFTile), kc = (o / kSFTile) & 3, b = o & (kSFTile - 1);
+    const int ks = static_cast<int>(blk % a.k_stages);
+    const int64_t et = blk / a.k_stages;
+    const int nt = static_cast<int>(et % a.n_tiles);
+    const int e = static_cast<int>(et / a.n_tiles);
+    const int tile_row = 128 * rb + ((b & 15) >> 2) * 32 + (b >> 4);
+    const int row = prep_row(a, nt, tile_row);
+    const int col = ks * 16 + kc * 4 + (b & 3);
+    a.out[blk * bb + kBStage + o] = a.sf[(static_cast<size_t>(e) * a.N + row) * a.ksf + col];
+  }
 }
 
 }  // namespace moe

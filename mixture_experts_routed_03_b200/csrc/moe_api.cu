@@ -169,7 +169,7 @@ int sm_count() {
 template <int FMT, int EPI>
 cudaError_t set_gemm_attr() {
   return cudaFuncSetAttribute(moe_gemm_kernel<FMT, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              GemmCfg<FMT>::kSmemBytes);
+                              GemmCfg<FMT, EPI>::kSmemBytes);
 }
 
 template <int FMT>
@@ -198,20 +198,27 @@ bool ensure_init() {
 }
 
 template <int FMT, int EPI>
-cudaError_t launch_gemm(const GemmArgs& a, const CUtensorMap& ta, const CUtensorMap& tb, int grid,
-                        cudaStream_t st) {
-  moe_gemm_kernel<FMT, EPI><<<grid, GemmCfg<FMT>::kThreads, GemmCfg<FMT>::kSmemBytes, st>>>(a, ta, tb);
+cudaError_t launch_gemm(const GemmArgs& a, const CUtensorMap& ta, int grid, cudaStream_t st) {
+  moe_gemm_kernel<FMT, EPI><<<grid, GemmCfg<FMT, EPI>::kThreads, GemmCfg<FMT, EPI>::kSmemBytes, st>>>(a, ta);
   return cudaGetLastError();
 }
 
 template <int EPI>
-cudaError_t launch_gemm_fmt(int fmt, const GemmArgs& a, const CUtensorMap& ta, const CUtensorMap& tb,
-                            int grid, cudaStream_t st) {
+cudaError_t launch_gemm_fmt(int fmt, const GemmArgs& a, const CUtensorMap& ta, int grid, cudaStream_t st) {
   switch (fmt) {
-    case FMT_BF16: return launch_gemm<FMT_BF16, EPI>(a, ta, tb, grid, st);
-    case FMT_FP8: return launch_gemm<FMT_FP8, EPI>(a, ta, tb, grid, st);
-    default: return launch_gemm<FMT_NVFP4, EPI>(a, ta, tb, grid, st);
+    case FMT_BF16: return launch_gemm<FMT_BF16, EPI>(a, ta, grid, st);
+    case FMT_FP8: return launch_gemm<FMT_FP8, EPI>(a, ta, grid, st);
+    default: return launch_gemm<FMT_NVFP4, EPI>(a, ta, grid, st);
   }
+}
+
+// Bytes of the prepared gate_up (L1) and down (L2) weight blobs.
+size_t prepared_bytes(const moe_problem_t* p, bool l1) {
+  const int fmt = p->format;
+  const size_t E = p->num_experts, H = p->hidden, I = p->intermediate_hidden;
+  const size_t n_tiles = l1 ? I / 128 : H / 256;
+  const size_t k_stages = size_t(l1 ? x_row_bytes(fmt, int(H)) : h_row_bytes(fmt, int(I))) / 128;
+  return E * n_tiles * k_stages * size_t(b_block_bytes(fmt));
 }
 
 int grid_for(int64_t n, int threads, int cap = 148 * 16) {
@@ -247,7 +254,7 @@ cudaError_t launch_permute(const moe_problem_t* p, const int64_t* idx, const Per
   perm_count_kernel<<<nblk, 256, E * sizeof(int), st>>>(idx, R, E, block_counts, status);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  perm_scatter_kernel<<<nblk, 256, (5 * E + 3) * sizeof(int), st>>>(idx, R, E, nblk, block_counts, o);
+  perm_scatter_kernel<<<nblk, 256, (5 * E + 3 + kPermChunk) * sizeof(int), st>>>(idx, R, E, nblk, block_counts, o);
   return cudaGetLastError();
 }
 
@@ -290,14 +297,12 @@ moe_status_t run_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_wei
   if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
 
   // L1: gate_up
-  CUtensorMap ta{}, tb{};
-  const uint32_t l1_box = (fmt == FMT_FP8) ? 64 : 128;
+  CUtensorMap ta{};
   if (!make_map(&ta, b.x_perm, x_row_bytes(fmt, H), uint64_t(R), 128)) return MOE_ERR_CUDA;
-  if (!make_map(&tb, w->w13, x_row_bytes(fmt, H), uint64_t(E) * 2 * I, l1_box)) return MOE_ERR_CUDA;
   GemmArgs a{};
   a.k_stages = x_row_bytes(fmt, H) / 128;
-  a.w_rows = 2 * I;
   a.n_tiles = I / 128;
+  a.wB = static_cast<const uint8_t*>(w->w13);
   a.I = I;
   a.H = H;
   a.topk = k;
@@ -312,8 +317,6 @@ moe_status_t run_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_wei
   a.topk_weights = topk_weights;
   a.sfa = b.x_sf;
   a.sfa_kc = H / 64;
-  a.sfb = static_cast<const uint8_t*>(w->w13_scale);
-  a.sfb_kc = H / 64;
   a.sa_t = reinterpret_cast<const float*>(b.x_sf);
   a.sa_ld = int(b.P);
   a.sb = static_cast<const float*>(w->w13_scale);
@@ -332,7 +335,7 @@ moe_status_t run_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_wei
   int grid1 = int(std::min<int64_t>(nsm, mtiles_bound * a.n_tiles));
   {
     TimScope ts(MOE_SLOT_GEMM1, st);
-    if (launch_gemm_fmt<EPI_L1>(fmt, a, ta, tb, std::max(grid1, 1), st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_gemm_fmt<EPI_L1>(fmt, a, ta, std::max(grid1, 1), st) != cudaSuccess) return MOE_ERR_CUDA;
   }
 
   // L2: down
@@ -341,17 +344,14 @@ moe_status_t run_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_wei
     zero_kernel<<<grid_for(M * H / 4, 256), 256, 0, st>>>(reinterpret_cast<float4*>(out), M * H / 4);
     if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
   }
-  CUtensorMap ta2{}, tb2{};
+  CUtensorMap ta2{};
   if (!make_map(&ta2, b.h, h_row_bytes(fmt, I), uint64_t(R), 128)) return MOE_ERR_CUDA;
-  if (!make_map(&tb2, w->w2, h_row_bytes(fmt, I), uint64_t(E) * H, 256)) return MOE_ERR_CUDA;
   GemmArgs a2 = a;
   a2.k_stages = h_row_bytes(fmt, I) / 128;
-  a2.w_rows = H;
   a2.n_tiles = H / 256;
+  a2.wB = static_cast<const uint8_t*>(w->w2);
   a2.sfa = b.h_sf;
   a2.sfa_kc = I / 64;
-  a2.sfb = static_cast<const uint8_t*>(w->w2_scale);
-  a2.sfb_kc = I / 64;
   a2.sa_t = reinterpret_cast<const float*>(b.h_sf);
   a2.sb = static_cast<const float*>(w->w2_scale);
   a2.sb_nb = H / 128;
@@ -361,8 +361,8 @@ moe_status_t run_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_wei
   int grid2 = int(std::min<int64_t>(nsm, mtiles_bound * a2.n_tiles));
   TimScope ts2(MOE_SLOT_GEMM2, st);
   cudaError_t e = (out_mode == MOE_OUT_ACCUMULATE)
-                      ? launch_gemm_fmt<EPI_L2_ACC>(fmt, a2, ta2, tb2, std::max(grid2, 1), st)
-                      : launch_gemm_fmt<EPI_L2_STAGED>(fmt, a2, ta2, tb2, std::max(grid2, 1), st);
+                      ? launch_gemm_fmt<EPI_L2_ACC>(fmt, a2, ta2, std::max(grid2, 1), st)
+                      : launch_gemm_fmt<EPI_L2_STAGED>(fmt, a2, ta2, std::max(grid2, 1), st);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -371,7 +371,8 @@ bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15)
 moe_status_t check_act_weights(const moe_problem_t* p, const moe_act_t* act, const moe_weights_t* w) {
   if (!act || !w || !act->x || !w->w13 || !w->w2) return MOE_ERR_INVALID_ARG;
   if (!aligned16(act->x) || !aligned16(w->w13) || !aligned16(w->w2)) return MOE_ERR_INVALID_ARG;
-  if (p->format != MOE_FMT_BF16 && (!act->x_scale || !w->w13_scale || !w->w2_scale)) return MOE_ERR_INVALID_ARG;
+  if (p->format != MOE_FMT_BF16 && !act->x_scale) return MOE_ERR_INVALID_ARG;
+  if (p->format == MOE_FMT_FP8_E4M3_B128 && (!w->w13_scale || !w->w2_scale)) return MOE_ERR_INVALID_ARG;
   if (p->format == MOE_FMT_NVFP4 &&
       (!w->gate_up_expert_scales || !w->down_expert_scales || !w->c_input_scales))
     return MOE_ERR_INVALID_ARG;
@@ -435,22 +436,51 @@ moe_status_t moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
-moe_status_t moe_prepare_weights(const moe_problem_t* p, const void* w13_scale, const void* w2_scale,
-                                 void* out_w13_scale, void* out_w2_scale, void* stream) {
+moe_status_t moe_get_prepared_weights_size(const moe_problem_t* p, size_t* w13_bytes, size_t* w2_bytes) {
   moe_status_t s = check_problem(p);
   if (s != MOE_OK) return s;
-  if (p->format != MOE_FMT_NVFP4) return MOE_ERR_UNSUPPORTED;
-  if (!w13_scale || !w2_scale || !out_w13_scale || !out_w2_scale) return MOE_ERR_INVALID_ARG;
+  if (!w13_bytes || !w2_bytes) return MOE_ERR_INVALID_ARG;
+  *w13_bytes = prepared_bytes(p, true);
+  *w2_bytes = prepared_bytes(p, false);
+  return MOE_OK;
+}
+
+moe_status_t moe_prepare_weights(const moe_problem_t* p, const moe_weights_t* logical, void* out_w13,
+                                 void* out_w2, void* stream) {
+  moe_status_t s = check_problem(p);
+  if (s != MOE_OK) return s;
+  if (!logical || !logical->w13 || !logical->w2 || !out_w13 || !out_w2) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(logical->w13) || !aligned16(logical->w2) || !aligned16(out_w13) || !aligned16(out_w2))
+    return MOE_ERR_INVALID_ARG;
+  if (p->format == MOE_FMT_NVFP4 && (!logical->w13_scale || !logical->w2_scale)) return MOE_ERR_INVALID_ARG;
   if (!ensure_init()) return MOE_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int64_t E = p->num_experts, H = p->hidden, I = p->intermediate_hidden;
-  const int64_t n13 = E * 2 * I * (H / 16), n2 = E * H * (I / 16);
-  prepare_sf_kernel<<<grid_for(n13, 256), 256, 0, st>>>(static_cast<const uint8_t*>(w13_scale),
-                                                       static_cast<uint8_t*>(out_w13_scale), E * 2 * I,
-                                                       int(H / 16));
-  prepare_sf_kernel<<<grid_for(n2, 256), 256, 0, st>>>(static_cast<const uint8_t*>(w2_scale),
-                                                      static_cast<uint8_t*>(out_w2_scale), E * H,
-                                                      int(I / 16));
+  const int fmt = p->format, E = p->num_experts, H = p->hidden, I = p->intermediate_hidden;
+  PrepArgs a{};
+  a.fmt = fmt;
+  a.E = E;
+  // gate_up: 2I rows, K = H
+  a.w = static_cast<const uint8_t*>(logical->w13);
+  a.sf = static_cast<const uint8_t*>(logical->w13_scale);
+  a.out = static_cast<uint8_t*>(out_w13);
+  a.N = 2 * I;
+  a.Kb = x_row_bytes(fmt, H);
+  a.ksf = H / 16;
+  a.n_tiles = I / 128;
+  a.k_stages = a.Kb / 128;
+  a.l1 = 1;
+  prepare_weights_kernel<<<grid_for(int64_t(prepared_bytes(p, true)) / 16, 256), 256, 0, st>>>(a);
+  // down: H rows, K = I
+  a.w = static_cast<const uint8_t*>(logical->w2);
+  a.sf = static_cast<const uint8_t*>(logical->w2_scale);
+  a.out = static_cast<uint8_t*>(out_w2);
+  a.N = H;
+  a.Kb = h_row_bytes(fmt, I);
+  a.ksf = I / 16;
+  a.n_tiles = H / 256;
+  a.k_stages = a.Kb / 128;
+  a.l1 = 0;
+  prepare_weights_kernel<<<grid_for(int64_t(prepared_bytes(p, false)) / 16, 256), 256, 0, st>>>(a);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

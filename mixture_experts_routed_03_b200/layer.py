@@ -55,15 +55,17 @@ class MoELayer:
         self.max_tokens = int(p["num_tokens"])
         self.prob = api.problem_from_dict(self.p, fast_math=fast_math)
         w = weights
-        self.w13, self.w2 = w["w13"], w["w2"]
-        self.w13_scale, self.w2_scale = w.get("w13_scale"), w.get("w2_scale")
         self.alpha1 = w.get("gate_up_expert_scales")
         self.alpha2 = w.get("down_expert_scales")
         self.c_in = w.get("c_input_scales")
-        if self.p["format"] == "nvfp4":
-            self.w13_scale = torch.empty_like(w["w13_scale"])
-            self.w2_scale = torch.empty_like(w["w2_scale"])
-            api.prepare_weights(self.prob, w["w13_scale"], w["w2_scale"], self.w13_scale, self.w2_scale)
+        # FP8 block scales stay logical; NVFP4 scales go into the prepared blobs
+        self.w13_scale = w.get("w13_scale") if self.p["format"] == "fp8" else None
+        self.w2_scale = w.get("w2_scale") if self.p["format"] == "fp8" else None
+        n13, n2 = api.prepared_weights_size(self.prob)
+        self.w13 = torch.empty(n13, dtype=torch.uint8, device=self.device)
+        self.w2 = torch.empty(n2, dtype=torch.uint8, device=self.device)
+        logical = api.weights(w["w13"], w.get("w13_scale"), w["w2"], w.get("w2_scale"))
+        api.prepare_weights(self.prob, logical, self.w13, self.w2)
         self.weights = api.weights(self.w13, self.w13_scale, self.w2, self.w2_scale,
                                    self.alpha1, self.alpha2, self.c_in)
         self.ws_bytes = api.workspace_size(self.prob)

@@ -63,9 +63,14 @@ def test_geometry_validation(lib, kw, code):
 
 
 def test_valid_geometry_and_sizes(lib):
-    for fmt in ("bf16", "fp8", "nvfp4"):
+    for fmt, eb in (("bf16", 2.0), ("fp8", 1.0), ("nvfp4", 0.5)):
         p = _prob(format=fmt, hidden=512, intermediate_hidden=256)
         assert api.workspace_size(p) > 0
+        a, b = api.prepared_weights_size(p)
+        # the prepared blobs hold exactly the weights (+ NVFP4 scales, 1/16 byte per element... 1 per 16)
+        extra = 1.0 / 16 if fmt == "nvfp4" else 0.0
+        assert a == int(8 * 2 * 256 * 512 * (eb + extra))
+        assert b == int(8 * 512 * 256 * (eb + extra))
         n, off = api.intermediate_size(p)
         assert off % 256 == 0 and n > off
     assert api.workspace_size(_prob(activation_clamp=float("inf"))) > 0
@@ -83,7 +88,8 @@ def test_null_pointer_arguments_rejected_before_launch(lib):
     assert lib.moe_ffn(ctypes.byref(p), ctypes.byref(a), ctypes.byref(w), ctypes.byref(lay), None, 5,
                        None, None, None, 0, None) == api.MOE_ERR_INVALID_ARG
     assert lib.moe_read_status(None, None) == api.MOE_ERR_INVALID_ARG
-    assert lib.moe_prepare_weights(ctypes.byref(p), None, None, None, None, None) == api.MOE_ERR_UNSUPPORTED
+    assert lib.moe_prepare_weights(ctypes.byref(p), None, None, None, None) == api.MOE_ERR_INVALID_ARG
+    assert lib.moe_prepare_weights(ctypes.byref(p), ctypes.byref(w), None, None, None) == api.MOE_ERR_INVALID_ARG
 
 
 def test_fused_needs_exactly_one_routing_source(lib):
