@@ -28,6 +28,8 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
                                                     const float* __restrict__ bias, int64_t M,
                                                     int E, int k, int64_t* __restrict__ idx_out,
                                                     float* __restrict__ w_out) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (t >= M) return;
@@ -93,6 +95,8 @@ __global__ void __launch_bounds__(256) perm_count_kernel(const int64_t* __restri
                                                          int64_t R, int E,
                                                          int* __restrict__ block_counts,
                                                          int* status) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ int cnt[];
   for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
   __syncthreads();
@@ -143,10 +147,44 @@ __device__ void warp_exclusive_scan(const int* v, int* out, int n) {
   if (lane == 31) out[n] = incl;
 }
 
+// Writes expert_counts, expert_start_indices, a_scale_offsets, expert_ids,
+// num_active and tile_offsets from the per-expert totals and their exclusive
+// scan (start, E+1 entries).  Called by every thread of one block; tmp and
+// tmp2 are E+1-entry shared scratch arrays.
+__device__ void write_expert_arrays(const int* total, const int* start, int* tmp, int* tmp2, int E,
+                                    const PermOut& o) {
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    o.expert_counts[e] = total[e];
+    o.expert_start_indices[e] = start[e];
+    tmp[e] = (total[e] + 127) / 128 * 128;  // padded rows
+    tmp2[e] = (total[e] > 0) ? 1 : 0;
+  }
+  if (threadIdx.x == 0) o.expert_start_indices[E] = start[E];
+  __syncthreads();
+  if (threadIdx.x < 32) warp_exclusive_scan(tmp, o.a_scale_offsets, E);
+  __syncthreads();
+  // active experts: compact with a scan of the flags (tmp becomes the ranks)
+  if (threadIdx.x < 32) warp_exclusive_scan(tmp2, tmp, E);
+  __syncthreads();
+  const int na = tmp[E];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    if (total[e] > 0) {
+      o.expert_ids[tmp[e]] = e;
+      tmp2[tmp[e]] = (total[e] + 127) / 128;  // m tiles of the a-th active expert
+    }
+    if (e >= na) o.expert_ids[e] = -1;
+  }
+  if (threadIdx.x == 0) *o.num_active = na;
+  __syncthreads();
+  if (threadIdx.x < 32) warp_exclusive_scan(tmp2, o.tile_offsets, na);
+}
+
 __global__ void __launch_bounds__(256) perm_scatter_kernel(const int64_t* __restrict__ idx,
                                                            int64_t R, int E, int nblk,
                                                            const int* __restrict__ block_counts,
                                                            PermOut o) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ int sm[];
   int* total = sm;                 // [E]
   int* start = total + E;          // [E+1]
@@ -179,36 +217,7 @@ __global__ void __launch_bounds__(256) perm_scatter_kernel(const int64_t* __rest
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) cursor[e] += start[e];
 
-  if (blockIdx.x == 0) {
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-      o.expert_counts[e] = total[e];
-      o.expert_start_indices[e] = start[e];
-      tmp[e] = (total[e] + 127) / 128 * 128;  // padded rows
-      tmp2[e] = (total[e] > 0) ? 1 : 0;
-    }
-    if (threadIdx.x == 0) o.expert_start_indices[E] = start[E];
-    __syncthreads();
-    if (threadIdx.x < 32) warp_exclusive_scan(tmp, o.a_scale_offsets, E);
-    __syncthreads();
-    // active experts: compact with a scan of the flags (reuse tmp for ranks)
-    if (threadIdx.x < 32) warp_exclusive_scan(tmp2, tmp, E);
-    __syncthreads();
-    const int na = tmp[E];
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-      if (total[e] > 0) {
-        o.expert_ids[tmp[e]] = e;
-        tmp2[tmp[e]] = (total[e] + 127) / 128;  // m tiles of the a-th active expert
-      }
-      if (e >= na) o.expert_ids[e] = -1;
-    }
-    if (threadIdx.x == 0) *o.num_active = na;
-    __syncthreads();
-    if (threadIdx.x < 32) warp_exclusive_scan(tmp2, o.tile_offsets, na);
-    __syncthreads();
-    if (threadIdx.x == 0 && na == 0) o.tile_offsets[0] = 0;
-  } else {
-    __syncthreads();
-  }
+  if (blockIdx.x == 0) write_expert_arrays(total, start, tmp, tmp2, E, o);
   __syncthreads();
 
   if (threadIdx.x < 32) {
@@ -231,6 +240,83 @@ __global__ void __launch_bounds__(256) perm_scatter_kernel(const int64_t* __rest
       if (valid && lane == 31 - __clz(peers)) cursor[v] += __popc(peers);
       __syncwarp();
     }
+  }
+}
+
+// Single-launch permutation for small problems (R <= kPermSmallMax slots,
+// E <= kPermSmallMaxE): one block of 32 warps; warp w owns a contiguous run
+// of slots and counts it into its own histogram row; the rows' prefix sums in
+// (expert, warp) order give every warp its first row per expert, so a second
+// ordered pass over each run yields the same stable order as the two-kernel
+// path.
+constexpr int kPermSmallMax = 16384;
+constexpr int kPermSmallMaxE = 256;
+
+__global__ void __launch_bounds__(1024) perm_small_kernel(const int64_t* __restrict__ idx, int R, int E,
+                                                          PermOut o, int* status) {
+  pdl_trigger();
+  pdl_wait();
+  extern __shared__ int sm[];
+  int* hist = sm;                  // [32][E]: counts, then each warp's running cursor
+  int* total = hist + 32 * E;      // [E]
+  int* start = total + E;          // [E+1]
+  int* tmp = start + E + 1;        // [E+1]
+  int* tmp2 = tmp + E + 1;         // [E+1]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const unsigned lt = (1u << lane) - 1u;
+  for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) hist[i] = 0;
+  __syncthreads();
+  const int per = (R + 31) / 32;
+  const int b0 = min(R, warp * per), b1 = min(R, b0 + per);
+  int* my = hist + warp * E;
+  for (int base = b0; base < b1; base += 32) {
+    const int s = base + lane;
+    int v = -1;
+    if (s < b1) {
+      const int64_t x = idx[s];
+      if (x >= 0 && x < E) v = static_cast<int>(x);
+      else if (x != -1) record_error(status, MOE_ERR_BAD_INDEX);
+    }
+    const unsigned peers = __match_any_sync(0xFFFFFFFFu, v >= 0 ? v : E + lane);
+    if (v >= 0 && lane == 31 - __clz(peers)) my[v] += __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int t = 0;
+    for (int w = 0; w < 32; ++w) t += hist[w * E + e];
+    total[e] = t;
+  }
+  __syncthreads();
+  if (threadIdx.x < 32) warp_exclusive_scan(total, start, E);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = start[e];
+    for (int w = 0; w < 32; ++w) {
+      const int c = hist[w * E + e];
+      hist[w * E + e] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  write_expert_arrays(total, start, tmp, tmp2, E, o);
+  for (int base = b0; base < b1; base += 32) {
+    const int s = base + lane;
+    int v = -1;
+    if (s < b1) {
+      const int64_t x = idx[s];
+      if (x >= 0 && x < E) v = static_cast<int>(x);
+    }
+    const unsigned peers = __match_any_sync(0xFFFFFFFFu, v >= 0 ? v : E + lane);
+    int row = -1;
+    if (v >= 0) {
+      row = my[v] + __popc(peers & lt);
+      o.src_info[row] = s;
+    }
+    if (s < b1) o.slot_to_row[s] = row;
+    __syncwarp();
+    if (v >= 0 && lane == 31 - __clz(peers)) my[v] += __popc(peers);
+    __syncwarp();
   }
 }
 
@@ -257,6 +343,8 @@ struct GatherArgs {
 };
 
 __global__ void __launch_bounds__(256) gather_kernel(GatherArgs g, int E) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (r >= g.R) return;
@@ -290,6 +378,8 @@ __global__ void __launch_bounds__(256) gather_kernel(GatherArgs g, int E) {
 }
 
 __global__ void __launch_bounds__(256) zero_kernel(float4* __restrict__ p, int64_t n4) {
+  pdl_trigger();
+  pdl_wait();
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x)
     p[i] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -298,6 +388,8 @@ __global__ void __launch_bounds__(256) zero_kernel(float4* __restrict__ p, int64
 // FP32 accumulator [n] -> BF16, round to nearest even; 8 elements per step.
 __global__ void __launch_bounds__(256) finalize_kernel(const float4* __restrict__ acc,
                                                        uint4* __restrict__ out, int64_t n8) {
+  pdl_trigger();
+  pdl_wait();
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const float4 a = acc[2 * i], b = acc[2 * i + 1];
@@ -313,6 +405,8 @@ __global__ void __launch_bounds__(256) combine_staged_kernel(const float* __rest
                                                              const float* __restrict__ w,
                                                              int64_t M, int H, int k,
                                                              uint4* __restrict__ out) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t n8 = M * (H / 8);
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {

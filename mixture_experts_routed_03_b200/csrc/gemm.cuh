@@ -24,14 +24,17 @@
 // up j0..j0+63 | gate j0+64..j0+127 | up j0+64..j0+127], so each 128-column
 // half of the accumulator holds matching gate and up columns.
 //
-// Roles (320 threads): warp 0 lane 0 issues the copies into a 4-stage ring
-// guarded by mbarriers; warp 1 lane 0 issues the MMAs (M = 128, N = 256, four
-// 32-byte K steps per stage) and commits them; warps 2..9 are the epilogue,
-// two warps per 32-lane TMEM quarter, one per 128-column half, one row per
-// thread.
+// Roles: warp 0 lane 0 issues the copies into a 4-stage ring guarded by
+// mbarriers; warp 1 lane 0 issues the MMAs (M = 128, N = 256, four 32-byte K
+// steps per stage) and commits them; for NVFP4, warp 2 lane 0 moves each
+// stage's scale factors from shared memory into one of two TMEM scale
+// buffers (tcgen05.cp), so their issue cost overlaps the MMAs; the last 8
+// warps are the epilogue, two per 32-lane TMEM quarter, one per 128-column
+// half, one row per thread.
 //
-// Tiles are (active expert, n tile, 128-row m tile), expert-major, m
-// fastest, handed out round-robin over at most one CTA per SM.
+// Tiles are (active expert, n tile, 128-row m tile), handed out round-robin
+// over at most one CTA per SM: expert-major with m fastest for gate_up,
+// n-major for down (see decode_tile).
 //
 // L1 epilogue: h = min(g,c) * sigmoid(min(g,c)) * clamp(u,-c,c) is formed in
 // registers, the accumulator is released, then h is re-quantised (BF16 by
@@ -64,8 +67,11 @@ constexpr int kSFTile = 512;                  // 128 rows x 4 scale bytes
 constexpr int kSFAStage = 4 * kSFTile;        // 4 K-steps of 64 e2m1
 constexpr int kSFBStage = 2 * 4 * kSFTile;    // 2 row blocks x 4 K-steps
 constexpr int kTmemCols = 512;
-constexpr int kSFACol = 256;                  // NVFP4: TMEM columns of the A scales
-constexpr int kSFBCol = 256 + 16;             // NVFP4: TMEM columns of the B scales
+// NVFP4 scale factors in TMEM: two buffers of 48 columns after the
+// accumulator, A scales (16 columns) then B scales (32 columns).
+constexpr int kSFCol0 = 256;
+constexpr int kSFBufCols = 48;
+constexpr int kSFBOff = 16;
 constexpr int kEpiWarps = 8;
 
 // Bytes of one prepared B block (one stage of one tile).
@@ -89,7 +95,10 @@ struct GemmCfg {
   static constexpr int kAccBufs = (FMT == FMT_NVFP4) ? 1 : 2;
   static constexpr int kStageBytes =
       kAStage + kBStage + ((FMT == FMT_NVFP4) ? (kSFBStage + kSFAStage) : 0);
-  static constexpr int kThreads = (2 + kEpiWarps) * 32;
+  // warp 0 producer, warp 1 MMA issuer, (NVFP4) warp 2 scale-factor copier,
+  // then the epilogue warps
+  static constexpr int kFirstEpiWarp = (FMT == FMT_NVFP4) ? 3 : 2;
+  static constexpr int kThreads = (kFirstEpiWarp + kEpiWarps) * 32;
   static constexpr int kBarrierBytes = 4096;
   static constexpr int kXposeStride = 36;   // floats per row of a 32 x 32 transpose buffer
   static constexpr int kXposeBytes = (EPI == EPI_L1) ? 0 : kEpiWarps * 32 * kXposeStride * 4;
@@ -99,6 +108,7 @@ struct GemmCfg {
 struct GemmArgs {
   int k_stages;       // K bytes / 128
   int n_tiles;        // tiles along N: I/128 (L1, 128 h columns per tile) or H/256 (L2)
+  int n_major;        // tile order: 1 n-major, 0 expert-major (see decode_tile)
   int I, H, topk;
   float clamp;
   int fast_math;
@@ -143,18 +153,39 @@ struct TileInfo {
   int n_tile;
 };
 
+// Tile T -> (expert, m tile, n tile).  Expert-major order: concurrent CTAs
+// share one expert's activation panel and weight tiles.  N-major order (the
+// down leg when its whole A operand fits in L2): concurrent CTAs add into the
+// same 256 output columns of every token, a slice of the FP32 accumulator
+// that stays in L2.
 __device__ __forceinline__ void decode_tile(const GemmArgs& p, int na, int T, TileInfo& t) {
   const int nt = p.n_tiles;
-  int lo = 0, hi = na;  // tile_offsets[lo]*nt <= T < tile_offsets[hi]*nt
+  const bool kNMajor = p.n_major != 0;
+  int g, scale;   // search key and the multiplier of tile_offsets
+  if (kNMajor) {
+    const int total_mt = __ldg(p.tile_offsets + na);
+    t.n_tile = T / total_mt;
+    g = T - t.n_tile * total_mt;
+    scale = 1;
+  } else {
+    g = T;
+    scale = nt;
+  }
+  int lo = 0, hi = na;  // tile_offsets[lo]*scale <= g < tile_offsets[hi]*scale
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
-    if (__ldg(p.tile_offsets + mid) * nt <= T) lo = mid; else hi = mid;
+    if (__ldg(p.tile_offsets + mid) * scale <= g) lo = mid; else hi = mid;
   }
   const int mt0 = __ldg(p.tile_offsets + lo);
-  const int nm = __ldg(p.tile_offsets + lo + 1) - mt0;
-  const int local = T - mt0 * nt;
-  t.n_tile = local / nm;
-  const int mt = local - t.n_tile * nm;
+  int mt;
+  if (kNMajor) {
+    mt = g - mt0;
+  } else {
+    const int nm = __ldg(p.tile_offsets + lo + 1) - mt0;
+    const int local = T - mt0 * nt;
+    t.n_tile = local / nm;
+    mt = local - t.n_tile * nm;
+  }
   t.e = __ldg(p.expert_ids + lo);
   const int start = __ldg(p.starts + t.e);
   const int cnt = __ldg(p.starts + t.e + 1) - start;
@@ -212,6 +243,9 @@ __global__ void __launch_bounds__(GemmCfg<FMT, EPI>::kThreads, 1)
   uint64_t* acc_empty = acc_full + NACC;
   uint64_t* final_bar = acc_empty + NACC;
   uint64_t* xbar = final_bar + 1;  // FP8 L1: one per TMEM lane quarter
+  uint64_t* sf_full = xbar + 4;    // NVFP4: scale buffer b holds the current stage's scales
+  uint64_t* sf_empty = sf_full + 2;   // NVFP4: the MMAs reading scale buffer b completed
+  uint64_t* sf_final = sf_empty + 2;  // NVFP4: the copier's last copies completed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S * SB + 512);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* xbuf = reinterpret_cast<float*>(smem + S * SB + 1024);  // FP8 L1: [2][2][128] amax
@@ -231,6 +265,11 @@ __global__ void __launch_bounds__(GemmCfg<FMT, EPI>::kThreads, 1)
     }
     mbar_init(final_bar, 1);
     for (int i = 0; i < 4; ++i) mbar_init(&xbar[i], 64);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sf_full[i], 1);
+      mbar_init(&sf_empty[i], 1);
+    }
+    mbar_init(sf_final, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -240,6 +279,8 @@ __global__ void __launch_bounds__(GemmCfg<FMT, EPI>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_trigger();
+  pdl_wait();   // the layout, activations and accumulator come from earlier kernels
 
   const int na = *p.num_active;
   const int total = (na > 0) ? __ldg(p.tile_offsets + na) * p.n_tiles : 0;
@@ -299,6 +340,8 @@ __global__ void __launch_bounds__(GemmCfg<FMT, EPI>::kThreads, 1)
       int ab = 0;
       uint32_t aphase = 0;
       bool ok = true;
+      int sb = 0;
+      uint32_t sphase = 0;
       for (int T = blockIdx.x; T < total && ok; T += gridDim.x) {
         if (FMT != FMT_FP8) {
           if (!mbar_wait(&acc_empty[ab], aphase ^ 1u, abort_flag, p.status, 2)) break;
@@ -322,16 +365,13 @@ __global__ void __launch_bounds__(GemmCfg<FMT, EPI>::kThreads, 1)
           uint8_t* sbp = sa + kAStage;
           const uint64_t adesc = sdesc_sw128(smem_u32(sa));
           const uint64_t bdesc = sdesc_sw128(smem_u32(sbp));
+          const uint32_t sfa_t = tmem + kSFCol0 + kSFBufCols * sb;
           if (FMT == FMT_NVFP4) {
-            const uint32_t sfb_s = smem_u32(sbp + kBStage);
-            const uint32_t sfa_s = sfb_s + kSFBStage;
-#pragma unroll
-            for (int kc = 0; kc < 4; ++kc) {
-              tmem_copy_sf(tmem + kSFACol + 4 * kc, sdesc_sf_tile(sfa_s + kc * kSFTile));
-              tmem_copy_sf(tmem + kSFBCol + 8 * kc, sdesc_sf_tile(sfb_s + kc * kSFTile));
-              tmem_copy_sf(tmem + kSFBCol + 8 * kc + 4,
-                           sdesc_sf_tile(sfb_s + 4 * kSFTile + kc * kSFTile));
+            if (!mbar_wait(&sf_full[sb], sphase, abort_flag, p.status, 8)) {
+              ok = false;
+              break;
             }
+            tc_fence_after();
           }
 #pragma unroll
           for (int kc = 0; kc < 4; ++kc) {
@@ -340,9 +380,16 @@ __global__ void __launch_bounds__(GemmCfg<FMT, EPI>::kThreads, 1)
             const uint64_t b = bdesc + static_cast<uint64_t>(2 * kc);
             if (FMT == FMT_BF16) mma_f16(d, a, b, kIdesc, acc);
             else if (FMT == FMT_FP8) mma_f8(d, a, b, kIdesc, acc);
-            else mma_nvf4(d, a, b, kIdesc, tmem + kSFACol + 4 * kc, tmem + kSFBCol + 8 * kc, acc);
+            else mma_nvf4(d, a, b, kIdesc, sfa_t + 4 * kc, sfa_t + kSFBOff + 8 * kc, acc);
           }
           mma_commit(&empty[stage]);
+          if (FMT == FMT_NVFP4) {
+            mma_commit(&sf_empty[sb]);
+            if (++sb == 2) {
+              sb = 0;
+              sphase ^= 1u;
+            }
+          }
           if (++stage == S) {
             stage = 0;
             phase ^= 1u;
@@ -367,9 +414,49 @@ __global__ void __launch_bounds__(GemmCfg<FMT, EPI>::kThreads, 1)
       mma_commit(final_bar);
       mbar_drain(final_bar, 0);
     }
-  } else {
+  } else if (FMT == FMT_NVFP4 && warp == 2) {
+    // ------------------------------------------------------------ scale copier
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int sb = 0;
+      uint32_t sphase = 0;
+      for (int T = blockIdx.x; T < total; T += gridDim.x) {
+        bool ok = true;
+        for (int ks = 0; ks < p.k_stages; ++ks) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, p.status, 9) ||
+              !mbar_wait(&sf_empty[sb], sphase ^ 1u, abort_flag, p.status, 10)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sfb_s = smem_u32(smem + stage * SB + kAStage + kBStage);
+          const uint32_t sfa_s = sfb_s + kSFBStage;
+          const uint32_t dst = tmem + kSFCol0 + kSFBufCols * sb;
+#pragma unroll
+          for (int kc = 0; kc < 4; ++kc) {
+            tmem_copy_sf(dst + 4 * kc, sdesc_sf_tile(sfa_s + kc * kSFTile));
+            tmem_copy_sf(dst + kSFBOff + 8 * kc, sdesc_sf_tile(sfb_s + kc * kSFTile));
+            tmem_copy_sf(dst + kSFBOff + 8 * kc + 4, sdesc_sf_tile(sfb_s + 4 * kSFTile + kc * kSFTile));
+          }
+          mma_commit(&sf_full[sb]);
+          if (++sb == 2) {
+            sb = 0;
+            sphase ^= 1u;
+          }
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+      }
+      mma_commit(sf_final);
+      mbar_drain(sf_final, 0);
+    }
+  } else if (warp >= Cfg::kFirstEpiWarp) {
     // ------------------------------------------------------------ epilogue
-    const int ew = warp - 2;
+    const int ew = warp - Cfg::kFirstEpiWarp;
     const int q = warp & 3;               // TMEM lane quarter this warp may access
     const int half = ew >> 2;             // 128-column half of the accumulator
     const int row_local = q * 32 + lane;
@@ -601,6 +688,8 @@ __device__ __forceinline__ int prep_row(const PrepArgs& a, int nt, int r) {
 }
 
 __global__ void __launch_bounds__(256) prepare_weights_kernel(PrepArgs a) {
+  pdl_trigger();
+  pdl_wait();
   const int bb = b_block_bytes(a.fmt);
   const int64_t blocks = static_cast<int64_t>(a.E) * a.n_tiles * a.k_stages;
   const int64_t n16 = blocks * (kBStage / 16);

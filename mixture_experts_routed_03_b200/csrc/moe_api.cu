@@ -8,6 +8,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "aux_kernels.cuh"
 #include "gemm.cuh"
@@ -160,6 +161,25 @@ struct TimScope {
 };
 
 // ---------------------------------------------------------------- launches
+// Every kernel is launched with programmatic stream serialisation: it may be
+// scheduled while the previous kernel of the stream drains, runs its
+// prologue, and waits (griddepcontrol.wait) before touching global memory.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kernel)(KArgs...), int grid, int block, size_t smem, cudaStream_t st,
+                     Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(static_cast<unsigned>(block));
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 int sm_count() {
   int dev = 0, n = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
@@ -199,8 +219,8 @@ bool ensure_init() {
 
 template <int FMT, int EPI>
 cudaError_t launch_gemm(const GemmArgs& a, const CUtensorMap& ta, int grid, cudaStream_t st) {
-  moe_gemm_kernel<FMT, EPI><<<grid, GemmCfg<FMT, EPI>::kThreads, GemmCfg<FMT, EPI>::kSmemBytes, st>>>(a, ta);
-  return cudaGetLastError();
+  return launch_k(moe_gemm_kernel<FMT, EPI>, grid, GemmCfg<FMT, EPI>::kThreads, GemmCfg<FMT, EPI>::kSmemBytes,
+                  st, a, ta);
 }
 
 template <int EPI>
@@ -235,15 +255,14 @@ cudaError_t launch_route(const moe_problem_t* p, const float* logits, const floa
   const int grid = int((M * 32 + 255) / 256);
   const int per = (E + 31) / 32;
   TimScope ts(MOE_SLOT_ROUTE, st);
-#define MOE_ROUTE(PER) route_kernel<PER><<<grid, 256, 0, st>>>(logits, bias, M, E, p->num_topk, idx, w)
-  if (per <= 1) MOE_ROUTE(1);
-  else if (per <= 2) MOE_ROUTE(2);
-  else if (per <= 4) MOE_ROUTE(4);
-  else if (per <= 8) MOE_ROUTE(8);
-  else if (per <= 16) MOE_ROUTE(16);
-  else MOE_ROUTE(32);
+#define MOE_ROUTE(PER) launch_k(route_kernel<PER>, grid, 256, 0, st, logits, bias, M, E, p->num_topk, idx, w)
+  if (per <= 1) return MOE_ROUTE(1);
+  if (per <= 2) return MOE_ROUTE(2);
+  if (per <= 4) return MOE_ROUTE(4);
+  if (per <= 8) return MOE_ROUTE(8);
+  if (per <= 16) return MOE_ROUTE(16);
+  return MOE_ROUTE(32);
 #undef MOE_ROUTE
-  return cudaGetLastError();
 }
 
 cudaError_t launch_permute(const moe_problem_t* p, const int64_t* idx, const PermOut& o, int* block_counts,
@@ -251,11 +270,12 @@ cudaError_t launch_permute(const moe_problem_t* p, const int64_t* idx, const Per
   const int E = p->num_experts;
   const int64_t R = p->num_tokens * p->num_topk;
   TimScope ts(MOE_SLOT_PERMUTE, st);
-  perm_count_kernel<<<nblk, 256, E * sizeof(int), st>>>(idx, R, E, block_counts, status);
-  cudaError_t e = cudaGetLastError();
+  if (R <= kPermSmallMax && E <= kPermSmallMaxE)
+    return launch_k(perm_small_kernel, 1, 1024, (36 * E + 3) * sizeof(int), st, idx, int(R), E, o, status);
+  cudaError_t e = launch_k(perm_count_kernel, nblk, 256, E * sizeof(int), st, idx, R, E, block_counts, status);
   if (e != cudaSuccess) return e;
-  perm_scatter_kernel<<<nblk, 256, (5 * E + 3 + kPermChunk) * sizeof(int), st>>>(idx, R, E, nblk, block_counts, o);
-  return cudaGetLastError();
+  return launch_k(perm_scatter_kernel, nblk, 256, (5 * E + 3 + kPermChunk) * sizeof(int), st, idx, R, E, nblk,
+                  static_cast<const int*>(block_counts), o);
 }
 
 struct FfnBuffers {
@@ -292,9 +312,9 @@ moe_status_t run_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_wei
   g.ld = int(b.P);
   {
     TimScope ts(MOE_SLOT_GATHER, st);
-    gather_kernel<<<grid_for(R * 32, 256, 1 << 30), 256, 0, st>>>(g, E);
+    if (launch_k(gather_kernel, grid_for(R * 32, 256, 1 << 30), 256, 0, st, g, E) != cudaSuccess)
+      return MOE_ERR_CUDA;
   }
-  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
 
   // L1: gate_up
   CUtensorMap ta{};
@@ -341,14 +361,19 @@ moe_status_t run_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_wei
   // L2: down
   if (out_mode == MOE_OUT_ACCUMULATE) {
     TimScope ts(MOE_SLOT_ZERO, st);
-    zero_kernel<<<grid_for(M * H / 4, 256), 256, 0, st>>>(reinterpret_cast<float4*>(out), M * H / 4);
-    if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_k(zero_kernel, grid_for(M * H / 4, 256), 256, 0, st, reinterpret_cast<float4*>(out),
+                 int64_t(M * H / 4)) != cudaSuccess)
+      return MOE_ERR_CUDA;
   }
   CUtensorMap ta2{};
   if (!make_map(&ta2, b.h, h_row_bytes(fmt, I), uint64_t(R), 128)) return MOE_ERR_CUDA;
   GemmArgs a2 = a;
   a2.k_stages = h_row_bytes(fmt, I) / 128;
   a2.n_tiles = H / 256;
+  // n-major keeps one 256-column slice of the FP32 accumulator hot in L2, at
+  // the price of re-reading the whole intermediate once per slice: worth it
+  // while the intermediate fits in L2 with room to spare
+  a2.n_major = (size_t(R) * h_row_bytes(fmt, I) <= (size_t(48) << 20)) ? 1 : 0;
   a2.wB = static_cast<const uint8_t*>(w->w2);
   a2.sfa = b.h_sf;
   a2.sfa_kc = I / 64;
@@ -469,7 +494,9 @@ moe_status_t moe_prepare_weights(const moe_problem_t* p, const moe_weights_t* lo
   a.n_tiles = I / 128;
   a.k_stages = a.Kb / 128;
   a.l1 = 1;
-  prepare_weights_kernel<<<grid_for(int64_t(prepared_bytes(p, true)) / 16, 256), 256, 0, st>>>(a);
+  if (launch_k(prepare_weights_kernel, grid_for(int64_t(prepared_bytes(p, true)) / 16, 256), 256, 0, st, a) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
   // down: H rows, K = I
   a.w = static_cast<const uint8_t*>(logical->w2);
   a.sf = static_cast<const uint8_t*>(logical->w2_scale);
@@ -480,8 +507,10 @@ moe_status_t moe_prepare_weights(const moe_problem_t* p, const moe_weights_t* lo
   a.n_tiles = H / 256;
   a.k_stages = a.Kb / 128;
   a.l1 = 0;
-  prepare_weights_kernel<<<grid_for(int64_t(prepared_bytes(p, false)) / 16, 256), 256, 0, st>>>(a);
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  return launch_k(prepare_weights_kernel, grid_for(int64_t(prepared_bytes(p, false)) / 16, 256), 256, 0, st, a) ==
+                 cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
 }
 
 moe_status_t moe_route(const moe_problem_t* p, const float* logits, const float* bias, int64_t* topk_idx,
@@ -558,16 +587,17 @@ moe_status_t moe_combine(const moe_problem_t* p, const moe_layout_t* layout, con
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int64_t M = p->num_tokens, H = p->hidden;
   TimScope ts(in_mode == MOE_IN_ACCUMULATED ? MOE_SLOT_FINALIZE : MOE_SLOT_COMBINE, st);
+  cudaError_t e;
   if (in_mode == MOE_IN_ACCUMULATED) {
-    finalize_kernel<<<grid_for(M * H / 8, 256), 256, 0, st>>>(static_cast<const float4*>(in),
-                                                             static_cast<uint4*>(out_bf16), M * H / 8);
+    e = launch_k(finalize_kernel, grid_for(M * H / 8, 256), 256, 0, st, static_cast<const float4*>(in),
+                 static_cast<uint4*>(out_bf16), int64_t(M * H / 8));
   } else {
     if (!layout || !layout->slot_to_row || !topk_weights) return MOE_ERR_INVALID_ARG;
-    combine_staged_kernel<<<grid_for(M * H / 8, 256), 256, 0, st>>>(
-        static_cast<const float*>(in), layout->slot_to_row, topk_weights, M, int(H), p->num_topk,
-        static_cast<uint4*>(out_bf16));
+    e = launch_k(combine_staged_kernel, grid_for(M * H / 8, 256), 256, 0, st, static_cast<const float*>(in),
+                 static_cast<const int*>(layout->slot_to_row), topk_weights, M, int(H), p->num_topk,
+                 static_cast<uint4*>(out_bf16));
   }
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 moe_status_t moe_fused(const moe_problem_t* p, const moe_act_t* act, const moe_weights_t* w,
@@ -622,9 +652,10 @@ moe_status_t moe_fused(const moe_problem_t* p, const moe_act_t* act, const moe_w
   if ((s = run_ffn(p, act, w, b, wts, MOE_OUT_ACCUMULATE, acc, st)) != MOE_OK) return s;
   const int64_t M = p->num_tokens, H = p->hidden;
   TimScope ts(MOE_SLOT_FINALIZE, st);
-  finalize_kernel<<<grid_for(M * H / 8, 256), 256, 0, st>>>(reinterpret_cast<const float4*>(acc),
-                                                           static_cast<uint4*>(out_bf16), M * H / 8);
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  return launch_k(finalize_kernel, grid_for(M * H / 8, 256), 256, 0, st, reinterpret_cast<const float4*>(acc),
+                  static_cast<uint4*>(out_bf16), int64_t(M * H / 8)) == cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
 }
 
 moe_status_t moe_timing_enable(int enable, int max_calls) {
