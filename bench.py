@@ -51,6 +51,9 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--chain", action="store_true",
+                    help="time the multi-launch chain moe_route/moe_permute/moe_ffn/moe_combine "
+                         "instead of the single moe_fused launch (per-kernel breakdown)")
     ap.add_argument("--set", action="append", default=[], metavar="KEY=VALUE",
                     help="override a workload field (a smaller case for profiling)")
     return ap.parse_args()
@@ -63,6 +66,33 @@ def workload(args):
         k, v = kv.split("=", 1)
         over[k] = type(workloads.WORKLOADS[args.workload].get(k, 0))(v) if k in workloads.WORKLOADS[args.workload] else float(v)
     return workloads.problem(args.workload, **over)
+
+
+def kernel_sources_sha():
+    """SHA-256 over the CUDA sources and the C header (identifies the kernels
+    a stored ncu traffic figure was measured on)."""
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "mixture_experts_routed_03_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            h.update(name.encode())
+            h.update(open(os.path.join(csrc, name), "rb").read())
+    h.update(open(os.path.join(ROOT, "include", "moe.h"), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def stored_traffic(workload, kernel):
+    """DRAM bytes per launch of `kernel` on `workload` from profiles/traffic.json,
+    or None when absent or measured on other kernel sources."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f)[workload]
+    except Exception:
+        return None
+    if rec.get("kernel") != kernel or rec.get("sources_sha") != kernel_sources_sha():
+        return None
+    return float(rec["dram_bytes_per_launch"])
 
 
 def load_peaks():
@@ -191,8 +221,26 @@ def run_ours(args, rank, world, local_rank):
     out = torch.empty((M, p["hidden"]), dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream()
 
-    def step():
+    lay = layer.LayoutBuffers(M, k, p["num_experts"], dev) if args.chain else None
+    acc = torch.empty((M, p["hidden"]), dtype=torch.float32, device=dev) if args.chain else None
+    ridx = torch.empty((M, k), dtype=torch.int64, device=dev) if args.chain and routed else None
+    rw = torch.empty((M, k), dtype=torch.float32, device=dev) if args.chain and routed else None
+
+    def chain():
+        prob = L.problem(M)
+        idx, w = d.get("topk_idx"), d.get("topk_weights")
         if routed:
+            api.route(prob, d["logits"], d["bias"], ridx, rw)
+            idx, w = ridx, rw
+        api.permute(prob, idx, lay.struct, L.ws, L.ws_bytes)
+        api.ffn(prob, api.act(d["x"], d["x_scale"]), L.weights, lay.struct, w, api.MOE_OUT_ACCUMULATE, acc,
+                L.ws, L.ws_bytes)
+        api.combine(prob, lay.struct, w, acc, api.MOE_IN_ACCUMULATED, out)
+
+    def step():
+        if args.chain:
+            chain()
+        elif routed:
             L.forward(d["x"], d["x_scale"], logits=d["logits"], bias=d["bias"], out=out)
         else:
             L.forward(d["x"], d["x_scale"], topk_idx=d["topk_idx"], topk_weights=d["topk_weights"], out=out)
@@ -225,6 +273,11 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     per_step = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     kern = api.timing_read()
+    # the single launch's phase boundaries of the last step (workspace header)
+    ts = L.ws[64:128].view(torch.int64).cpu().tolist()
+    names = ("route", "permute", "gather+zero", "gemm1", "gemm2", "finalize")
+    phases = ({n: (ts[i + 1] - ts[i]) / 1e3 for i, n in enumerate(names)}
+              if not args.chain and ts[6] > ts[0] else None)
     api.timing_enable(False, 0)
     L.check_status()
     t_ms = sum(per_step)
@@ -277,7 +330,7 @@ def run_ours(args, rank, world, local_rank):
         tt = torch.tensor([t_ms, e2e_ms], device=dev, dtype=torch.float64)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
         t_ms, e2e_ms = float(tt[0]), float(tt[1])
-    return dict(p=p, t_ms=t_ms, per_step=per_step, kern=kern, launches=launches, e2e_ms=e2e_ms,
+    return dict(p=p, t_ms=t_ms, per_step=per_step, kern=kern, launches=launches, e2e_ms=e2e_ms, phases=phases,
                 h2d=h2d, d2h=d2h, num_active=num_active, clocks=clocks.summary(), R=R, M=M,
                 host_inputs=(d, L) if rank == 0 else None)
 
@@ -337,17 +390,22 @@ def main_ours(args):
     wm = work_model(p, r["num_active"])
     kern = r["kern"]
     step_ms = r["t_ms"] / args.steps
-    # dominant kernel of the step
-    slot = max(("gemm1", "gemm2"), key=lambda s: kern[s][0])
+    # dominant kernel of the step: the single moe_fused launch (whose
+    # algorithmic work is the whole layer's), or the larger GEMM of a chain
+    if kern.get("fused", (0.0, 0))[1]:
+        slot, work = "fused", wm["layer"]
+    else:
+        slot = max(("gemm1", "gemm2"), key=lambda s: kern[s][0])
+        work = wm[slot]
     k_ms = kern[slot][0] / max(kern[slot][1], 1)
     bound = BOUND.get(args.workload, "hbm")
     if bound == "tensor":
         peak = peaks["bf16_tflops"] * FMT_TENSOR_RATIO[p["format"]]
-        achieved = wm[slot]["flops"] / (k_ms / 1e3) / 1e12
+        achieved = work["flops"] / (k_ms / 1e3) / 1e12
         unit = "TFLOP/s"
     else:
         peak = peaks["hbm_gbs"]
-        achieved = wm[slot]["bytes"] / (k_ms / 1e3) / 1e9
+        achieved = work["bytes"] / (k_ms / 1e3) / 1e9
         unit = "GB/s"
     total_k = sum(v[0] for v in kern.values()) or 1.0
     line = {
@@ -365,6 +423,7 @@ def main_ours(args):
                   "nvfp4": "e2m1+e4m3 scales (f32 accumulate)"}[p["format"]],
         "data": "synthetic (seeded torch generators; random-init experts of the workload's shapes)",
         "config": {"workload": args.workload + ("" if not args.set else " (" + ",".join(args.set) + ")"),
+                   "path": "multi-launch chain" if args.chain else "moe_fused (one launch)",
                    "num_tokens": p["num_tokens"], "hidden": p["hidden"],
                    "intermediate_hidden": p["intermediate_hidden"], "num_experts": p["num_experts"],
                    "num_topk": p["num_topk"], "format": p["format"], "routing": p["routing"],
@@ -373,11 +432,15 @@ def main_ours(args):
         "tokens_per_s": p["num_tokens"] * world * args.steps / (r["t_ms"] / 1e3),
         "layer_tflops": wm["layer"]["flops"] / (step_ms / 1e3) / 1e12,
         "layer_gbs": wm["layer"]["bytes"] / (step_ms / 1e3) / 1e9,
-        "roofline": {"kernel": slot, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-                     "frac": achieved / peak, "traffic": None,
+        "roofline": {"kernel": {"fused": "moe_fused_kernel", "gemm1": "moe_gemm_kernel (gate_up)",
+                                "gemm2": "moe_gemm_kernel (down)"}[slot], "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                     "frac": achieved / peak,
+                     "traffic": stored_traffic(args.workload, {"fused": "moe_fused_kernel", "gemm1": "gemm1",
+                                                              "gemm2": "gemm2"}[slot]) if not args.set else None,
                      "peak_source": f"{peak_src} ({'bf16 burst x nominal ' + p['format'] + ' ratio' if bound == 'tensor' else 'hbm copy'})",
                      "kernel_ms": k_ms},
         "kernels_ms": {s: v[0] / max(v[1], 1) for s, v in kern.items() if v[1]},
+        "fused_phases_us": r["phases"],
         "kernel_share": {s: v[0] / total_k for s, v in kern.items() if v[1]},
         "gpu_launches": r["launches"],
         "e2e": {"value": e2e_value, "unit": "routed_tokens/s", "h2d_bytes_per_step": r["h2d"],

@@ -268,7 +268,8 @@ moe_status_t moe_fused(const moe_problem_t* problem, const moe_act_t* act,
 #define MOE_SLOT_GEMM2 5
 #define MOE_SLOT_FINALIZE 6
 #define MOE_SLOT_COMBINE 7
-#define MOE_NUM_SLOTS 8
+#define MOE_SLOT_FUSED 8   /* the single moe_fused launch */
+#define MOE_NUM_SLOTS 9
 moe_status_t moe_timing_enable(int enable, int max_calls);
 moe_status_t moe_timing_read(float* ms /* [MOE_NUM_SLOTS] */, int* launches /* [MOE_NUM_SLOTS] */);
 

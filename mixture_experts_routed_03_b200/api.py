@@ -41,7 +41,7 @@ EXPORTS = (
     "moe_fused", "moe_read_status", "moe_status_string", "moe_timing_enable", "moe_timing_read",
 )
 
-SLOTS = ("route", "permute", "gather", "gemm1", "zero", "gemm2", "finalize", "combine")
+SLOTS = ("route", "permute", "gather", "gemm1", "zero", "gemm2", "finalize", "combine", "fused")
 
 
 class MoEError(RuntimeError):

@@ -15,7 +15,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 OUT = os.path.join(HERE, "libmoe_b200.so")
 SOURCES = ["moe_api.cu"]
-DEPS = ["moe_api.cu", "gemm.cuh", "aux_kernels.cuh", "common.cuh"]
+DEPS = ["moe_api.cu", "gemm.cuh", "aux_kernels.cuh", "common.cuh", "fused.cuh"]
 HEADER = os.path.join(os.path.dirname(HERE), "include", "moe.h")
 
 NVCC_FLAGS = [

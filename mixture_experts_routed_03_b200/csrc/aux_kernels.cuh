@@ -1,7 +1,11 @@
 // aux_kernels.cuh -- the memory-bound steps around the expert GEMMs:
 // routing from logits, the counting-sort permutation, the activation gather
 // into expert order, accumulator zeroing, the BF16 finalise and the staged
-// (deterministic) combine, and the one-time NVFP4 scale-tile preparation.
+// (deterministic) combine.
+//
+// Each step is a __device__ function over a "virtual block" (an index and the
+// calling block's threads), wrapped by a small __global__ kernel; the
+// single-launch fused kernel calls the same functions between grid barriers.
 #pragma once
 
 #include "common.cuh"
@@ -16,6 +20,15 @@ namespace moe {
 // lower id on ties; NaN scores map to the smallest key.  The weights are the
 // softmax of the unbiased logits over the chosen k.
 // ---------------------------------------------------------------------------
+struct RouteArgs {
+  const float* logits;   // [M][E]
+  const float* bias;     // [E] or null
+  int64_t M;
+  int E, k;
+  int64_t* idx_out;      // [M][k]
+  float* w_out;          // [M][k]
+};
+
 __device__ __forceinline__ uint64_t route_key(float s, int e) {
   if (s == 0.0f) s = 0.0f;  // -0 and +0 are the same score
   const uint32_t b = __float_as_uint(s);
@@ -23,26 +36,19 @@ __device__ __forceinline__ uint64_t route_key(float s, int e) {
   return (static_cast<uint64_t>(ord) << 32) | static_cast<uint32_t>(0xFFFFFFFFu - e);
 }
 
+// Routes token t with the calling (full) warp.
 template <int PER>
-__global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits,
-                                                    const float* __restrict__ bias, int64_t M,
-                                                    int E, int k, int64_t* __restrict__ idx_out,
-                                                    float* __restrict__ w_out) {
-  pdl_trigger();
-  pdl_wait();
-  const int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (t >= M) return;
-  const float* row = logits + t * E;
+__device__ __forceinline__ void route_token(const RouteArgs& a, int64_t t, int lane) {
+  const float* row = a.logits + t * a.E;
   uint64_t key[PER];
 #pragma unroll
   for (int i = 0; i < PER; ++i) {
     const int e = lane + 32 * i;
     key[i] = 0;
-    if (e < E) key[i] = route_key(__fadd_rn(row[e], bias ? bias[e] : 0.0f), e);
+    if (e < a.E) key[i] = route_key(__fadd_rn(row[e], a.bias ? a.bias[e] : 0.0f), e);
   }
   int my_e = 0;
-  for (int j = 0; j < k; ++j) {
+  for (int j = 0; j < a.k; ++j) {
     uint64_t best = 0;
     int bi = 0;
 #pragma unroll
@@ -63,7 +69,7 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
       if (i == bi && best == m) key[i] = 0;
     if (lane == j) my_e = e;
   }
-  const bool mine = lane < k;
+  const bool mine = lane < a.k;
   const float l = mine ? row[my_e] : -INFINITY;
   float mx = l;
 #pragma unroll
@@ -73,46 +79,50 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
 #pragma unroll
   for (int off = 16; off; off >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, off);
   if (mine) {
-    idx_out[t * k + lane] = my_e;
-    w_out[t * k + lane] = __fdiv_rn(ex, sum);
+    a.idx_out[t * a.k + lane] = my_e;
+    a.w_out[t * a.k + lane] = __fdiv_rn(ex, sum);
   }
+}
+
+// Tokens warp_id, warp_id + nwarps, ... (all lanes of the calling warp).
+__device__ __forceinline__ void route_tokens(const RouteArgs& a, int64_t warp_id, int64_t nwarps, int lane) {
+  const int per = (a.E + 31) / 32;
+  for (int64_t t = warp_id; t < a.M; t += nwarps) {
+    if (per <= 1) route_token<1>(a, t, lane);
+    else if (per <= 2) route_token<2>(a, t, lane);
+    else if (per <= 4) route_token<4>(a, t, lane);
+    else if (per <= 8) route_token<8>(a, t, lane);
+    else if (per <= 16) route_token<16>(a, t, lane);
+    else route_token<32>(a, t, lane);
+  }
+}
+
+__global__ void __launch_bounds__(256) route_kernel(RouteArgs a) {
+  pdl_trigger();
+  pdl_wait();
+  const int64_t nw = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  route_tokens(a, (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5, nw, threadIdx.x & 31);
 }
 
 // ---------------------------------------------------------------------------
 // Permutation (Struct_mega_ffn_ep_combine_send: expert_start_indices,
 // expert_ids, a_scale_offsets, src_info, num_active_experts): a stable
 // counting sort of the flat slots s = t*k + j by expert.
-//   pass 1: per 1024-slot chunk, count slots per expert (shared atomics)
-//   pass 2: per chunk, the expert totals and this chunk's offset within each
-//           expert give every slot its row; one warp walks the chunk in
-//           order, ranking equal experts inside each 32-slot round with
-//           __match_any_sync, so rows ascend in slot index.  Chunk 0 also
-//           writes the per-expert arrays and the GEMM tile table.
+//   small problems: one block; warp w owns a contiguous run of slots and
+//           counts it into its own histogram row; the rows' prefix sums in
+//           (expert, warp) order give every warp its first row per expert,
+//           and a second ordered pass over each run writes the rows.
+//   large problems, pass 1: per 1024-slot chunk, count slots per expert.
+//   large problems, pass 2: per chunk, the expert totals and this chunk's
+//           offset within each expert give every slot its row; one warp walks
+//           the chunk in order, ranking equal experts inside each 32-slot
+//           round with __match_any_sync, so rows ascend in slot index.
+// Chunk 0 (or the one block) also writes the per-expert arrays and the GEMM
+// tile table.
 // ---------------------------------------------------------------------------
 constexpr int kPermChunk = 1024;
-
-__global__ void __launch_bounds__(256) perm_count_kernel(const int64_t* __restrict__ idx,
-                                                         int64_t R, int E,
-                                                         int* __restrict__ block_counts,
-                                                         int* status) {
-  pdl_trigger();
-  pdl_wait();
-  extern __shared__ int cnt[];
-  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
-  __syncthreads();
-  const int64_t base = static_cast<int64_t>(blockIdx.x) * kPermChunk;
-  for (int i = threadIdx.x; i < kPermChunk; i += blockDim.x) {
-    const int64_t s = base + i;
-    if (s < R) {
-      const int64_t v = idx[s];
-      if (v >= 0 && v < E) atomicAdd(&cnt[v], 1);
-      else if (v != -1) record_error(status, MOE_ERR_BAD_INDEX);
-    }
-  }
-  __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x)
-    block_counts[static_cast<size_t>(blockIdx.x) * E + e] = cnt[e];
-}
+constexpr int kPermSmallMax = 16384;
+constexpr int kPermSmallMaxE = 256;
 
 struct PermOut {
   int* expert_counts;
@@ -124,6 +134,24 @@ struct PermOut {
   int* a_scale_offsets;
   int* tile_offsets;
 };
+
+struct PermArgs {
+  const int64_t* idx;    // [R]
+  int64_t R;
+  int E;
+  int nblk;              // chunks of kPermChunk slots
+  int* block_counts;     // [nblk][E]
+  PermOut o;
+  int* status;
+};
+
+__host__ __device__ inline bool perm_small_case(int64_t R, int E) {
+  return R <= kPermSmallMax && E <= kPermSmallMaxE;
+}
+
+// Shared-memory ints of the two-pass (per chunk) and the one-block permutation.
+__host__ __device__ inline int perm_chunk_smem_ints(int E) { return 5 * E + 3 + kPermChunk; }
+__host__ __device__ inline int perm_small_smem_ints(int E, int nwarps) { return nwarps * E + 4 * E + 3; }
 
 // Exclusive scan of v[0..n) by one warp (n <= 1024); writes out[0..n] (n+1
 // entries, out[n] = total).  Each lane owns a contiguous run of entries.
@@ -177,37 +205,54 @@ __device__ void write_expert_arrays(const int* total, const int* start, int* tmp
   if (threadIdx.x == 0) *o.num_active = na;
   __syncthreads();
   if (threadIdx.x < 32) warp_exclusive_scan(tmp2, o.tile_offsets, na);
+  __syncthreads();
 }
 
-__global__ void __launch_bounds__(256) perm_scatter_kernel(const int64_t* __restrict__ idx,
-                                                           int64_t R, int E, int nblk,
-                                                           const int* __restrict__ block_counts,
-                                                           PermOut o) {
-  pdl_trigger();
-  pdl_wait();
-  extern __shared__ int sm[];
+// Pass 1 of the large case for chunk c.
+__device__ void perm_count_chunk(const PermArgs& a, int c, int* sm) {
+  int* cnt = sm;
+  for (int e = threadIdx.x; e < a.E; e += blockDim.x) cnt[e] = 0;
+  __syncthreads();
+  const int64_t base = static_cast<int64_t>(c) * kPermChunk;
+  for (int i = threadIdx.x; i < kPermChunk; i += blockDim.x) {
+    const int64_t s = base + i;
+    if (s < a.R) {
+      const int64_t v = a.idx[s];
+      if (v >= 0 && v < a.E) atomicAdd(&cnt[v], 1);
+      else if (v != -1) record_error(a.status, MOE_ERR_BAD_INDEX);
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < a.E; e += blockDim.x)
+    a.block_counts[static_cast<size_t>(c) * a.E + e] = cnt[e];
+  __syncthreads();
+}
+
+// Pass 2 of the large case for chunk c.
+__device__ void perm_scatter_chunk(const PermArgs& a, int c, int* sm) {
+  const int E = a.E;
   int* total = sm;                 // [E]
   int* start = total + E;          // [E+1]
   int* cursor = start + E + 1;     // [E]
   int* tmp = cursor + E;           // [E+1]
   int* tmp2 = tmp + E + 1;         // [E+1]
   int* sidx = tmp2 + E + 1;        // [kPermChunk] this chunk's expert ids
-  const int64_t base = static_cast<int64_t>(blockIdx.x) * kPermChunk;
+  const int64_t base = static_cast<int64_t>(c) * kPermChunk;
   for (int i = threadIdx.x; i < kPermChunk; i += blockDim.x) {
     const int64_t s = base + i;
     int v = -1;
-    if (s < R) {
-      const int64_t x = idx[s];
+    if (s < a.R) {
+      const int64_t x = a.idx[s];
       v = (x >= 0 && x < E) ? static_cast<int>(x) : -1;
     }
     sidx[i] = v;
   }
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     int tot = 0, before = 0;
-    for (int b = 0; b < nblk; ++b) {
-      const int c = block_counts[static_cast<size_t>(b) * E + e];
-      tot += c;
-      if (b < static_cast<int>(blockIdx.x)) before += c;
+    for (int b = 0; b < a.nblk; ++b) {
+      const int n = a.block_counts[static_cast<size_t>(b) * E + e];
+      tot += n;
+      if (b < c) before += n;
     }
     total[e] = tot;
     cursor[e] = before;
@@ -216,66 +261,55 @@ __global__ void __launch_bounds__(256) perm_scatter_kernel(const int64_t* __rest
   if (threadIdx.x < 32) warp_exclusive_scan(total, start, E);
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) cursor[e] += start[e];
-
-  if (blockIdx.x == 0) write_expert_arrays(total, start, tmp, tmp2, E, o);
+  if (c == 0) write_expert_arrays(total, start, tmp, tmp2, E, a.o);
   __syncthreads();
-
   if (threadIdx.x < 32) {
     const int lane = threadIdx.x;
     const unsigned lt = (1u << lane) - 1u;
     for (int rnd = 0; rnd < kPermChunk / 32; ++rnd) {
       const int64_t s = base + rnd * 32 + lane;
-      if (base + rnd * 32 >= R) break;
+      if (base + rnd * 32 >= a.R) break;
       const int v = sidx[rnd * 32 + lane];
       const bool valid = v >= 0;
-      const int key = valid ? v : (E + lane);
-      const unsigned peers = __match_any_sync(0xFFFFFFFFu, key);
+      const unsigned peers = __match_any_sync(0xFFFFFFFFu, valid ? v : (E + lane));
       int row = -1;
       if (valid) {
         row = cursor[v] + __popc(peers & lt);
-        o.src_info[row] = static_cast<int>(s);
+        a.o.src_info[row] = static_cast<int>(s);
       }
-      if (s < R) o.slot_to_row[s] = row;
+      if (s < a.R) a.o.slot_to_row[s] = row;
       __syncwarp();
       if (valid && lane == 31 - __clz(peers)) cursor[v] += __popc(peers);
       __syncwarp();
     }
   }
+  __syncthreads();
 }
 
-// Single-launch permutation for small problems (R <= kPermSmallMax slots,
-// E <= kPermSmallMaxE): one block of 32 warps; warp w owns a contiguous run
-// of slots and counts it into its own histogram row; the rows' prefix sums in
-// (expert, warp) order give every warp its first row per expert, so a second
-// ordered pass over each run yields the same stable order as the two-kernel
-// path.
-constexpr int kPermSmallMax = 16384;
-constexpr int kPermSmallMaxE = 256;
-
-__global__ void __launch_bounds__(1024) perm_small_kernel(const int64_t* __restrict__ idx, int R, int E,
-                                                          PermOut o, int* status) {
-  pdl_trigger();
-  pdl_wait();
-  extern __shared__ int sm[];
-  int* hist = sm;                  // [32][E]: counts, then each warp's running cursor
-  int* total = hist + 32 * E;      // [E]
+// The whole small case in the calling block.
+__device__ void perm_small_block(const PermArgs& a, int* sm) {
+  const int E = a.E;
+  const int R = static_cast<int>(a.R);
+  const int nw = blockDim.x >> 5;
+  int* hist = sm;                  // [nw][E]: counts, then each warp's running cursor
+  int* total = hist + nw * E;      // [E]
   int* start = total + E;          // [E+1]
   int* tmp = start + E + 1;        // [E+1]
   int* tmp2 = tmp + E + 1;         // [E+1]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const unsigned lt = (1u << lane) - 1u;
-  for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) hist[i] = 0;
+  for (int i = threadIdx.x; i < nw * E; i += blockDim.x) hist[i] = 0;
   __syncthreads();
-  const int per = (R + 31) / 32;
+  const int per = (R + nw - 1) / nw;
   const int b0 = min(R, warp * per), b1 = min(R, b0 + per);
   int* my = hist + warp * E;
   for (int base = b0; base < b1; base += 32) {
     const int s = base + lane;
     int v = -1;
     if (s < b1) {
-      const int64_t x = idx[s];
+      const int64_t x = a.idx[s];
       if (x >= 0 && x < E) v = static_cast<int>(x);
-      else if (x != -1) record_error(status, MOE_ERR_BAD_INDEX);
+      else if (x != -1) record_error(a.status, MOE_ERR_BAD_INDEX);
     }
     const unsigned peers = __match_any_sync(0xFFFFFFFFu, v >= 0 ? v : E + lane);
     if (v >= 0 && lane == 31 - __clz(peers)) my[v] += __popc(peers);
@@ -284,7 +318,7 @@ __global__ void __launch_bounds__(1024) perm_small_kernel(const int64_t* __restr
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     int t = 0;
-    for (int w = 0; w < 32; ++w) t += hist[w * E + e];
+    for (int w = 0; w < nw; ++w) t += hist[w * E + e];
     total[e] = t;
   }
   __syncthreads();
@@ -292,32 +326,54 @@ __global__ void __launch_bounds__(1024) perm_small_kernel(const int64_t* __restr
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     int run = start[e];
-    for (int w = 0; w < 32; ++w) {
+    for (int w = 0; w < nw; ++w) {
       const int c = hist[w * E + e];
       hist[w * E + e] = run;
       run += c;
     }
   }
   __syncthreads();
-  write_expert_arrays(total, start, tmp, tmp2, E, o);
+  write_expert_arrays(total, start, tmp, tmp2, E, a.o);
   for (int base = b0; base < b1; base += 32) {
     const int s = base + lane;
     int v = -1;
     if (s < b1) {
-      const int64_t x = idx[s];
+      const int64_t x = a.idx[s];
       if (x >= 0 && x < E) v = static_cast<int>(x);
     }
     const unsigned peers = __match_any_sync(0xFFFFFFFFu, v >= 0 ? v : E + lane);
     int row = -1;
     if (v >= 0) {
       row = my[v] + __popc(peers & lt);
-      o.src_info[row] = s;
+      a.o.src_info[row] = s;
     }
-    if (s < b1) o.slot_to_row[s] = row;
+    if (s < b1) a.o.slot_to_row[s] = row;
     __syncwarp();
     if (v >= 0 && lane == 31 - __clz(peers)) my[v] += __popc(peers);
     __syncwarp();
   }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(256) perm_count_kernel(PermArgs a) {
+  pdl_trigger();
+  pdl_wait();
+  extern __shared__ int sm[];
+  perm_count_chunk(a, blockIdx.x, sm);
+}
+
+__global__ void __launch_bounds__(256) perm_scatter_kernel(PermArgs a) {
+  pdl_trigger();
+  pdl_wait();
+  extern __shared__ int sm[];
+  perm_scatter_chunk(a, blockIdx.x, sm);
+}
+
+__global__ void __launch_bounds__(1024) perm_small_kernel(PermArgs a) {
+  pdl_trigger();
+  pdl_wait();
+  extern __shared__ int sm[];
+  perm_small_block(a, sm);
 }
 
 // ---------------------------------------------------------------------------
@@ -332,6 +388,7 @@ struct GatherArgs {
   const int* starts;
   const int* a_scale_offsets;
   int64_t R;                 // rows allocated (M*k)
+  int E;
   int row_bytes;
   int topk;
   int H;
@@ -342,27 +399,50 @@ struct GatherArgs {
   int ld;                    // padded rows allocated
 };
 
-__global__ void __launch_bounds__(256) gather_kernel(GatherArgs g, int E) {
-  pdl_trigger();
-  pdl_wait();
-  const int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (r >= g.R) return;
-  if (r >= g.starts[E]) return;  // rows past the valid slots
-  const int s = g.src_info[r];
-  const int64_t t = s / g.topk;
+// Token and padded scale row of routed row r.
+__device__ __forceinline__ void gather_locate(const GatherArgs& g, int64_t r, int64_t& t, int& pr) {
+  t = g.src_info[r] / g.topk;
   // the expert owning row r: starts[e] <= r < starts[e+1]
-  int lo = 0, hi = E;
+  int lo = 0, hi = g.E;
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
     if (g.starts[mid] <= r) lo = mid; else hi = mid;
   }
-  const int e = lo;
-  const int pr = g.a_scale_offsets[e] + static_cast<int>(r - g.starts[e]);
+  pr = g.a_scale_offsets[lo] + static_cast<int>(r - g.starts[lo]);
+}
+
+// Copies rows r0 and r1 (r1 < 0: none) of x into expert order with all of a
+// lane's loads of both 4 KB slices in flight before any store.
+__device__ __forceinline__ void gather_copy2(const GatherArgs& g, int64_t r0, int64_t t0, int64_t r1, int64_t t1,
+                                             int lane) {
   const int nvec = g.row_bytes / 16;
-  const uint4* src = reinterpret_cast<const uint4*>(g.x + t * g.row_bytes);
-  uint4* dst = reinterpret_cast<uint4*>(g.x_perm + r * g.row_bytes);
-  for (int i = lane; i < nvec; i += 32) dst[i] = src[i];
+  const uint4* __restrict__ s0 = reinterpret_cast<const uint4*>(g.x + t0 * g.row_bytes);
+  const uint4* __restrict__ s1 = reinterpret_cast<const uint4*>(g.x + (r1 >= 0 ? t1 : t0) * g.row_bytes);
+  uint4* __restrict__ d0 = reinterpret_cast<uint4*>(g.x_perm + r0 * g.row_bytes);
+  uint4* __restrict__ d1 = reinterpret_cast<uint4*>(g.x_perm + (r1 >= 0 ? r1 : r0) * g.row_bytes);
+  for (int i0 = 0; i0 < nvec; i0 += 256) {
+    uint4 v0[8], v1[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int i = i0 + lane + 32 * j;
+      if (i < nvec) {
+        v0[j] = __ldg(s0 + i);
+        if (r1 >= 0) v1[j] = __ldg(s1 + i);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int i = i0 + lane + 32 * j;
+      if (i < nvec) {
+        d0[i] = v0[j];
+        if (r1 >= 0) d1[i] = v1[j];
+      }
+    }
+  }
+}
+
+// The block scales of routed row r (token t, padded scale row pr).
+__device__ __forceinline__ void gather_scales(const GatherArgs& g, int64_t t, int pr, int lane) {
   if (g.fmt == 1) {
     const float* xs = static_cast<const float*>(g.x_scale) + t * (g.H / 128);
     for (int kb = lane; kb < g.H / 128; kb += 32) g.sa_t[static_cast<size_t>(kb) * g.ld + pr] = xs[kb];
@@ -377,25 +457,71 @@ __global__ void __launch_bounds__(256) gather_kernel(GatherArgs g, int E) {
   }
 }
 
+// Rows warp_id, warp_id + nwarps, ... below the number of valid slots, ROWS
+// rows per step (2 when few warps per SM must keep enough bytes in flight).
+template <int ROWS>
+__device__ __forceinline__ void gather_rows(const GatherArgs& g, int64_t warp_id, int64_t nwarps, int lane) {
+  const int64_t valid = g.starts[g.E];
+  for (int64_t r0 = warp_id; r0 < valid; r0 += ROWS * nwarps) {
+    const int64_t r1 = (ROWS == 2 && r0 + nwarps < valid) ? r0 + nwarps : -1;
+    int64_t t0, t1 = 0;
+    int p0, p1 = 0;
+    gather_locate(g, r0, t0, p0);
+    if (r1 >= 0) gather_locate(g, r1, t1, p1);
+    gather_copy2(g, r0, t0, r1, t1, lane);
+    gather_scales(g, t0, p0, lane);
+    if (r1 >= 0) gather_scales(g, t1, p1, lane);
+  }
+}
+
+__global__ void __launch_bounds__(256) gather_kernel(GatherArgs g) {
+  pdl_trigger();
+  pdl_wait();
+  const int64_t nw = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  gather_rows<1>(g, (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5, nw, threadIdx.x & 31);
+}
+
+__device__ __forceinline__ void zero_range(float4* __restrict__ p, int64_t n4, int64_t i0, int64_t stride) {
+  for (int64_t i = i0; i < n4; i += stride) p[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
 __global__ void __launch_bounds__(256) zero_kernel(float4* __restrict__ p, int64_t n4) {
   pdl_trigger();
   pdl_wait();
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
-    p[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  zero_range(p, n4, static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x,
+             static_cast<int64_t>(gridDim.x) * blockDim.x);
 }
 
-// FP32 accumulator [n] -> BF16, round to nearest even; 8 elements per step.
+// FP32 accumulator [n] -> BF16, round to nearest even; 8 elements per item,
+// four items' loads in flight per thread.
+__device__ __forceinline__ void finalize_range(const float4* __restrict__ acc, uint4* __restrict__ out, int64_t n8,
+                                               int64_t i0, int64_t stride) {
+  for (int64_t ib = i0; ib < n8; ib += 4 * stride) {
+    float4 a[4], b[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int64_t i = ib + j * stride;
+      if (i < n8) {
+        a[j] = acc[2 * i];
+        b[j] = acc[2 * i + 1];
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int64_t i = ib + j * stride;
+      if (i < n8)
+        out[i] = make_uint4(pack_bf16x2(a[j].x, a[j].y), pack_bf16x2(a[j].z, a[j].w), pack_bf16x2(b[j].x, b[j].y),
+                            pack_bf16x2(b[j].z, b[j].w));
+    }
+  }
+}
+
 __global__ void __launch_bounds__(256) finalize_kernel(const float4* __restrict__ acc,
                                                        uint4* __restrict__ out, int64_t n8) {
   pdl_trigger();
   pdl_wait();
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const float4 a = acc[2 * i], b = acc[2 * i + 1];
-    out[i] = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y),
-                        pack_bf16x2(b.z, b.w));
-  }
+  finalize_range(acc, out, n8, static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x,
+                 static_cast<int64_t>(gridDim.x) * blockDim.x);
 }
 
 // Staged combine (DistributedEPCombine): out[t] = bf16(sum_j w[t,j] *

@@ -17,8 +17,12 @@ namespace moe {
 struct WsHeader {
   int status;        // sticky: the first device error code, 0 if none
   int timeout_site;  // where a bounded wait gave up (diagnostics only)
-  int pad[62];
+  int grid_bar[2];   // single-launch layer: barrier arrivals, generation
+  int pad[12];
+  unsigned long long phase_ns[8];  // single-launch layer: %globaltimer after each phase
+  int pad2[32];
 };
+static_assert(sizeof(WsHeader) == 256, "the workspace header is 256 bytes");
 
 // A bounded wait gives up after this many nanoseconds of %globaltimer.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;

@@ -102,7 +102,9 @@ struct GemmCfg {
   static constexpr int kBarrierBytes = 4096;
   static constexpr int kXposeStride = 36;   // floats per row of a 32 x 32 transpose buffer
   static constexpr int kXposeBytes = (EPI == EPI_L1) ? 0 : kEpiWarps * 32 * kXposeStride * 4;
-  static constexpr int kSmemBytes = 1024 /*align*/ + kStages * kStageBytes + kBarrierBytes + kXposeBytes;
+  static constexpr int kHeaderBytes = 1024;   // TMEM address, abort flag (kept across phases)
+  static constexpr int kPhaseBytes = kStages * kStageBytes + kBarrierBytes + kXposeBytes;
+  static constexpr int kSmemBytes = 1024 /*align*/ + kHeaderBytes + kPhaseBytes;
 };
 
 struct GemmArgs {
@@ -225,18 +227,20 @@ __device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, 
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
+// One GEMM over all its tiles by the calling CTA (tiles cta, cta + ncta, ...).
+// `smem` is this phase's 1024-byte-aligned shared memory (kPhaseBytes),
+// `tmem` a 512-column TMEM allocation, `abort_flag` the CTA's abort flag.
+// Ends with a block-wide barrier; no copy or MMA of the phase is in flight
+// when it returns.
 template <int FMT, int EPI>
-__global__ void __launch_bounds__(GemmCfg<FMT, EPI>::kThreads, 1)
-    moe_gemm_kernel(const __grid_constant__ GemmArgs p, const __grid_constant__ CUtensorMap tmA) {
+__device__ __forceinline__ void gemm_phase(const GemmArgs& p, const CUtensorMap* tmA, uint8_t* smem,
+                                           uint32_t tmem, volatile int* abort_flag, int cta, int ncta) {
   using Cfg = GemmCfg<FMT, EPI>;
   constexpr int S = Cfg::kStages;
   constexpr int NACC = Cfg::kAccBufs;
   constexpr int SB = Cfg::kStageBytes;
   constexpr int BB = b_block_bytes(FMT);
 
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * SB);
   uint64_t* empty = full + S;
   uint64_t* acc_full = empty + S;
@@ -246,8 +250,6 @@ __global__ void __launch_bounds__(GemmCfg<FMT, EPI>::kThreads, 1)
   uint64_t* sf_full = xbar + 4;    // NVFP4: scale buffer b holds the current stage's scales
   uint64_t* sf_empty = sf_full + 2;   // NVFP4: the MMAs reading scale buffer b completed
   uint64_t* sf_final = sf_empty + 2;  // NVFP4: the copier's last copies completed
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S * SB + 512);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* xbuf = reinterpret_cast<float*>(smem + S * SB + 1024);  // FP8 L1: [2][2][128] amax
   float* xpose = reinterpret_cast<float*>(smem + S * SB + Cfg::kBarrierBytes);  // L2: per-warp 32 x 32
 
@@ -270,17 +272,10 @@ __global__ void __launch_bounds__(GemmCfg<FMT, EPI>::kThreads, 1)
       mbar_init(&sf_empty[i], 1);
     }
     mbar_init(sf_final, 1);
-    *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) prefetch_tensormap(&tmA);
-  if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
-  tc_fence_before();
+  if (warp == 0 && lane == 0) prefetch_tensormap(tmA);
   __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  pdl_trigger();
-  pdl_wait();   // the layout, activations and accumulator come from earlier kernels
 
   const int na = *p.num_active;
   const int total = (na > 0) ? __ldg(p.tile_offsets + na) * p.n_tiles : 0;
@@ -291,7 +286,7 @@ __global__ void __launch_bounds__(GemmCfg<FMT, EPI>::kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       int issued = 0;
-      for (int T = blockIdx.x; T < total; T += gridDim.x) {
+      for (int T = cta; T < total; T += ncta) {
         TileInfo t;
         decode_tile(p, na, T, t);
         const uint8_t* wb =
@@ -301,7 +296,7 @@ __global__ void __launch_bounds__(GemmCfg<FMT, EPI>::kThreads, 1)
           uint8_t* sa = smem + stage * SB;
           uint8_t* sbp = sa + kAStage;
           mbar_arrive_expect_tx(&full[stage], SB);
-          tma_load_2d(sa, &tmA, &full[stage], ks * kBK, t.row0);
+          tma_load_2d(sa, tmA, &full[stage], ks * kBK, t.row0);
           bulk_load(sbp, wb + static_cast<size_t>(ks) * BB, BB, &full[stage]);
           if (FMT == FMT_NVFP4) {
             bulk_load(sbp + BB,
@@ -342,7 +337,7 @@ __global__ void __launch_bounds__(GemmCfg<FMT, EPI>::kThreads, 1)
       bool ok = true;
       int sb = 0;
       uint32_t sphase = 0;
-      for (int T = blockIdx.x; T < total && ok; T += gridDim.x) {
+      for (int T = cta; T < total && ok; T += ncta) {
         if (FMT != FMT_FP8) {
           if (!mbar_wait(&acc_empty[ab], aphase ^ 1u, abort_flag, p.status, 2)) break;
           tc_fence_after();
@@ -421,7 +416,7 @@ __global__ void __launch_bounds__(GemmCfg<FMT, EPI>::kThreads, 1)
       uint32_t phase = 0;
       int sb = 0;
       uint32_t sphase = 0;
-      for (int T = blockIdx.x; T < total; T += gridDim.x) {
+      for (int T = cta; T < total; T += ncta) {
         bool ok = true;
         for (int ks = 0; ks < p.k_stages; ++ks) {
           if (!mbar_wait(&full[stage], phase, abort_flag, p.status, 9) ||
@@ -464,7 +459,7 @@ __global__ void __launch_bounds__(GemmCfg<FMT, EPI>::kThreads, 1)
     int ab = 0;
     uint32_t aphase = 0;
     int xpar = 0;          // FP8 L1: amax exchange buffer / barrier phase
-    for (int T = blockIdx.x; T < total; T += gridDim.x) {
+    for (int T = cta; T < total; T += ncta) {
       TileInfo t;
       decode_tile(p, na, T, t);
       const bool valid = row_local < t.rows;
@@ -664,7 +659,44 @@ __global__ void __launch_bounds__(GemmCfg<FMT, EPI>::kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
+// The same phase as an out-of-line call: the single-launch kernel strings
+// several phases together, and separate calls keep their register
+// allocations from interfering.
+template <int FMT, int EPI>
+__device__ __noinline__ void gemm_phase_call(const GemmArgs& p, const CUtensorMap* tmA, uint8_t* smem,
+                                             uint32_t tmem, volatile int* abort_flag, int cta, int ncta) {
+  gemm_phase<FMT, EPI>(p, tmA, smem, tmem, abort_flag, cta, ncta);
+}
+
+// Shared-memory header of every kernel that runs GEMM phases.
+struct SmemHeader {
+  uint32_t tmem;
+  int abort;
+};
+
+__device__ __forceinline__ uint8_t* smem_base_1024() {
+  extern __shared__ uint8_t smem_raw[];
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+}
+
+template <int FMT, int EPI>
+__global__ void __launch_bounds__(GemmCfg<FMT, EPI>::kThreads, 1)
+    moe_gemm_kernel(const __grid_constant__ GemmArgs p, const __grid_constant__ CUtensorMap tmA) {
+  uint8_t* base = smem_base_1024();
+  SmemHeader* hdr = reinterpret_cast<SmemHeader*>(base);
+  if (threadIdx.x == 0) hdr->abort = 0;
+  if ((threadIdx.x >> 5) == 1) tmem_alloc(&hdr->tmem, kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = hdr->tmem;
+  pdl_trigger();
+  pdl_wait();   // the layout, activations and accumulator come from earlier kernels
+  gemm_phase<FMT, EPI>(p, &tmA, base + GemmCfg<FMT, EPI>::kHeaderBytes, tmem, &hdr->abort, blockIdx.x,
+                       gridDim.x);
+  if ((threadIdx.x >> 5) == 1) tmem_dealloc(tmem, kTmemCols);
 }
 
 // ---------------------------------------------------------------------------

@@ -11,6 +11,7 @@
 #include <utility>
 
 #include "aux_kernels.cuh"
+#include "fused.cuh"
 #include "gemm.cuh"
 
 using namespace moe;
@@ -200,8 +201,17 @@ cudaError_t set_attrs_fmt() {
   return set_gemm_attr<FMT, EPI_L2_STAGED>();
 }
 
+template <int FMT>
+cudaError_t set_fused_attr() {
+  return cudaFuncSetAttribute(moe_fused_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              fused_smem_bytes<FMT>());
+}
+
 cudaError_t set_all_attrs() {
   cudaError_t e;
+  if ((e = set_fused_attr<FMT_BF16>()) != cudaSuccess) return e;
+  if ((e = set_fused_attr<FMT_FP8>()) != cudaSuccess) return e;
+  if ((e = set_fused_attr<FMT_NVFP4>()) != cudaSuccess) return e;
   if ((e = set_attrs_fmt<FMT_BF16>()) != cudaSuccess) return e;
   if ((e = set_attrs_fmt<FMT_FP8>()) != cudaSuccess) return e;
   return set_attrs_fmt<FMT_NVFP4>();
@@ -248,34 +258,43 @@ int grid_for(int64_t n, int threads, int cap = 148 * 16) {
   return int(g);
 }
 
-cudaError_t launch_route(const moe_problem_t* p, const float* logits, const float* bias, int64_t* idx,
-                         float* w, cudaStream_t st) {
-  const int E = p->num_experts;
-  const int64_t M = p->num_tokens;
-  const int grid = int((M * 32 + 255) / 256);
-  const int per = (E + 31) / 32;
-  TimScope ts(MOE_SLOT_ROUTE, st);
-#define MOE_ROUTE(PER) launch_k(route_kernel<PER>, grid, 256, 0, st, logits, bias, M, E, p->num_topk, idx, w)
-  if (per <= 1) return MOE_ROUTE(1);
-  if (per <= 2) return MOE_ROUTE(2);
-  if (per <= 4) return MOE_ROUTE(4);
-  if (per <= 8) return MOE_ROUTE(8);
-  if (per <= 16) return MOE_ROUTE(16);
-  return MOE_ROUTE(32);
-#undef MOE_ROUTE
+RouteArgs route_args(const moe_problem_t* p, const float* logits, const float* bias, int64_t* idx, float* w) {
+  RouteArgs a{};
+  a.logits = logits;
+  a.bias = bias;
+  a.M = p->num_tokens;
+  a.E = p->num_experts;
+  a.k = p->num_topk;
+  a.idx_out = idx;
+  a.w_out = w;
+  return a;
 }
 
-cudaError_t launch_permute(const moe_problem_t* p, const int64_t* idx, const PermOut& o, int* block_counts,
-                           int nblk, int* status, cudaStream_t st) {
-  const int E = p->num_experts;
-  const int64_t R = p->num_tokens * p->num_topk;
+cudaError_t launch_route(const RouteArgs& a, cudaStream_t st) {
+  TimScope ts(MOE_SLOT_ROUTE, st);
+  return launch_k(route_kernel, grid_for(a.M * 32, 256, 1 << 30), 256, 0, st, a);
+}
+
+PermArgs perm_args(const moe_problem_t* p, const int64_t* idx, const PermOut& o, int* block_counts, int nblk,
+                   int* status) {
+  PermArgs a{};
+  a.idx = idx;
+  a.R = p->num_tokens * p->num_topk;
+  a.E = p->num_experts;
+  a.nblk = nblk;
+  a.block_counts = block_counts;
+  a.o = o;
+  a.status = status;
+  return a;
+}
+
+cudaError_t launch_permute(const PermArgs& a, cudaStream_t st) {
   TimScope ts(MOE_SLOT_PERMUTE, st);
-  if (R <= kPermSmallMax && E <= kPermSmallMaxE)
-    return launch_k(perm_small_kernel, 1, 1024, (36 * E + 3) * sizeof(int), st, idx, int(R), E, o, status);
-  cudaError_t e = launch_k(perm_count_kernel, nblk, 256, E * sizeof(int), st, idx, R, E, block_counts, status);
+  if (perm_small_case(a.R, a.E))
+    return launch_k(perm_small_kernel, 1, 1024, perm_small_smem_ints(a.E, 32) * sizeof(int), st, a);
+  cudaError_t e = launch_k(perm_count_kernel, a.nblk, 256, a.E * sizeof(int), st, a);
   if (e != cudaSuccess) return e;
-  return launch_k(perm_scatter_kernel, nblk, 256, (5 * E + 3 + kPermChunk) * sizeof(int), st, idx, R, E, nblk,
-                  static_cast<const int*>(block_counts), o);
+  return launch_k(perm_scatter_kernel, a.nblk, 256, perm_chunk_smem_ints(a.E) * sizeof(int), st, a);
 }
 
 struct FfnBuffers {
@@ -287,21 +306,29 @@ struct FfnBuffers {
   int* status;
 };
 
-moe_status_t run_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_weights_t* w,
-                     const FfnBuffers& b, const float* topk_weights,
-                     int out_mode, float* out, cudaStream_t st) {
+// Everything the FFN kernels need: the gather, the two GEMMs and their A maps.
+struct FfnPlan {
+  GatherArgs g;
+  GemmArgs l1, l2;
+  CUtensorMap ta1, ta2;
+  int grid1, grid2;
+};
+
+moe_status_t plan_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_weights_t* w, const FfnBuffers& b,
+                      const float* topk_weights, float* out, FfnPlan& pl) {
   const int fmt = p->format, H = p->hidden, I = p->intermediate_hidden, E = p->num_experts, k = p->num_topk;
   const int64_t M = p->num_tokens, R = M * k;
   const int nsm = sm_count();
 
-  // gather
-  GatherArgs g{};
+  GatherArgs& g = pl.g;
+  g = GatherArgs{};
   g.x = static_cast<const uint8_t*>(act->x);
   g.x_scale = act->x_scale;
   g.src_info = b.src_info;
   g.starts = b.starts;
   g.a_scale_offsets = b.a_scale_offsets;
   g.R = R;
+  g.E = E;
   g.row_bytes = x_row_bytes(fmt, H);
   g.topk = k;
   g.H = H;
@@ -310,16 +337,11 @@ moe_status_t run_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_wei
   g.sa_t = reinterpret_cast<float*>(b.x_sf);
   g.sfa = b.x_sf;
   g.ld = int(b.P);
-  {
-    TimScope ts(MOE_SLOT_GATHER, st);
-    if (launch_k(gather_kernel, grid_for(R * 32, 256, 1 << 30), 256, 0, st, g, E) != cudaSuccess)
-      return MOE_ERR_CUDA;
-  }
 
   // L1: gate_up
-  CUtensorMap ta{};
-  if (!make_map(&ta, b.x_perm, x_row_bytes(fmt, H), uint64_t(R), 128)) return MOE_ERR_CUDA;
-  GemmArgs a{};
+  if (!make_map(&pl.ta1, b.x_perm, x_row_bytes(fmt, H), uint64_t(R), 128)) return MOE_ERR_CUDA;
+  GemmArgs& a = pl.l1;
+  a = GemmArgs{};
   a.k_stages = x_row_bytes(fmt, H) / 128;
   a.n_tiles = I / 128;
   a.wB = static_cast<const uint8_t*>(w->w13);
@@ -352,22 +374,12 @@ moe_status_t run_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_wei
   a.h_scale_ld = int(b.P);
   a.status = b.status;
   const int64_t mtiles_bound = (R + 127) / 128 + std::min<int64_t>(E, R);
-  int grid1 = int(std::min<int64_t>(nsm, mtiles_bound * a.n_tiles));
-  {
-    TimScope ts(MOE_SLOT_GEMM1, st);
-    if (launch_gemm_fmt<EPI_L1>(fmt, a, ta, std::max(grid1, 1), st) != cudaSuccess) return MOE_ERR_CUDA;
-  }
+  pl.grid1 = std::max(1, int(std::min<int64_t>(nsm, mtiles_bound * a.n_tiles)));
 
   // L2: down
-  if (out_mode == MOE_OUT_ACCUMULATE) {
-    TimScope ts(MOE_SLOT_ZERO, st);
-    if (launch_k(zero_kernel, grid_for(M * H / 4, 256), 256, 0, st, reinterpret_cast<float4*>(out),
-                 int64_t(M * H / 4)) != cudaSuccess)
-      return MOE_ERR_CUDA;
-  }
-  CUtensorMap ta2{};
-  if (!make_map(&ta2, b.h, h_row_bytes(fmt, I), uint64_t(R), 128)) return MOE_ERR_CUDA;
-  GemmArgs a2 = a;
+  if (!make_map(&pl.ta2, b.h, h_row_bytes(fmt, I), uint64_t(R), 128)) return MOE_ERR_CUDA;
+  GemmArgs& a2 = pl.l2;
+  a2 = a;
   a2.k_stages = h_row_bytes(fmt, I) / 128;
   a2.n_tiles = H / 256;
   // n-major keeps one 256-column slice of the FP32 accumulator hot in L2, at
@@ -383,12 +395,54 @@ moe_status_t run_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_wei
   a2.sb_kb = I / 128;
   a2.alpha = w->down_expert_scales;
   a2.out = out;
-  int grid2 = int(std::min<int64_t>(nsm, mtiles_bound * a2.n_tiles));
+  pl.grid2 = std::max(1, int(std::min<int64_t>(nsm, mtiles_bound * a2.n_tiles)));
+  return MOE_OK;
+}
+
+moe_status_t run_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_weights_t* w,
+                     const FfnBuffers& b, const float* topk_weights,
+                     int out_mode, float* out, cudaStream_t st) {
+  const int fmt = p->format;
+  const int64_t M = p->num_tokens, R = M * p->num_topk, H = p->hidden;
+  FfnPlan pl;
+  moe_status_t s = plan_ffn(p, act, w, b, topk_weights, out, pl);
+  if (s != MOE_OK) return s;
+  {
+    TimScope ts(MOE_SLOT_GATHER, st);
+    if (launch_k(gather_kernel, grid_for(R * 32, 256, 1 << 30), 256, 0, st, pl.g) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
+  {
+    TimScope ts(MOE_SLOT_GEMM1, st);
+    if (launch_gemm_fmt<EPI_L1>(fmt, pl.l1, pl.ta1, pl.grid1, st) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  if (out_mode == MOE_OUT_ACCUMULATE) {
+    TimScope ts(MOE_SLOT_ZERO, st);
+    if (launch_k(zero_kernel, grid_for(M * H / 4, 256), 256, 0, st, reinterpret_cast<float4*>(out),
+                 int64_t(M * H / 4)) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
   TimScope ts2(MOE_SLOT_GEMM2, st);
   cudaError_t e = (out_mode == MOE_OUT_ACCUMULATE)
-                      ? launch_gemm_fmt<EPI_L2_ACC>(fmt, a2, ta2, std::max(grid2, 1), st)
-                      : launch_gemm_fmt<EPI_L2_STAGED>(fmt, a2, ta2, std::max(grid2, 1), st);
+                      ? launch_gemm_fmt<EPI_L2_ACC>(fmt, pl.l2, pl.ta2, pl.grid2, st)
+                      : launch_gemm_fmt<EPI_L2_STAGED>(fmt, pl.l2, pl.ta2, pl.grid2, st);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// The single-launch layer: a cooperative launch of moe_fused_kernel<FMT>.
+template <int FMT>
+cudaError_t launch_fused_fmt(const FusedArgs& f, const FfnPlan& pl, int grid, cudaStream_t st) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(GemmCfg<FMT, EPI_L1>::kThreads);
+  cfg.dynamicSmemBytes = fused_smem_bytes<FMT>();
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, moe_fused_kernel<FMT>, f, pl.ta1, pl.ta2);
 }
 
 bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; }
@@ -520,7 +574,8 @@ moe_status_t moe_route(const moe_problem_t* p, const float* logits, const float*
   if (p->num_topk > 32) return MOE_ERR_UNSUPPORTED;
   if (p->num_tokens == 0) return MOE_OK;
   if (!logits || !topk_idx || !topk_weights) return MOE_ERR_INVALID_ARG;
-  return launch_route(p, logits, bias, topk_idx, topk_weights, static_cast<cudaStream_t>(stream)) == cudaSuccess
+  return launch_route(route_args(p, logits, bias, topk_idx, topk_weights), static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
              ? MOE_OK
              : MOE_ERR_CUDA;
 }
@@ -536,8 +591,9 @@ moe_status_t moe_permute(const moe_problem_t* p, const int64_t* topk_idx, const 
   uint8_t* base = static_cast<uint8_t*>(ws);
   PermOut o{layout->expert_counts, layout->expert_start_indices, layout->src_info, layout->slot_to_row,
             layout->expert_ids,    layout->num_active,           layout->a_scale_offsets, layout->tile_offsets};
-  return launch_permute(p, topk_idx, o, reinterpret_cast<int*>(base + L.block_counts), L.nblk,
-                        reinterpret_cast<int*>(base + L.header), static_cast<cudaStream_t>(stream)) == cudaSuccess
+  return launch_permute(perm_args(p, topk_idx, o, reinterpret_cast<int*>(base + L.block_counts), L.nblk,
+                                  reinterpret_cast<int*>(base + L.header)),
+                        static_cast<cudaStream_t>(stream)) == cudaSuccess
              ? MOE_OK
              : MOE_ERR_CUDA;
 }
@@ -618,12 +674,14 @@ moe_status_t moe_fused(const moe_problem_t* p, const moe_act_t* act, const moe_w
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* base = static_cast<uint8_t*>(ws);
   int* status = reinterpret_cast<int*>(base + L.header);
+  FusedArgs f{};
   const int64_t* idx = topk_idx;
   const float* wts = topk_weights;
   if (from_logits) {
     int64_t* ridx = reinterpret_cast<int64_t*>(base + L.route_idx);
     float* rw = reinterpret_cast<float*>(base + L.route_w);
-    if (launch_route(p, logits, bias, ridx, rw, st) != cudaSuccess) return MOE_ERR_CUDA;
+    f.route = route_args(p, logits, bias, ridx, rw);
+    f.do_route = 1;
     idx = ridx;
     wts = rw;
   }
@@ -631,8 +689,8 @@ moe_status_t moe_fused(const moe_problem_t* p, const moe_act_t* act, const moe_w
             reinterpret_cast<int*>(base + L.src_info),   reinterpret_cast<int*>(base + L.slot_to_row),
             reinterpret_cast<int*>(base + L.expert_ids), reinterpret_cast<int*>(base + L.num_active),
             reinterpret_cast<int*>(base + L.a_scale_offsets), reinterpret_cast<int*>(base + L.tile_offsets)};
-  if (launch_permute(p, idx, o, reinterpret_cast<int*>(base + L.block_counts), L.nblk, status, st) != cudaSuccess)
-    return MOE_ERR_CUDA;
+  f.perm = perm_args(p, idx, o, reinterpret_cast<int*>(base + L.block_counts), L.nblk, status);
+  f.perm_small = perm_small_case(f.perm.R, f.perm.E) ? 1 : 0;
   FfnBuffers b{};
   b.counts = o.expert_counts;
   b.starts = o.expert_start_indices;
@@ -649,13 +707,29 @@ moe_status_t moe_fused(const moe_problem_t* p, const moe_act_t* act, const moe_w
   b.P = L.P;
   b.status = status;
   float* acc = reinterpret_cast<float*>(base + L.acc);
-  if ((s = run_ffn(p, act, w, b, wts, MOE_OUT_ACCUMULATE, acc, st)) != MOE_OK) return s;
+  FfnPlan pl;
+  if ((s = plan_ffn(p, act, w, b, wts, acc, pl)) != MOE_OK) return s;
   const int64_t M = p->num_tokens, H = p->hidden;
-  TimScope ts(MOE_SLOT_FINALIZE, st);
-  return launch_k(finalize_kernel, grid_for(M * H / 8, 256), 256, 0, st, reinterpret_cast<const float4*>(acc),
-                  static_cast<uint4*>(out_bf16), int64_t(M * H / 8)) == cudaSuccess
-             ? MOE_OK
-             : MOE_ERR_CUDA;
+  f.gather = pl.g;
+  f.acc = reinterpret_cast<float4*>(acc);
+  f.acc_n4 = M * H / 4;
+  f.out = static_cast<uint4*>(out_bf16);
+  f.out_n8 = M * H / 8;
+  f.l1 = pl.l1;
+  f.l2 = pl.l2;
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(base + L.header);
+  f.gbar = hdr->grid_bar;
+  f.status = status;
+  f.phase_ns = hdr->phase_ns;
+  const int grid = sm_count();
+  TimScope ts(MOE_SLOT_FUSED, st);
+  cudaError_t e;
+  switch (p->format) {
+    case FMT_BF16: e = launch_fused_fmt<FMT_BF16>(f, pl, grid, st); break;
+    case FMT_FP8: e = launch_fused_fmt<FMT_FP8>(f, pl, grid, st); break;
+    default: e = launch_fused_fmt<FMT_NVFP4>(f, pl, grid, st); break;
+  }
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 moe_status_t moe_timing_enable(int enable, int max_calls) {
