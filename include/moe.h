@@ -251,6 +251,33 @@ moe_status_t moe_fused(const moe_problem_t* problem, const moe_act_t* act,
                        const float* topk_weights, const float* logits, const float* bias,
                        void* out_bf16, void* workspace, size_t workspace_bytes, void* stream);
 
+/* moe_permute without a workspace and without allocating, for callers that
+ * cannot call cudaMalloc: a host runtime that links this library but has no
+ * device allocator of its own to hand out scratch, or a serving loop that
+ * reserves all device memory once at start-up and must not allocate per
+ * request (cudaMalloc can synchronise the device and can fail under memory
+ * pressure).  It computes the same layout as moe_permute.  The caller still
+ * passes topk_idx and the layout arrays, plus device_status: one device
+ * int32 that the call sets to MOE_OK before its kernels run and that they
+ * set to the first device error (MOE_ERR_BAD_INDEX for an index outside
+ * [-1, num_experts)).  The pages have no counterpart of this entry point.
+ *
+ * Its scratch is a file-scope device array of 32768 int32 (128 KB), which
+ * every GPU that loads the library holds until the process exits.  Problems
+ * with more than 16384 slots or more than 256 experts keep their per-chunk
+ * expert counts there, which limits them to
+ * ceil(num_tokens*num_topk/1024) * num_experts <= 32768; larger problems
+ * return MOE_ERR_UNSUPPORTED and launch nothing.  Smaller problems run in
+ * one block and need no scratch.  The counts are rewritten in full by every
+ * call, so nothing has to start at zero; the array keeps the last call's
+ * contents.  The first call on each device looks up the array's device
+ * address with that device current; make that first call before any stream
+ * capture.  All calls share the one array: calls that overlap on the GPU
+ * (on other streams, or from other host threads) race on it.  No memory is
+ * allocated or freed, by this library or any other. */
+moe_status_t moe_permute_noalloc(const moe_problem_t* problem, const int64_t* topk_idx,
+                                 const moe_layout_t* layout, int32_t* device_status, void* stream);
+
 /* Per-kernel timing, for measurement.  moe_timing_enable(1, max_calls)
  * creates CUDA events for up to max_calls calls (once, on the current
  * device); from then on every moe_fused / moe_ffn / moe_permute / moe_route /

@@ -39,6 +39,7 @@ EXPORTS = (
     "moe_get_prepared_weights_size",
     "moe_route", "moe_permute", "moe_ffn", "moe_get_intermediate_size", "moe_combine",
     "moe_fused", "moe_read_status", "moe_status_string", "moe_timing_enable", "moe_timing_read",
+    "moe_permute_noalloc",
 )
 
 SLOTS = ("route", "permute", "gather", "gemm1", "zero", "gemm2", "finalize", "combine", "fused")
@@ -111,6 +112,7 @@ def lib():
             "moe_fused": [P, ctypes.POINTER(Act), ctypes.POINTER(Weights), vp, vp, vp, vp, vp, vp, sz, vp],
             "moe_read_status": [vp, vp],
             "moe_timing_enable": [ctypes.c_int, ctypes.c_int],
+            "moe_permute_noalloc": [P, vp, ctypes.POINTER(Layout), vp, vp],
             "moe_timing_read": [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int)],
         }
         for name, args in sig.items():
@@ -237,6 +239,13 @@ def combine(prob, lay, topk_weights, inp, in_mode, out_bf16, stream=None):
     _check("moe_combine", lib().moe_combine(ctypes.byref(prob), None if lay is None else ctypes.byref(lay),
                                             _ptr(topk_weights), _ptr(inp), int(in_mode),
                                             _ptr(out_bf16), _stream(stream)))
+
+
+def permute_noalloc(prob, topk_idx, lay, device_status, stream=None):
+    """moe_permute without a workspace (see include/moe.h)."""
+    _check("moe_permute_noalloc", lib().moe_permute_noalloc(ctypes.byref(prob), _ptr(topk_idx),
+                                                            ctypes.byref(lay), _ptr(device_status),
+                                                            _stream(stream)))
 
 
 def fused(prob, a, w, out_bf16, ws, ws_bytes, topk_idx=None, topk_weights=None, logits=None,

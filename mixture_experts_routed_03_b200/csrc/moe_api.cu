@@ -463,6 +463,36 @@ bool layout_ok(const moe_layout_t* l) {
          l->num_active && l->a_scale_offsets && l->tile_offsets;
 }
 
+
+// ------------------------------------------------------ allocation-free permute
+// Scratch of moe_permute_noalloc, the entry point for callers that cannot
+// allocate device memory (a host runtime without a device allocator, a
+// serving loop that must not allocate per request): the per-chunk expert
+// counts of the two-pass permutation live in this file-scope device array,
+// which every GPU that loads the library holds until the process exits.
+// kNoAllocCountEntries bounds chunks x experts.  Pass 1 rewrites every entry
+// it covers, so no clearing is needed; concurrent calls race on the array.
+constexpr int kNoAllocCountEntries = 32768;   // 128 KB
+static __device__ __align__(256) int g_noalloc_counts[kNoAllocCountEntries];
+
+// Device address of g_noalloc_counts per device, looked up once per device
+// with that device current (host code cannot use the symbol itself).
+int* noalloc_counts_ptr() {
+  static int* ptrs[64] = {nullptr};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_counts) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<int*>(p);
+  }
+  return ptrs[dev];
+}
+
+__global__ void set_int_kernel(int* p, int v) { *p = v; }
+
 }  // namespace
 
 // =============================================================== C ABI
@@ -730,6 +760,30 @@ moe_status_t moe_fused(const moe_problem_t* p, const moe_act_t* act, const moe_w
     default: e = launch_fused_fmt<FMT_NVFP4>(f, pl, grid, st); break;
   }
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status_t moe_permute_noalloc(const moe_problem_t* p, const int64_t* topk_idx, const moe_layout_t* layout,
+                                 int32_t* device_status, void* stream) {
+  moe_status_t s = check_problem(p);
+  if (s != MOE_OK) return s;
+  if (p->num_tokens == 0) return MOE_OK;
+  if (!topk_idx || !layout_ok(layout) || !device_status) return MOE_ERR_INVALID_ARG;
+  const int64_t R = p->num_tokens * p->num_topk;
+  const int E = p->num_experts;
+  const int64_t nblk = (R + kPermChunk - 1) / kPermChunk;
+  const bool small = perm_small_case(R, E);
+  if (!small && nblk * E > kNoAllocCountEntries) return MOE_ERR_UNSUPPORTED;
+  int* counts = small ? nullptr : noalloc_counts_ptr();
+  if (!small && !counts) return MOE_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the status word must start at zero; the counts are fully rewritten by pass 1
+  set_int_kernel<<<1, 1, 0, st>>>(device_status, MOE_OK);
+  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  PermOut o{layout->expert_counts, layout->expert_start_indices, layout->src_info, layout->slot_to_row,
+            layout->expert_ids,    layout->num_active,           layout->a_scale_offsets, layout->tile_offsets};
+  return launch_permute(perm_args(p, topk_idx, o, counts, int(nblk), device_status), st) == cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
 }
 
 moe_status_t moe_timing_enable(int enable, int max_calls) {
