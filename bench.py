@@ -95,6 +95,34 @@ def stored_traffic(workload, kernel):
     return float(rec["dram_bytes_per_launch"])
 
 
+def dist_env():
+    """(world size, rank, local rank) from the torchrun environment."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def rank_seed(seed, rank):
+    """Each rank draws its own batch (and its own copy of the experts)."""
+    return seed + rank
+
+
+def max_over_ranks(values, world, device):
+    """Element-wise maximum of per-rank floats; every rank calls it at the same
+    point (a no-op on one rank)."""
+    if world <= 1:
+        return [float(v) for v in values]
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_throughput(units_per_rank, world, steps, t_ms):
+    """Units all ranks processed per second, over the slowest rank's time."""
+    return units_per_rank * world * steps / (t_ms / 1e3)
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -210,7 +238,7 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     p = workload(args)
-    d = workloads.make_inputs(p, seed=args.seed + rank, device=dev)
+    d = workloads.make_inputs(p, seed=rank_seed(args.seed, rank), device=dev)
     wts = {k: d.get(k) for k in ("w13", "w13_scale", "w2", "w2_scale", "gate_up_expert_scales",
                                  "down_expert_scales", "c_input_scales")}
     L = layer.MoELayer(p, wts, device=dev)
@@ -326,10 +354,7 @@ def run_ours(args, rank, world, local_rank):
     num_active = int(torch.unique(idx[idx >= 0]).numel())
 
     # ---- max over ranks
-    if world > 1:
-        tt = torch.tensor([t_ms, e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_ms, e2e_ms = float(tt[0]), float(tt[1])
+    t_ms, e2e_ms = max_over_ranks([t_ms, e2e_ms], world, dev)
     return dict(p=p, t_ms=t_ms, per_step=per_step, kern=kern, launches=launches, e2e_ms=e2e_ms, phases=phases,
                 h2d=h2d, d2h=d2h, num_active=num_active, clocks=clocks.summary(), R=R, M=M,
                 host_inputs=(d, L) if rank == 0 else None)
@@ -376,17 +401,17 @@ def cpu_baseline(p, d, seconds):
 def main_ours(args):
     import torch
     import torch.distributed as dist
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    import datetime
+    world, rank, local_rank = dist_env()
     if world > 1:
-        dist.init_process_group("nccl", device_id=torch.device("cuda", local_rank))
+        # a short timeout ends a collective whose peer has gone with an error
+        dist.init_process_group("nccl", device_id=torch.device("cuda", local_rank),
+                                timeout=datetime.timedelta(seconds=120))
     r = run_ours(args, rank, world, local_rank)
     p = r["p"]
     peaks, peak_src = load_peaks()
-    units = r["R"] * world * args.steps
-    value = units / (r["t_ms"] / 1e3)
-    e2e_value = units / (r["e2e_ms"] / 1e3)
+    value = job_throughput(r["R"], world, args.steps, r["t_ms"])
+    e2e_value = job_throughput(r["R"], world, args.steps, r["e2e_ms"])
     wm = work_model(p, r["num_active"])
     kern = r["kern"]
     step_ms = r["t_ms"] / args.steps
@@ -429,7 +454,7 @@ def main_ours(args):
                    "num_topk": p["num_topk"], "format": p["format"], "routing": p["routing"],
                    "active_experts": r["num_active"], "parallelism": f"dp{world} (replicas)",
                    "l2": "flushed (512 MiB write) before every timed step, outside the step interval"},
-        "tokens_per_s": p["num_tokens"] * world * args.steps / (r["t_ms"] / 1e3),
+        "tokens_per_s": job_throughput(p["num_tokens"], world, args.steps, r["t_ms"]),
         "layer_tflops": wm["layer"]["flops"] / (step_ms / 1e3) / 1e12,
         "layer_gbs": wm["layer"]["bytes"] / (step_ms / 1e3) / 1e9,
         "roofline": {"kernel": {"fused": "moe_fused_kernel", "gemm1": "moe_gemm_kernel (gate_up)",
@@ -460,11 +485,11 @@ def main_ours(args):
 # --------------------------------------------------------------------------- reference arm
 
 def main_reference(args):
-    """The CPU oracle timed on the host cores, on this workload (rank 0 only)."""
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
+    """The CPU oracle timed on the host cores, on this workload (rank 0 only;
+    the other ranks return without work)."""
+    world, rank, _ = dist_env()
     if rank != 0:
-        return
+        return None
     import numpy as np
     import torch
 

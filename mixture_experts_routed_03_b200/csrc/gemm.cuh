@@ -481,13 +481,19 @@ __device__ __forceinline__ void gemm_phase(const GemmArgs& p, const CUtensorMap*
           nb_lo = nb_hi = (t.n_tile * kBN + half * 128) >> 7;
         }
         bool ok = true;
+        // The activation scale of K block ks+1 (a per-row load from L2) is
+        // issued before block ks is waited for, taking its latency off the
+        // per-block critical path; the weight scales are warp-uniform L1 hits.
+        const float* sa_col = p.sa_t + pr;
+        float nx_sa = sa_col[0];
         for (int ks = 0; ks < p.k_stages; ++ks) {
+          const float sa = nx_sa;
+          if (ks + 1 < p.k_stages) nx_sa = sa_col[static_cast<size_t>(ks + 1) * p.sa_ld];
           if (!mbar_wait(&acc_full[ab], aphase, abort_flag, p.status, 5)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const float sa = p.sa_t[static_cast<size_t>(ks) * p.sa_ld + pr];
           const float s_lo = sa * __ldg(sbe + nb_lo * p.sb_kb + ks);
           const float s_hi = sa * __ldg(sbe + nb_hi * p.sb_kb + ks);
           const uint32_t base = tmem + ab * kBN + half * 128 + lane_off;
@@ -514,13 +520,25 @@ __device__ __forceinline__ void gemm_phase(const GemmArgs& p, const CUtensorMap*
         if (!mbar_wait(&acc_full[ab], aphase, abort_flag, p.status, 6)) break;
         tc_fence_after();
         const uint32_t base = tmem + ab * kBN + half * 128 + lane_off;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          float v[32];
+        {
+          // all 128 columns in one TMEM round trip
+          uint32_t r0[32], r1[32], r2[32], r3[32];
           __syncwarp();
-          tmem_ld32(base + 32 * c, v);
+          tmem_ld32_async(base, r0);
+          tmem_ld32_async(base + 32, r1);
+          tmem_ld32_async(base + 64, r2);
+          tmem_ld32_async(base + 96, r3);
+          tmem_wait_ld(r0);
+          tmem_wait_ld(r1);
+          tmem_wait_ld(r2);
+          tmem_wait_ld(r3);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) acc[32 * c + i] = v[i];
+          for (int i = 0; i < 32; ++i) {
+            acc[i] = __uint_as_float(r0[i]);
+            acc[32 + i] = __uint_as_float(r1[i]);
+            acc[64 + i] = __uint_as_float(r2[i]);
+            acc[96 + i] = __uint_as_float(r3[i]);
+          }
         }
         tc_fence_before();
         __syncwarp();
