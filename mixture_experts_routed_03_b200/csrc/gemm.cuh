@@ -101,7 +101,14 @@ struct GemmCfg {
   static constexpr int kThreads = (kFirstEpiWarp + kEpiWarps) * 32;
   static constexpr int kBarrierBytes = 4096;
   static constexpr int kXposeStride = 36;   // floats per row of a 32 x 32 transpose buffer
-  static constexpr int kXposeBytes = (EPI == EPI_L1) ? 0 : kEpiWarps * 32 * kXposeStride * 4;
+  // L2: per-warp 32 x 32 FP32 transposes.  FP8 L1: per-quarter staging of
+  // the 32 rows x 128 h bytes the quarter's two warps produce, so that the
+  // rows leave as whole 128-byte segments (rows padded to 144 bytes against
+  // bank conflicts).
+  static constexpr int kHStageStride = 144;
+  static constexpr int kXposeBytes = (EPI != EPI_L1)        ? kEpiWarps * 32 * kXposeStride * 4
+                                     : (FMT == FMT_FP8) ? 4 * 32 * kHStageStride
+                                                        : 0;
   static constexpr int kHeaderBytes = 1024;   // TMEM address, abort flag (kept across phases)
   static constexpr int kPhaseBytes = kStages * kStageBytes + kBarrierBytes + kXposeBytes;
   static constexpr int kSmemBytes = 1024 /*align*/ + kHeaderBytes + kPhaseBytes;
@@ -160,31 +167,29 @@ struct TileInfo {
 // down leg when its whole A operand fits in L2): concurrent CTAs add into the
 // same 256 output columns of every token, a slice of the FP32 accumulator
 // that stays in L2.
-__device__ __forceinline__ void decode_tile(const GemmArgs& p, int na, int T, TileInfo& t) {
-  const int nt = p.n_tiles;
-  const bool kNMajor = p.n_major != 0;
-  int g, scale;   // search key and the multiplier of tile_offsets
-  if (kNMajor) {
+// Search key of tile T: n-major order gives the n tile directly and keys the
+// expert search by m tile; expert-major order keys it by T itself.
+__device__ __forceinline__ int tile_key(const GemmArgs& p, int na, int T, TileInfo& t, int& scale) {
+  if (p.n_major != 0) {
     const int total_mt = __ldg(p.tile_offsets + na);
     t.n_tile = T / total_mt;
-    g = T - t.n_tile * total_mt;
     scale = 1;
-  } else {
-    g = T;
-    scale = nt;
+    return T - t.n_tile * total_mt;
   }
-  int lo = 0, hi = na;  // tile_offsets[lo]*scale <= g < tile_offsets[hi]*scale
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (__ldg(p.tile_offsets + mid) * scale <= g) lo = mid; else hi = mid;
-  }
+  scale = p.n_tiles;
+  return T;
+}
+
+// The rest of the decode once the active-expert slot `lo` of tile T is known
+// (tile_offsets[lo]*scale <= g < tile_offsets[lo+1]*scale).
+__device__ __forceinline__ void tile_finish(const GemmArgs& p, int lo, int g, int T, TileInfo& t) {
   const int mt0 = __ldg(p.tile_offsets + lo);
   int mt;
-  if (kNMajor) {
+  if (p.n_major != 0) {
     mt = g - mt0;
   } else {
     const int nm = __ldg(p.tile_offsets + lo + 1) - mt0;
-    const int local = T - mt0 * nt;
+    const int local = T - mt0 * p.n_tiles;
     t.n_tile = local / nm;
     mt = local - t.n_tile * nm;
   }
@@ -196,6 +201,37 @@ __device__ __forceinline__ void decode_tile(const GemmArgs& p, int na, int T, Ti
   t.srow0 = __ldg(p.a_scale_offsets + t.e) + mt * kBM;
 }
 
+// Tile T -> (expert, m tile, n tile) by one thread: binary search over the
+// active experts' tile offsets.
+__device__ __forceinline__ void decode_tile(const GemmArgs& p, int na, int T, TileInfo& t) {
+  int scale;
+  const int g = tile_key(p, na, T, t, scale);
+  int lo = 0, hi = na;  // tile_offsets[lo]*scale <= g < tile_offsets[hi]*scale
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(p.tile_offsets + mid) * scale <= g) lo = mid; else hi = mid;
+  }
+  tile_finish(p, lo, g, T, t);
+}
+
+// The same decode by a whole converged warp: each round probes 32 evenly
+// spaced offsets at once and keeps the bucket the key falls in, so up to
+// 1024 active experts take two dependent loads instead of ten.
+__device__ __forceinline__ void decode_tile_warp(const GemmArgs& p, int na, int T, TileInfo& t, int lane) {
+  int scale;
+  const int g = tile_key(p, na, T, t, scale);
+  int base = 0, len = na;  // the slot lies in [base, base + len); offsets[base]*scale <= g
+  while (len > 1) {
+    const int step = (len + 31) >> 5;
+    const bool le = lane * step < len && __ldg(p.tile_offsets + base + lane * step) * scale <= g;
+    const unsigned m = __ballot_sync(0xFFFFFFFFu, le);
+    const int j = 31 - __clz(m);
+    base += j * step;
+    len = min(step, len - j * step);
+  }
+  tile_finish(p, base, g, T, t);
+}
+
 // A wait used while tearing down after an abort: ignores the abort flag.
 __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
   const unsigned long long t0 = globaltimer_ns();
@@ -204,11 +240,25 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
   }
 }
 
-__device__ __forceinline__ float clamped_swiglu(float g, float u, float c, int fast) {
+template <bool FAST>
+__device__ __forceinline__ float clamped_swiglu(float g, float u, float c) {
   const float gc = fminf(g, c);
   const float uc = fminf(fmaxf(u, -c), c);
-  if (fast) return __fmul_rn(__fdividef(gc, 1.0f + __expf(-gc)), uc);
+  if (FAST) return __fmul_rn(__fdividef(gc, 1.0f + __expf(-gc)), uc);
   return __fmul_rn(__fdiv_rn(gc, 1.0f + expf(-gc)), uc);
+}
+
+// h[i] = clamped SwiGLU of (gate acc[i], up acc[64 + i]), i < 64.  The
+// precision switch is taken once, outside the unrolled loop, so only one of
+// the two sequences runs.
+__device__ __forceinline__ void swiglu_row(const float (&acc)[128], float (&h)[64], float c, int fast) {
+  if (fast) {
+#pragma unroll
+    for (int i = 0; i < 64; ++i) h[i] = clamped_swiglu<true>(acc[i], acc[64 + i], c);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 64; ++i) h[i] = clamped_swiglu<false>(acc[i], acc[64 + i], c);
+  }
 }
 
 // Byte offset of (padded row pr, scale column j) inside the 512-byte scale
@@ -250,6 +300,7 @@ __device__ __forceinline__ void gemm_phase(const GemmArgs& p, const CUtensorMap*
   uint64_t* sf_full = xbar + 4;    // NVFP4: scale buffer b holds the current stage's scales
   uint64_t* sf_empty = sf_full + 2;   // NVFP4: the MMAs reading scale buffer b completed
   uint64_t* sf_final = sf_empty + 2;  // NVFP4: the copier's last copies completed
+  uint64_t* hbar = sf_final + 1;      // FP8 L1: one per TMEM lane quarter (h rows staged)
   float* xbuf = reinterpret_cast<float*>(smem + S * SB + 1024);  // FP8 L1: [2][2][128] amax
   float* xpose = reinterpret_cast<float*>(smem + S * SB + Cfg::kBarrierBytes);  // L2: per-warp 32 x 32
 
@@ -272,6 +323,7 @@ __device__ __forceinline__ void gemm_phase(const GemmArgs& p, const CUtensorMap*
       mbar_init(&sf_empty[i], 1);
     }
     mbar_init(sf_final, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&hbar[i], 64);
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) prefetch_tensormap(tmA);
@@ -461,7 +513,7 @@ __device__ __forceinline__ void gemm_phase(const GemmArgs& p, const CUtensorMap*
     int xpar = 0;          // FP8 L1: amax exchange buffer / barrier phase
     for (int T = cta; T < total; T += ncta) {
       TileInfo t;
-      decode_tile(p, na, T, t);
+      decode_tile_warp(p, na, T, t, lane);
       const bool valid = row_local < t.rows;
       const int r = t.row0 + row_local;
       const int pr = t.srow0 + row_local;
@@ -558,8 +610,7 @@ __device__ __forceinline__ void gemm_phase(const GemmArgs& p, const CUtensorMap*
         // h for intermediate columns j0 + 64*half + i, i < 64
         const int hcol0 = t.n_tile * 128 + half * 64;
         float h[64];
-#pragma unroll
-        for (int i = 0; i < 64; ++i) h[i] = clamped_swiglu(acc[i], acc[64 + i], p.clamp, p.fast_math);
+        swiglu_row(acc, h, p.clamp, p.fast_math);
         uint8_t* hrow = p.h_out + static_cast<size_t>(r) * p.h_row_bytes;
         if constexpr (FMT == FMT_FP8) {
           float amax = 0.0f;
@@ -576,19 +627,32 @@ __device__ __forceinline__ void gemm_phase(const GemmArgs& p, const CUtensorMap*
           xpar ^= 1;
           const float s = __fdiv_rn(amax, 448.0f);
           const float inv = (s != 0.0f) ? __frcp_rn(s) : 0.0f;
-          if (valid) {
-            uint32_t w[16];
+          uint32_t w[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const uint32_t lo = cvt_e4m3x2(__fmul_rn(h[4 * i], inv), __fmul_rn(h[4 * i + 1], inv));
-              const uint32_t hi =
-                  cvt_e4m3x2(__fmul_rn(h[4 * i + 2], inv), __fmul_rn(h[4 * i + 3], inv));
-              w[i] = (s != 0.0f) ? (lo | (hi << 16)) : 0u;
-            }
-            uint4* dst = reinterpret_cast<uint4*>(hrow + hcol0);
+          for (int i = 0; i < 16; ++i) {
+            const uint32_t lo = cvt_e4m3x2(__fmul_rn(h[4 * i], inv), __fmul_rn(h[4 * i + 1], inv));
+            const uint32_t hi = cvt_e4m3x2(__fmul_rn(h[4 * i + 2], inv), __fmul_rn(h[4 * i + 3], inv));
+            w[i] = (s != 0.0f) ? (lo | (hi << 16)) : 0u;
+          }
+          // this thread's 64 bytes into the quarter's staging rows; once both
+          // warps of the quarter are in, each stores 16 whole rows (8 lanes
+          // x 16 bytes per row, 4 rows per instruction)
+          uint8_t* stg = reinterpret_cast<uint8_t*>(xpose) + q * (32 * Cfg::kHStageStride);
+          uint4* srow = reinterpret_cast<uint4*>(stg + lane * Cfg::kHStageStride + half * 64);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
-            if (half == 0) p.h_scale_t[static_cast<size_t>(t.n_tile) * p.h_scale_ld + pr] = s;
+          for (int i = 0; i < 4; ++i) srow[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+          if (valid && half == 0) p.h_scale_t[static_cast<size_t>(t.n_tile) * p.h_scale_ld + pr] = s;
+          mbar_arrive(&hbar[q]);
+          if (!mbar_wait(&hbar[q], static_cast<uint32_t>(xpar ^ 1), abort_flag, p.status, 11)) break;
+          const int rows_here = t.rows - q * 32;
+          uint8_t* hbase = p.h_out + static_cast<size_t>(t.row0 + q * 32) * p.h_row_bytes + t.n_tile * 128;
+#pragma unroll
+          for (int it = 0; it < 4; ++it) {
+            const int row = half * 16 + it * 4 + (lane >> 3);
+            const int c16 = lane & 7;
+            const uint4 v = *reinterpret_cast<const uint4*>(stg + row * Cfg::kHStageStride + c16 * 16);
+            if (row < rows_here)
+              *reinterpret_cast<uint4*>(hbase + static_cast<size_t>(row) * p.h_row_bytes + c16 * 16) = v;
           }
         } else if constexpr (FMT == FMT_BF16) {
           if (valid) {
