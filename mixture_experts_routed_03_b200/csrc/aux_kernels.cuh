@@ -122,6 +122,7 @@ __global__ void __launch_bounds__(256) route_kernel(RouteArgs a) {
 // ---------------------------------------------------------------------------
 constexpr int kPermChunk = 1024;
 constexpr int kPermSmallMax = 16384;
+constexpr int kPermBatch = 8;       // rounds of 32 slots whose loads one warp issues together
 constexpr int kPermSmallMaxE = 256;
 
 struct PermOut {
@@ -303,17 +304,27 @@ __device__ void perm_small_block(const PermArgs& a, int* sm) {
   const int per = (R + nw - 1) / nw;
   const int b0 = min(R, warp * per), b1 = min(R, b0 + per);
   int* my = hist + warp * E;
-  for (int base = b0; base < b1; base += 32) {
-    const int s = base + lane;
-    int v = -1;
-    if (s < b1) {
-      const int64_t x = a.idx[s];
-      if (x >= 0 && x < E) v = static_cast<int>(x);
-      else if (x != -1) record_error(a.status, MOE_ERR_BAD_INDEX);
+  // Each warp's slots go in batches of kPermBatch rounds of 32: the batch's
+  // index loads are issued together, so a batch costs one memory latency.
+  for (int base = b0; base < b1; base += 32 * kPermBatch) {
+    int v[kPermBatch];
+#pragma unroll
+    for (int j = 0; j < kPermBatch; ++j) {
+      const int s = base + 32 * j + lane;
+      v[j] = -1;
+      if (s < b1) {
+        const int64_t x = a.idx[s];
+        if (x >= 0 && x < E) v[j] = static_cast<int>(x);
+        else if (x != -1) record_error(a.status, MOE_ERR_BAD_INDEX);
+      }
     }
-    const unsigned peers = __match_any_sync(0xFFFFFFFFu, v >= 0 ? v : E + lane);
-    if (v >= 0 && lane == 31 - __clz(peers)) my[v] += __popc(peers);
-    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < kPermBatch; ++j) {
+      if (base + 32 * j >= b1) break;
+      const unsigned peers = __match_any_sync(0xFFFFFFFFu, v[j] >= 0 ? v[j] : E + lane);
+      if (v[j] >= 0 && lane == 31 - __clz(peers)) my[v[j]] += __popc(peers);
+      __syncwarp();
+    }
   }
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
@@ -334,23 +345,32 @@ __device__ void perm_small_block(const PermArgs& a, int* sm) {
   }
   __syncthreads();
   write_expert_arrays(total, start, tmp, tmp2, E, a.o);
-  for (int base = b0; base < b1; base += 32) {
-    const int s = base + lane;
-    int v = -1;
-    if (s < b1) {
-      const int64_t x = a.idx[s];
-      if (x >= 0 && x < E) v = static_cast<int>(x);
+  for (int base = b0; base < b1; base += 32 * kPermBatch) {
+    int v[kPermBatch];
+#pragma unroll
+    for (int j = 0; j < kPermBatch; ++j) {
+      const int s = base + 32 * j + lane;
+      v[j] = -1;
+      if (s < b1) {
+        const int64_t x = a.idx[s];
+        if (x >= 0 && x < E) v[j] = static_cast<int>(x);
+      }
     }
-    const unsigned peers = __match_any_sync(0xFFFFFFFFu, v >= 0 ? v : E + lane);
-    int row = -1;
-    if (v >= 0) {
-      row = my[v] + __popc(peers & lt);
-      a.o.src_info[row] = s;
+#pragma unroll
+    for (int j = 0; j < kPermBatch; ++j) {
+      if (base + 32 * j >= b1) break;
+      const int s = base + 32 * j + lane;
+      const unsigned peers = __match_any_sync(0xFFFFFFFFu, v[j] >= 0 ? v[j] : E + lane);
+      int row = -1;
+      if (v[j] >= 0) {
+        row = my[v[j]] + __popc(peers & lt);
+        a.o.src_info[row] = s;
+      }
+      if (s < b1) a.o.slot_to_row[s] = row;
+      __syncwarp();
+      if (v[j] >= 0 && lane == 31 - __clz(peers)) my[v[j]] += __popc(peers);
+      __syncwarp();
     }
-    if (s < b1) a.o.slot_to_row[s] = row;
-    __syncwarp();
-    if (v >= 0 && lane == 31 - __clz(peers)) my[v] += __popc(peers);
-    __syncwarp();
   }
   __syncthreads();
 }

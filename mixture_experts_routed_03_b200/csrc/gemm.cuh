@@ -33,8 +33,9 @@
 // half, one row per thread.
 //
 // Tiles are (active expert, n tile, 128-row m tile), handed out round-robin
-// over at most one CTA per SM: expert-major with m fastest for gate_up,
-// n-major for down (see decode_tile).
+// over at most one CTA per SM, in groups of n tiles (see decode_tile):
+// expert-major with m fastest for gate_up, a few output n tiles at a time for
+// down.
 //
 // L1 epilogue: h = min(g,c) * sigmoid(min(g,c)) * clamp(u,-c,c) is formed in
 // registers, the accumulator is released, then h is re-quantised (BF16 by
@@ -117,7 +118,7 @@ struct GemmCfg {
 struct GemmArgs {
   int k_stages;       // K bytes / 128
   int n_tiles;        // tiles along N: I/128 (L1, 128 h columns per tile) or H/256 (L2)
-  int n_major;        // tile order: 1 n-major, 0 expert-major (see decode_tile)
+  int n_group;        // n tiles per group of the tile order (1 .. n_tiles, see decode_tile)
   int I, H, topk;
   float clamp;
   int fast_math;
@@ -162,37 +163,40 @@ struct TileInfo {
   int n_tile;
 };
 
-// Tile T -> (expert, m tile, n tile).  Expert-major order: concurrent CTAs
-// share one expert's activation panel and weight tiles.  N-major order (the
-// down leg when its whole A operand fits in L2): concurrent CTAs add into the
-// same 256 output columns of every token, a slice of the FP32 accumulator
-// that stays in L2.
-// Search key of tile T: n-major order gives the n tile directly and keys the
-// expert search by m tile; expert-major order keys it by T itself.
-__device__ __forceinline__ int tile_key(const GemmArgs& p, int na, int T, TileInfo& t, int& scale) {
-  if (p.n_major != 0) {
-    const int total_mt = __ldg(p.tile_offsets + na);
-    t.n_tile = T / total_mt;
-    scale = 1;
-    return T - t.n_tile * total_mt;
+// Tile T -> (expert, m tile, n tile).  The n tiles are taken in groups of
+// n_group; inside a group the order is expert-major with m fastest, so
+// concurrently running CTAs share one expert's activation panel and weight
+// tiles.  One group of all n tiles is plain expert-major order (gate_up).
+// The down leg adds into the FP32 accumulator: with n_group small the CTAs
+// work on an accumulator slice of n_group*256 columns of every token at a
+// time, which stays in L2, at the price of reading the intermediate once per
+// group.
+
+// Search key of tile T inside its group, the group's width `scale` (the
+// multiplier of tile_offsets) and its first n tile.
+__device__ __forceinline__ int tile_key(const GemmArgs& p, int na, int T, int& scale, int& nbase) {
+  const int G = p.n_group;
+  if (G >= p.n_tiles) {
+    scale = p.n_tiles;
+    nbase = 0;
+    return T;
   }
-  scale = p.n_tiles;
-  return T;
+  const int per_group = __ldg(p.tile_offsets + na) * G;
+  const int gi = T / per_group;
+  nbase = gi * G;
+  scale = min(G, p.n_tiles - nbase);
+  return T - gi * per_group;
 }
 
-// The rest of the decode once the active-expert slot `lo` of tile T is known
+// The rest of the decode once the active-expert slot `lo` of the key is known
 // (tile_offsets[lo]*scale <= g < tile_offsets[lo+1]*scale).
-__device__ __forceinline__ void tile_finish(const GemmArgs& p, int lo, int g, int T, TileInfo& t) {
+__device__ __forceinline__ void tile_finish(const GemmArgs& p, int lo, int g, int scale, int nbase, TileInfo& t) {
   const int mt0 = __ldg(p.tile_offsets + lo);
-  int mt;
-  if (p.n_major != 0) {
-    mt = g - mt0;
-  } else {
-    const int nm = __ldg(p.tile_offsets + lo + 1) - mt0;
-    const int local = T - mt0 * p.n_tiles;
-    t.n_tile = local / nm;
-    mt = local - t.n_tile * nm;
-  }
+  const int nm = __ldg(p.tile_offsets + lo + 1) - mt0;
+  const int local = g - mt0 * scale;
+  const int n_in = local / nm;
+  const int mt = local - n_in * nm;
+  t.n_tile = nbase + n_in;
   t.e = __ldg(p.expert_ids + lo);
   const int start = __ldg(p.starts + t.e);
   const int cnt = __ldg(p.starts + t.e + 1) - start;
@@ -204,22 +208,22 @@ __device__ __forceinline__ void tile_finish(const GemmArgs& p, int lo, int g, in
 // Tile T -> (expert, m tile, n tile) by one thread: binary search over the
 // active experts' tile offsets.
 __device__ __forceinline__ void decode_tile(const GemmArgs& p, int na, int T, TileInfo& t) {
-  int scale;
-  const int g = tile_key(p, na, T, t, scale);
+  int scale, nbase;
+  const int g = tile_key(p, na, T, scale, nbase);
   int lo = 0, hi = na;  // tile_offsets[lo]*scale <= g < tile_offsets[hi]*scale
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
     if (__ldg(p.tile_offsets + mid) * scale <= g) lo = mid; else hi = mid;
   }
-  tile_finish(p, lo, g, T, t);
+  tile_finish(p, lo, g, scale, nbase, t);
 }
 
 // The same decode by a whole converged warp: each round probes 32 evenly
 // spaced offsets at once and keeps the bucket the key falls in, so up to
 // 1024 active experts take two dependent loads instead of ten.
 __device__ __forceinline__ void decode_tile_warp(const GemmArgs& p, int na, int T, TileInfo& t, int lane) {
-  int scale;
-  const int g = tile_key(p, na, T, t, scale);
+  int scale, nbase;
+  const int g = tile_key(p, na, T, scale, nbase);
   int base = 0, len = na;  // the slot lies in [base, base + len); offsets[base]*scale <= g
   while (len > 1) {
     const int step = (len + 31) >> 5;
@@ -229,7 +233,7 @@ __device__ __forceinline__ void decode_tile_warp(const GemmArgs& p, int na, int 
     base += j * step;
     len = min(step, len - j * step);
   }
-  tile_finish(p, base, g, T, t);
+  tile_finish(p, base, g, scale, nbase, t);
 }
 
 // A wait used while tearing down after an abort: ignores the abort flag.
@@ -517,6 +521,12 @@ __device__ __forceinline__ void gemm_phase(const GemmArgs& p, const CUtensorMap*
       const bool valid = row_local < t.rows;
       const int r = t.row0 + row_local;
       const int pr = t.srow0 + row_local;
+      // Down leg: the row's flat slot is loaded now and its router weight
+      // once the first partial has been taken, so neither load's latency
+      // falls on the epilogue's tail.
+      const bool gather_wgt = EPI == EPI_L2_ACC && valid;
+      const int s_flat = gather_wgt ? __ldg(p.src_info + r) : 0;
+      float wgt = 1.0f;
 
       // acc[0..127]: this thread's row, columns 128*half .. 128*half+127 of
       // the tile (L1: 64 gate then 64 up; L2: output columns)
@@ -565,12 +575,14 @@ __device__ __forceinline__ void gemm_phase(const GemmArgs& p, const CUtensorMap*
             ab = 0;
             aphase ^= 1u;
           }
+          if (ks == 0 && gather_wgt) wgt = __ldg(p.topk_weights + s_flat);
         }
         if (!ok) break;
       } else {
         // BF16 / NVFP4: the whole K sum is in TMEM; read it, release it.
         if (!mbar_wait(&acc_full[ab], aphase, abort_flag, p.status, 6)) break;
         tc_fence_after();
+        if (gather_wgt) wgt = __ldg(p.topk_weights + s_flat);
         const uint32_t base = tmem + ab * kBN + half * 128 + lane_off;
         {
           // all 128 columns in one TMEM round trip
@@ -696,18 +708,37 @@ __device__ __forceinline__ void gemm_phase(const GemmArgs& p, const CUtensorMap*
             *reinterpret_cast<uint32_t*>(p.h_sf + sf_tile_offset(pr, hcol0 >> 4, p.h_sf_kc)) = sfw;
           }
         }
-      } else {
-        // L2: write the rows through a per-warp 32 x 32 transpose so that one
-        // warp instruction covers four whole 128-byte row segments (8 lanes
-        // per row) instead of 32 scattered 16-byte pieces.
+      } else if constexpr (EPI == EPI_L2_ACC && FMT == FMT_NVFP4) {
+        // L2, accumulate (NVFP4): each thread's router-weighted row segment goes
+        // through its own 128-byte shared-memory slot into asynchronous bulk
+        // reduce-adds (32 columns each) on the token's FP32 accumulator row;
+        // the warp moves on to the next tile while the TMA engine finishes
+        // the reductions.
         const int n0 = t.n_tile * kBN + half * 128;
-        int tok = r;
-        float wgt = 1.0f;
-        if (valid && EPI == EPI_L2_ACC) {
-          const int s_flat = __ldg(p.src_info + r);
-          tok = s_flat / p.topk;
-          wgt = __ldg(p.topk_weights + s_flat);
+        const int tok = gather_wgt ? s_flat / p.topk : r;
+        float* slot = xpose + (ew * 32 + lane) * Cfg::kXposeStride;
+        float* grow = p.out + static_cast<size_t>(tok) * p.H + n0;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          bulk_wait_read();   // the slot's previous contents have been read
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            reinterpret_cast<float4*>(slot)[i] =
+                make_float4(acc[32 * c + 4 * i] * wgt, acc[32 * c + 4 * i + 1] * wgt,
+                            acc[32 * c + 4 * i + 2] * wgt, acc[32 * c + 4 * i + 3] * wgt);
+          fence_async_smem();
+          if (valid) {
+            bulk_reduce_add_f32(grow + 32 * c, slot, 128);
+            bulk_commit();
+          }
         }
+      } else {
+        // L2, staged or accumulate: write the rows through a per-warp 32 x 32
+        // transpose so that one warp instruction covers four whole 128-byte
+        // row segments (8 lanes per row) instead of 32 scattered 16-byte
+        // pieces; accumulate mode adds them with float4 atomics.
+        const int n0 = t.n_tile * kBN + half * 128;
+        const int tok = gather_wgt ? s_flat / p.topk : r;
         float* xb = xpose + ew * (32 * Cfg::kXposeStride);
         const int rows_here = t.rows - q * 32;   // valid rows of this warp's quarter
 #pragma unroll
@@ -727,15 +758,16 @@ __device__ __forceinline__ void gemm_phase(const GemmArgs& p, const CUtensorMap*
             const float4 v = *reinterpret_cast<const float4*>(xb + row * Cfg::kXposeStride + 4 * c4);
             if (row < rows_here) {
               float4* dst = reinterpret_cast<float4*>(p.out + static_cast<size_t>(rtok) * p.H + n0 + 32 * c) + c4;
-              const float4 o = make_float4(v.x * rw, v.y * rw, v.z * rw, v.w * rw);
-              if (EPI == EPI_L2_ACC) atomicAdd(dst, o);
-              else *dst = o;
+              if (EPI == EPI_L2_ACC) atomicAdd(dst, make_float4(v.x * rw, v.y * rw, v.z * rw, v.w * rw));
+              else *dst = v;
             }
           }
           __syncwarp();
         }
       }
     }
+    // every bulk reduction of this thread has landed before the phase ends
+    if (EPI == EPI_L2_ACC && FMT == FMT_NVFP4) bulk_wait_done();
   }
 
   tc_fence_before();

@@ -344,6 +344,7 @@ moe_status_t plan_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_we
   a = GemmArgs{};
   a.k_stages = x_row_bytes(fmt, H) / 128;
   a.n_tiles = I / 128;
+  a.n_group = a.n_tiles;   // expert-major
   a.wB = static_cast<const uint8_t*>(w->w13);
   a.I = I;
   a.H = H;
@@ -382,10 +383,15 @@ moe_status_t plan_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_we
   a2 = a;
   a2.k_stages = h_row_bytes(fmt, I) / 128;
   a2.n_tiles = H / 256;
-  // n-major keeps one 256-column slice of the FP32 accumulator hot in L2, at
-  // the price of re-reading the whole intermediate once per slice: worth it
-  // while the intermediate fits in L2 with room to spare
-  a2.n_major = (size_t(R) * h_row_bytes(fmt, I) <= (size_t(48) << 20)) ? 1 : 0;
+  // Output n tiles in groups: a group's slice of the FP32 accumulator
+  // (M x 256*group floats) stays in L2 while its tiles add into it, and the
+  // intermediate is read once per group.  While the intermediate itself fits
+  // in L2 the re-reads are free and one n tile per group is best.
+  // (Measured on FP8, M = 16384, 16 n tiles: groups of 3 were 8% slower
+  // than plain expert-major order, so when the intermediate does not fit the
+  // order stays expert-major.)
+  const size_t kL2Budget = size_t(48) << 20;
+  a2.n_group = (size_t(R) * h_row_bytes(fmt, I) <= kL2Budget) ? 1 : a2.n_tiles;
   a2.wB = static_cast<const uint8_t*>(w->w2);
   a2.sfa = b.h_sf;
   a2.sfa_kc = I / 64;
