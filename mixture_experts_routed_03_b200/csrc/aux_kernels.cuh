@@ -151,62 +151,77 @@ __host__ __device__ inline bool perm_small_case(int64_t R, int E) {
 }
 
 // Shared-memory ints of the two-pass (per chunk) and the one-block permutation.
-__host__ __device__ inline int perm_chunk_smem_ints(int E) { return 5 * E + 3 + kPermChunk; }
-__host__ __device__ inline int perm_small_smem_ints(int E, int nwarps) { return nwarps * E + 4 * E + 3; }
+__host__ __device__ inline int perm_chunk_smem_ints(int E) { return 3 * E + 1 + kPermChunk; }
+__host__ __device__ inline int perm_small_smem_ints(int E, int nwarps) { return nwarps * E + 2 * E + 1; }
 
 // Exclusive scan of v[0..n) by one warp (n <= 1024); writes out[0..n] (n+1
 // entries, out[n] = total).  Each lane owns a contiguous run of entries.
-__device__ void warp_exclusive_scan(const int* v, int* out, int n) {
-  const int lane = threadIdx.x & 31;
-  const int per = (n + 31) / 32;
-  const int b = min(n, lane * per), e = min(n, b + per);
-  int local = 0;
-  for (int i = b; i < e; ++i) local += v[i];
-  int incl = local;
+// One warp turns the per-expert totals (shared memory, E entries) into
+// start[0..E] (shared memory: the exclusive scan, start[E] = routed rows) and,
+// when `tables` is set, the layout arrays in global memory: expert_counts,
+// expert_start_indices, a_scale_offsets (scan of the counts padded to 128),
+// expert_ids (active experts in order, -1 after them), num_active and
+// tile_offsets (scan of the active experts' 128-row m tiles).  The four scans
+// run together: each lane takes E/32 consecutive experts, sums them, and one
+// round of shuffles scans the four sums at once.
+__device__ void expert_tables_warp(const int* total, int* start, int E, const PermOut& o, bool tables, int lane) {
+  const int per = (E + 31) >> 5;
+  const int b = min(E, lane * per), e_end = min(E, b + per);
+  int c = 0, pad = 0, act = 0, mt = 0;
+  for (int e = b; e < e_end; ++e) {
+    const int t = total[e];
+    const int m = (t + 127) >> 7;
+    c += t;
+    pad += m << 7;
+    act += t > 0 ? 1 : 0;
+    mt += m;
+  }
+  int ic = c, ip = pad, ia = act, im = mt;
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
-    const int o = __shfl_up_sync(0xFFFFFFFFu, incl, off);
-    if (lane >= off) incl += o;
-  }
-  int run = incl - local;
-  for (int i = b; i < e; ++i) {
-    out[i] = run;
-    run += v[i];
-  }
-  if (lane == 31) out[n] = incl;
-}
-
-// Writes expert_counts, expert_start_indices, a_scale_offsets, expert_ids,
-// num_active and tile_offsets from the per-expert totals and their exclusive
-// scan (start, E+1 entries).  Called by every thread of one block; tmp and
-// tmp2 are E+1-entry shared scratch arrays.
-__device__ void write_expert_arrays(const int* total, const int* start, int* tmp, int* tmp2, int E,
-                                    const PermOut& o) {
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    o.expert_counts[e] = total[e];
-    o.expert_start_indices[e] = start[e];
-    tmp[e] = (total[e] + 127) / 128 * 128;  // padded rows
-    tmp2[e] = (total[e] > 0) ? 1 : 0;
-  }
-  if (threadIdx.x == 0) o.expert_start_indices[E] = start[E];
-  __syncthreads();
-  if (threadIdx.x < 32) warp_exclusive_scan(tmp, o.a_scale_offsets, E);
-  __syncthreads();
-  // active experts: compact with a scan of the flags (tmp becomes the ranks)
-  if (threadIdx.x < 32) warp_exclusive_scan(tmp2, tmp, E);
-  __syncthreads();
-  const int na = tmp[E];
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    if (total[e] > 0) {
-      o.expert_ids[tmp[e]] = e;
-      tmp2[tmp[e]] = (total[e] + 127) / 128;  // m tiles of the a-th active expert
+    const int xc = __shfl_up_sync(0xFFFFFFFFu, ic, off);
+    const int xp = __shfl_up_sync(0xFFFFFFFFu, ip, off);
+    const int xa = __shfl_up_sync(0xFFFFFFFFu, ia, off);
+    const int xm = __shfl_up_sync(0xFFFFFFFFu, im, off);
+    if (lane >= off) {
+      ic += xc;
+      ip += xp;
+      ia += xa;
+      im += xm;
     }
-    if (e >= na) o.expert_ids[e] = -1;
   }
-  if (threadIdx.x == 0) *o.num_active = na;
-  __syncthreads();
-  if (threadIdx.x < 32) warp_exclusive_scan(tmp2, o.tile_offsets, na);
-  __syncthreads();
+  const int na = __shfl_sync(0xFFFFFFFFu, ia, 31);
+  int rc = ic - c, rp = ip - pad, ra = ia - act, rm = im - mt;   // exclusive bases of this lane
+  for (int e = b; e < e_end; ++e) {
+    const int t = total[e];
+    const int m = (t + 127) >> 7;
+    start[e] = rc;
+    if (tables) {
+      o.expert_counts[e] = t;
+      o.expert_start_indices[e] = rc;
+      o.a_scale_offsets[e] = rp;
+      if (t > 0) {
+        o.expert_ids[ra] = e;
+        o.tile_offsets[ra] = rm;
+      }
+      if (e >= na) o.expert_ids[e] = -1;
+    }
+    rc += t;
+    rp += m << 7;
+    if (t > 0) {
+      ++ra;
+      rm += m;
+    }
+  }
+  if (lane == 31) {
+    start[E] = ic;
+    if (tables) {
+      o.expert_start_indices[E] = ic;
+      o.a_scale_offsets[E] = ip;
+      *o.num_active = na;
+      o.tile_offsets[na] = im;
+    }
+  }
 }
 
 // Pass 1 of the large case for chunk c.
@@ -235,9 +250,7 @@ __device__ void perm_scatter_chunk(const PermArgs& a, int c, int* sm) {
   int* total = sm;                 // [E]
   int* start = total + E;          // [E+1]
   int* cursor = start + E + 1;     // [E]
-  int* tmp = cursor + E;           // [E+1]
-  int* tmp2 = tmp + E + 1;         // [E+1]
-  int* sidx = tmp2 + E + 1;        // [kPermChunk] this chunk's expert ids
+  int* sidx = cursor + E;          // [kPermChunk] this chunk's expert ids
   const int64_t base = static_cast<int64_t>(c) * kPermChunk;
   for (int i = threadIdx.x; i < kPermChunk; i += blockDim.x) {
     const int64_t s = base + i;
@@ -259,10 +272,9 @@ __device__ void perm_scatter_chunk(const PermArgs& a, int c, int* sm) {
     cursor[e] = before;
   }
   __syncthreads();
-  if (threadIdx.x < 32) warp_exclusive_scan(total, start, E);
+  if (threadIdx.x < 32) expert_tables_warp(total, start, E, a.o, c == 0, threadIdx.x);
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) cursor[e] += start[e];
-  if (c == 0) write_expert_arrays(total, start, tmp, tmp2, E, a.o);
   __syncthreads();
   if (threadIdx.x < 32) {
     const int lane = threadIdx.x;
@@ -292,11 +304,9 @@ __device__ void perm_small_block(const PermArgs& a, int* sm) {
   const int E = a.E;
   const int R = static_cast<int>(a.R);
   const int nw = blockDim.x >> 5;
-  int* hist = sm;                  // [nw][E]: counts, then each warp's running cursor
+  int* hist = sm;                  // [nw][E]: counts, then each warp's running offset inside the expert
   int* total = hist + nw * E;      // [E]
   int* start = total + E;          // [E+1]
-  int* tmp = start + E + 1;        // [E+1]
-  int* tmp2 = tmp + E + 1;         // [E+1]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const unsigned lt = (1u << lane) - 1u;
   for (int i = threadIdx.x; i < nw * E; i += blockDim.x) hist[i] = 0;
@@ -304,10 +314,12 @@ __device__ void perm_small_block(const PermArgs& a, int* sm) {
   const int per = (R + nw - 1) / nw;
   const int b0 = min(R, warp * per), b1 = min(R, b0 + per);
   int* my = hist + warp * E;
-  // Each warp's slots go in batches of kPermBatch rounds of 32: the batch's
-  // index loads are issued together, so a batch costs one memory latency.
+  // Each warp's slots go in batches of kPermBatch rounds of 32: a batch's
+  // index loads are issued together.  A warp whose slots fit in one batch
+  // keeps them in registers for the second pass.
+  const bool one_batch = b1 - b0 <= 32 * kPermBatch;
+  int v[kPermBatch];
   for (int base = b0; base < b1; base += 32 * kPermBatch) {
-    int v[kPermBatch];
 #pragma unroll
     for (int j = 0; j < kPermBatch; ++j) {
       const int s = base + 32 * j + lane;
@@ -327,33 +339,30 @@ __device__ void perm_small_block(const PermArgs& a, int* sm) {
     }
   }
   __syncthreads();
+  // per expert: each warp's offset inside the expert (exclusive over warps)
+  // and the expert's total
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    int t = 0;
-    for (int w = 0; w < nw; ++w) t += hist[w * E + e];
-    total[e] = t;
-  }
-  __syncthreads();
-  if (threadIdx.x < 32) warp_exclusive_scan(total, start, E);
-  __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    int run = start[e];
+    int run = 0;
     for (int w = 0; w < nw; ++w) {
       const int c = hist[w * E + e];
       hist[w * E + e] = run;
       run += c;
     }
+    total[e] = run;
   }
   __syncthreads();
-  write_expert_arrays(total, start, tmp, tmp2, E, a.o);
+  if (warp == 0) expert_tables_warp(total, start, E, a.o, true, lane);
+  __syncthreads();
   for (int base = b0; base < b1; base += 32 * kPermBatch) {
-    int v[kPermBatch];
+    if (!one_batch) {
 #pragma unroll
-    for (int j = 0; j < kPermBatch; ++j) {
-      const int s = base + 32 * j + lane;
-      v[j] = -1;
-      if (s < b1) {
-        const int64_t x = a.idx[s];
-        if (x >= 0 && x < E) v[j] = static_cast<int>(x);
+      for (int j = 0; j < kPermBatch; ++j) {
+        const int s = base + 32 * j + lane;
+        v[j] = -1;
+        if (s < b1) {
+          const int64_t x = a.idx[s];
+          if (x >= 0 && x < E) v[j] = static_cast<int>(x);
+        }
       }
     }
 #pragma unroll
@@ -363,7 +372,7 @@ __device__ void perm_small_block(const PermArgs& a, int* sm) {
       const unsigned peers = __match_any_sync(0xFFFFFFFFu, v[j] >= 0 ? v[j] : E + lane);
       int row = -1;
       if (v[j] >= 0) {
-        row = my[v[j]] + __popc(peers & lt);
+        row = start[v[j]] + my[v[j]] + __popc(peers & lt);
         a.o.src_info[row] = s;
       }
       if (s < b1) a.o.slot_to_row[s] = row;
