@@ -33,6 +33,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 DEFAULT_WORKLOAD = "fp8_block"
+METRIC = "routed tokens/sec and achieved TFLOPS (% of roofline) per MoE layer, 1 B200"
 FLUSH_BYTES = 512 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FMT_TENSOR_RATIO = {"bf16": 1.0, "fp8": 2.0, "nvfp4": 4.0}   # nominal dense ratio to bf16
@@ -434,7 +435,7 @@ def main_ours(args):
         unit = "GB/s"
     total_k = sum(v[0] for v in kern.values()) or 1.0
     line = {
-        "metric": "routed tokens/sec per MoE layer (moe_fused), 1 B200 per rank",
+        "metric": METRIC,
         "value": value,
         "unit": "routed_tokens/s",
         "n_gpus": world,
@@ -535,7 +536,7 @@ def main_reference(args):
     sample = f"{n} of {M} tokens per step ({n * k} routed slots), float64 numpy oracle"
     line = {
         "impl": "reference",
-        "metric": "routed tokens/sec per MoE layer (moe_fused), 1 B200 per rank",
+        "metric": METRIC,
         "value": value, "unit": "routed_tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64",
