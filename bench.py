@@ -356,7 +356,9 @@ def run_ours(args, rank, world, local_rank):
 
     # ---- max over ranks
     t_ms, e2e_ms = max_over_ranks([t_ms, e2e_ms], world, dev)
+    regime = api.tile_regime(L.problem(M))
     return dict(p=p, t_ms=t_ms, per_step=per_step, kern=kern, launches=launches, e2e_ms=e2e_ms, phases=phases,
+                regime=regime,
                 h2d=h2d, d2h=d2h, num_active=num_active, clocks=clocks.summary(), R=R, M=M,
                 host_inputs=(d, L) if rank == 0 else None)
 
@@ -453,7 +455,8 @@ def main_ours(args):
                    "num_tokens": p["num_tokens"], "hidden": p["hidden"],
                    "intermediate_hidden": p["intermediate_hidden"], "num_experts": p["num_experts"],
                    "num_topk": p["num_topk"], "format": p["format"], "routing": p["routing"],
-                   "active_experts": r["num_active"], "parallelism": f"dp{world} (replicas)",
+                   "active_experts": r["num_active"], "gemm_tiles": r["regime"],
+                   "parallelism": f"dp{world} (replicas)",
                    "l2": "flushed (512 MiB write) before every timed step, outside the step interval"},
         "tokens_per_s": job_throughput(p["num_tokens"], world, args.steps, r["t_ms"]),
         "layer_tflops": wm["layer"]["flops"] / (step_ms / 1e3) / 1e12,

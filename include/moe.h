@@ -92,7 +92,7 @@ typedef enum {
 
 /* The problem statement, after flashinfer.megamoe.MegaMoESymmBuffer
  * (num_experts, num_topk, hidden, intermediate_hidden, activation_clamp,
- * fast_math). */
+ * fast_math), plus the GEMM tile regime. */
 typedef struct {
   int64_t num_tokens;           /* M >= 0 */
   int32_t hidden;               /* H, multiple of 256 */
@@ -102,7 +102,22 @@ typedef struct {
   float activation_clamp;       /* c of the clamped SwiGLU; +inf disables the clamp */
   int32_t format;               /* moe_format_t */
   int32_t fast_math;            /* nonzero: the SiLU uses the fast exponential */
+  int32_t tile_regime;          /* moe_tile_regime_t: the grouped GEMMs' tile shape */
 } moe_problem_t;
+
+/* Tile shape of the grouped GEMMs (the tile-regime choice the pages make
+ * between prefill and decode batches).  AUTO picks SMALL_M for BF16 and FP8
+ * when the routed rows average at most 64 per expert (num_tokens*num_topk <=
+ * 64*num_experts), else LARGE_M.  LARGE_M: 128 routed rows x 256 weight rows
+ * per tile.  SMALL_M: the operands swapped, 256 weight rows x 32 routed rows
+ * per tile, so the tensor work follows the routed rows that exist; BF16 and
+ * FP8 only (MOE_ERR_UNSUPPORTED for NVFP4).  Results agree between regimes
+ * up to FP32 summation order. */
+typedef enum {
+  MOE_TILE_AUTO = 0,
+  MOE_TILE_LARGE_M = 1,
+  MOE_TILE_SMALL_M = 2
+} moe_tile_regime_t;
 
 /* Activations (device).  x_scale is NULL for BF16. */
 typedef struct {
@@ -176,6 +191,11 @@ moe_status_t moe_get_workspace_size(const moe_problem_t* problem, size_t* bytes)
 /* Zeroes the workspace header (the sticky status word).  Call once after
  * allocating a workspace and after moe_read_status reported an error. */
 moe_status_t moe_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
+
+/* The tile regime (moe_tile_regime_t, MOE_TILE_LARGE_M or MOE_TILE_SMALL_M)
+ * the grouped GEMMs of this problem use once MOE_TILE_AUTO is resolved
+ * (tile regimes of the pages' prefill and decode batches; host only). */
+moe_status_t moe_get_tile_regime(const moe_problem_t* problem, int32_t* regime);
 
 /* Bytes of the prepared gate_up and down weight blobs. */
 moe_status_t moe_get_prepared_weights_size(const moe_problem_t* problem, size_t* w13_bytes,

@@ -39,7 +39,7 @@ EXPORTS = (
     "moe_get_prepared_weights_size",
     "moe_route", "moe_permute", "moe_ffn", "moe_get_intermediate_size", "moe_combine",
     "moe_fused", "moe_read_status", "moe_status_string", "moe_timing_enable", "moe_timing_read",
-    "moe_permute_noalloc",
+    "moe_permute_noalloc", "moe_get_tile_regime",
 )
 
 SLOTS = ("route", "permute", "gather", "gemm1", "zero", "gemm2", "finalize", "combine", "fused")
@@ -61,6 +61,7 @@ class Problem(ctypes.Structure):
         ("activation_clamp", ctypes.c_float),
         ("format", ctypes.c_int32),
         ("fast_math", ctypes.c_int32),
+        ("tile_regime", ctypes.c_int32),
     ]
 
 
@@ -108,6 +109,7 @@ def lib():
             "moe_ffn": [P, ctypes.POINTER(Act), ctypes.POINTER(Weights), ctypes.POINTER(Layout),
                         vp, i32, vp, vp, vp, sz, vp],
             "moe_get_intermediate_size": [P, ctypes.POINTER(sz), ctypes.POINTER(sz)],
+            "moe_get_tile_regime": [P, ctypes.POINTER(i32)],
             "moe_combine": [P, ctypes.POINTER(Layout), vp, vp, i32, vp, vp],
             "moe_fused": [P, ctypes.POINTER(Act), ctypes.POINTER(Weights), vp, vp, vp, vp, vp, vp, sz, vp],
             "moe_read_status": [vp, vp],
@@ -154,18 +156,22 @@ def _check(fn, code):
         raise MoEError(fn, code)
 
 
+TILE_REGIMES = {"auto": 0, "large_m": 1, "small_m": 2}
+
+
 def problem(num_tokens, hidden, intermediate_hidden, num_experts, num_topk,
-            activation_clamp=10.0, format="bf16", fast_math=1):
+            activation_clamp=10.0, format="bf16", fast_math=1, tile_regime="auto"):
     fmt = FORMATS[format] if isinstance(format, str) else int(format)
     clamp = float(activation_clamp)
+    regime = TILE_REGIMES[tile_regime] if isinstance(tile_regime, str) else int(tile_regime)
     return Problem(int(num_tokens), int(hidden), int(intermediate_hidden), int(num_experts),
-                   int(num_topk), math.inf if math.isinf(clamp) else clamp, fmt, int(fast_math))
+                   int(num_topk), math.inf if math.isinf(clamp) else clamp, fmt, int(fast_math), regime)
 
 
 def problem_from_dict(d, num_tokens=None, fast_math=1):
     return problem(d["num_tokens"] if num_tokens is None else num_tokens, d["hidden"],
                    d["intermediate_hidden"], d["num_experts"], d["num_topk"],
-                   d.get("activation_clamp", 10.0), d["format"], fast_math)
+                   d.get("activation_clamp", 10.0), d["format"], fast_math, d.get("tile_regime", "auto"))
 
 
 def act(x, x_scale=None):
@@ -194,6 +200,13 @@ def workspace_size(prob):
     n = ctypes.c_size_t(0)
     _check("moe_get_workspace_size", lib().moe_get_workspace_size(ctypes.byref(prob), ctypes.byref(n)))
     return n.value
+
+
+def tile_regime(prob):
+    """'large_m' or 'small_m': the grouped GEMMs' tile shape for this problem."""
+    r = ctypes.c_int32(0)
+    _check("moe_get_tile_regime", lib().moe_get_tile_regime(ctypes.byref(prob), ctypes.byref(r)))
+    return {v: k for k, v in TILE_REGIMES.items()}[r.value]
 
 
 def intermediate_size(prob):

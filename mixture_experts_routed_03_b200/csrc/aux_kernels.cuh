@@ -426,7 +426,37 @@ struct GatherArgs {
   float* sa_t;               // FP8: [H/128][ld]
   uint8_t* sfa;              // NVFP4: tiles [P/128][H/64]
   int ld;                    // padded rows allocated
+  // small-M GEMMs: their tile table (32-row tiles), built here; null otherwise
+  const int* expert_ids;
+  const int* num_active;
+  int* tiles32;
 };
+
+// Tile table of the small-M GEMMs: tiles32[a] = 32-row tiles of the active
+// experts before slot a, tiles32[num_active] = all of them.  One warp.
+__device__ void small_tile_table(const GatherArgs& g, int lane) {
+  const int na = *g.num_active;
+  const int per = (na + 31) >> 5;
+  const int b = min(na, lane * per), e_end = min(na, b + per);
+  int sum = 0;
+  for (int a = b; a < e_end; ++a) {
+    const int e = g.expert_ids[a];
+    sum += (g.starts[e + 1] - g.starts[e] + 31) >> 5;
+  }
+  int incl = sum;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int x = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+    if (lane >= off) incl += x;
+  }
+  int run = incl - sum;
+  for (int a = b; a < e_end; ++a) {
+    g.tiles32[a] = run;
+    const int e = g.expert_ids[a];
+    run += (g.starts[e + 1] - g.starts[e] + 31) >> 5;
+  }
+  if (lane == 31) g.tiles32[na] = incl;
+}
 
 // Token and padded scale row of routed row r.
 __device__ __forceinline__ void gather_locate(const GatherArgs& g, int64_t r, int64_t& t, int& pr) {
@@ -506,6 +536,7 @@ __device__ __forceinline__ void gather_rows(const GatherArgs& g, int64_t warp_id
 __global__ void __launch_bounds__(256) gather_kernel(GatherArgs g) {
   pdl_trigger();
   pdl_wait();
+  if (g.tiles32 && blockIdx.x == 0 && threadIdx.x < 32) small_tile_table(g, threadIdx.x);
   const int64_t nw = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   gather_rows<1>(g, (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5, nw, threadIdx.x & 31);
 }

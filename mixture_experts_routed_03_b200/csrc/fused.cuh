@@ -1,7 +1,9 @@
 // fused.cuh -- the whole routed-MoE layer in one launch.
 //
 // A cooperative, persistent kernel (one CTA per SM, all resident) runs the
-// steps of the layer as phases separated by grid-wide barriers:
+// steps of the layer as phases separated by grid-wide barriers (the GEMM
+// phases use the large-M tiles, or with SWAP the small-M swapped-operand
+// tiles):
 //
 //   route (when routing from logits)  ->  permute (one block, or two passes
 //   over 1024-slot chunks)  ->  gather into expert order  ->  gate_up GEMM
@@ -21,6 +23,7 @@
 
 #include "aux_kernels.cuh"
 #include "gemm.cuh"
+#include "gemm_swap.cuh"
 
 namespace moe {
 
@@ -93,12 +96,32 @@ __device__ __forceinline__ void stamp(const FusedArgs& f, int i) {
   if (blockIdx.x == 0 && threadIdx.x == 0) f.phase_ns[i] = globaltimer_ns();
 }
 
+// Block shape of the single launch: that of its GEMM phases (large-M tiles,
+// or the swapped-operand small-M tiles).
+template <int FMT, bool SWAP>
+struct FusedShape {
+  static constexpr int kThreads = GemmCfg<FMT, EPI_L1>::kThreads;
+  static constexpr int kHeaderBytes = GemmCfg<FMT, EPI_L1>::kHeaderBytes;
+  static constexpr int kSmemBytes = GemmCfg<FMT, EPI_L1>::kSmemBytes > GemmCfg<FMT, EPI_L2_ACC>::kSmemBytes
+                                        ? GemmCfg<FMT, EPI_L1>::kSmemBytes
+                                        : GemmCfg<FMT, EPI_L2_ACC>::kSmemBytes;
+  static_assert(GemmCfg<FMT, EPI_L1>::kThreads == GemmCfg<FMT, EPI_L2_ACC>::kThreads, "one block shape");
+};
 template <int FMT>
-__global__ void __launch_bounds__(GemmCfg<FMT, EPI_L1>::kThreads, 1)
+struct FusedShape<FMT, true> {
+  static constexpr int kThreads = SwapCfg<FMT, EPI_L1>::kThreads;
+  static constexpr int kHeaderBytes = SwapCfg<FMT, EPI_L1>::kHeaderBytes;
+  static constexpr int kSmemBytes = SwapCfg<FMT, EPI_L1>::kSmemBytes > SwapCfg<FMT, EPI_L2_ACC>::kSmemBytes
+                                        ? SwapCfg<FMT, EPI_L1>::kSmemBytes
+                                        : SwapCfg<FMT, EPI_L2_ACC>::kSmemBytes;
+  static_assert(SwapCfg<FMT, EPI_L1>::kThreads == SwapCfg<FMT, EPI_L2_ACC>::kThreads, "one block shape");
+};
+
+template <int FMT, bool SWAP>
+__global__ void __launch_bounds__(FusedShape<FMT, SWAP>::kThreads, 1)
     moe_fused_kernel(const __grid_constant__ FusedArgs f, const __grid_constant__ CUtensorMap tmA1,
                      const __grid_constant__ CUtensorMap tmA2) {
-  static_assert(GemmCfg<FMT, EPI_L1>::kThreads == GemmCfg<FMT, EPI_L2_ACC>::kThreads, "one block shape");
-  constexpr int kHdr = GemmCfg<FMT, EPI_L1>::kHeaderBytes;
+  constexpr int kHdr = FusedShape<FMT, SWAP>::kHeaderBytes;
   SmemHeader* hdr = reinterpret_cast<SmemHeader*>(smem_base_1024());
   if (threadIdx.x == 0) hdr->abort = 0;
   if ((threadIdx.x >> 5) == 1) tmem_alloc(&hdr->tmem, kTmemCols);
@@ -128,13 +151,18 @@ __global__ void __launch_bounds__(GemmCfg<FMT, EPI_L1>::kThreads, 1)
   if (ok) ok = grid_barrier(f.gbar, &hdr->abort, f.status);
   stamp(f, 2);
   if (ok) {
+    if (f.gather.tiles32 && blockIdx.x == 0 && threadIdx.x < 32) small_tile_table(f.gather, threadIdx.x);
     const GridIdx g = grid_idx();
     gather_rows<2>(f.gather, g.gw, g.tw, g.lane);
     ok = grid_barrier(f.gbar, &hdr->abort, f.status);
   }
   stamp(f, 3);
   if (ok) {
-    gemm_phase<FMT, EPI_L1>(f.l1, &tmA1, smem_base_1024() + kHdr, hdr->tmem, &hdr->abort, blockIdx.x, gridDim.x);
+    if constexpr (SWAP)
+      gemm_phase_swap<FMT, EPI_L1>(f.l1, &tmA1, smem_base_1024() + kHdr, hdr->tmem, &hdr->abort, blockIdx.x,
+                                   gridDim.x);
+    else
+      gemm_phase<FMT, EPI_L1>(f.l1, &tmA1, smem_base_1024() + kHdr, hdr->tmem, &hdr->abort, blockIdx.x, gridDim.x);
     // the accumulator is zeroed last, just before the down GEMM adds into it
     const GridIdx g = grid_idx();
     zero_range(f.acc, f.acc_n4, g.gt, g.tt);
@@ -142,8 +170,12 @@ __global__ void __launch_bounds__(GemmCfg<FMT, EPI_L1>::kThreads, 1)
   }
   stamp(f, 4);
   if (ok) {
-    gemm_phase<FMT, EPI_L2_ACC>(f.l2, &tmA2, smem_base_1024() + kHdr, hdr->tmem, &hdr->abort, blockIdx.x,
-                                gridDim.x);
+    if constexpr (SWAP)
+      gemm_phase_swap<FMT, EPI_L2_ACC>(f.l2, &tmA2, smem_base_1024() + kHdr, hdr->tmem, &hdr->abort, blockIdx.x,
+                                       gridDim.x);
+    else
+      gemm_phase<FMT, EPI_L2_ACC>(f.l2, &tmA2, smem_base_1024() + kHdr, hdr->tmem, &hdr->abort, blockIdx.x,
+                                  gridDim.x);
     ok = grid_barrier(f.gbar, &hdr->abort, f.status);
   }
   stamp(f, 5);
@@ -159,11 +191,9 @@ __global__ void __launch_bounds__(GemmCfg<FMT, EPI_L1>::kThreads, 1)
   if ((threadIdx.x >> 5) == 1) tmem_dealloc(hdr->tmem, kTmemCols);
 }
 
-template <int FMT>
+template <int FMT, bool SWAP>
 __host__ __device__ constexpr int fused_smem_bytes() {
-  return GemmCfg<FMT, EPI_L1>::kSmemBytes > GemmCfg<FMT, EPI_L2_ACC>::kSmemBytes
-             ? GemmCfg<FMT, EPI_L1>::kSmemBytes
-             : GemmCfg<FMT, EPI_L2_ACC>::kSmemBytes;
+  return FusedShape<FMT, SWAP>::kSmemBytes;
 }
 
 }  // namespace moe

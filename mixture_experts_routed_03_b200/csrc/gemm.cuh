@@ -127,7 +127,8 @@ struct GemmArgs {
   const int* num_active;
   const int* starts;            // expert_start_indices
   const int* a_scale_offsets;
-  const int* tile_offsets;
+  const int* tile_offsets;       // tile table: m tiles of tile_rows rows per active expert, prefix summed
+  int tile_rows;                 // 128 (kBM), or kNT for the swapped-operand GEMM
   const int* src_info;
   const float* topk_weights;
   // prepared weights: [E][n_tiles][k_stages] blocks of b_block_bytes(FMT)
@@ -200,9 +201,9 @@ __device__ __forceinline__ void tile_finish(const GemmArgs& p, int lo, int g, in
   t.e = __ldg(p.expert_ids + lo);
   const int start = __ldg(p.starts + t.e);
   const int cnt = __ldg(p.starts + t.e + 1) - start;
-  t.row0 = start + mt * kBM;
-  t.rows = min(kBM, cnt - mt * kBM);
-  t.srow0 = __ldg(p.a_scale_offsets + t.e) + mt * kBM;
+  t.row0 = start + mt * p.tile_rows;
+  t.rows = min(p.tile_rows, cnt - mt * p.tile_rows);
+  t.srow0 = __ldg(p.a_scale_offsets + t.e) + mt * p.tile_rows;
 }
 
 // Tile T -> (expert, m tile, n tile) by one thread: binary search over the

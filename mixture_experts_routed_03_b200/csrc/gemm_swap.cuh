@@ -1,0 +1,359 @@
+// gemm_swap.cuh -- the grouped GEMMs for small per-expert batches, with the
+// operands swapped (BF16 and FP8).
+//
+// When an expert receives only a few routed rows (decode, or many experts
+// per token), a 128-row tile of routed rows is mostly padding and the tensor
+// core time per K block, not the weight stream, sets the pace.  Here the
+// weights are the MMA's M side and the routed rows its N side: a tile is
+// (active expert, 256 weight rows = the same prepared block as the large-M
+// GEMM, kNT = 32 routed rows), issued as two M128 x N32 MMAs per K step
+// (weight rows 0-127 and 128-255), so the tensor work follows the rows that
+// exist.  The accumulators are 128 TMEM lanes (weight rows) x 32 columns
+// (routed rows); per-K-block FP8 partials take 64 columns, so eight of them
+// are in flight.
+//
+// Roles as in the large-M GEMM: warp 0 lane 0 loads the stage (TMA of the
+// 32 routed rows, one bulk copy of the prepared weight block), warp 1 lane 0
+// issues the MMAs, warps 2..9 are the epilogue: warp (q, half) reads lanes
+// 32q..32q+31 of the accumulator of weight rows 128*half.., one weight row
+// per thread and 32 routed rows in its registers.
+//
+// Gate_up epilogue: every thread stages its promoted FP32 row in shared
+// memory; after a barrier of the eight warps each warp takes four routed
+// rows, one lane per four intermediate columns, forms the clamped SwiGLU from
+// the staged gate and up rows, re-quantises (BF16, or FP8 with one scale per
+// routed row and 128 columns) and writes the row segment whole.
+// Down epilogue: a thread holds one output column for 32 routed rows and adds
+// them, router-weighted, into the FP32 accumulator rows of their tokens
+// (a warp's 32 lanes cover 128 contiguous bytes of one row), or stores them
+// in staged mode.
+#pragma once
+
+#include "gemm.cuh"
+
+namespace moe {
+
+constexpr int kNT = 32;                 // routed rows per tile (the MMA's N)
+constexpr int kTStage = kNT * kBK;      // 4 KB of routed rows per stage
+
+template <int FMT, int EPI>
+struct SwapCfg {
+  static_assert(FMT != FMT_NVFP4, "the swapped-operand GEMM covers BF16 and FP8");
+  static constexpr int kStages = (EPI == EPI_L1) ? 5 : 6;
+  static constexpr int kStageBytes = kTStage + kBStage;    // 36 KB
+  static constexpr int kAccCols = 2 * kNT;                  // weight-row halves 0 | 1
+  static constexpr int kAccBufs = (FMT == FMT_FP8) ? 8 : 4;
+  static_assert(kAccBufs * kAccCols <= kTmemCols, "TMEM");
+  static constexpr int kFirstEpiWarp = 2;
+  static constexpr int kThreads = (kFirstEpiWarp + kEpiWarps) * 32;
+  static constexpr int kBarrierBytes = 4096;
+  static constexpr int kSStride = kNT + 1;                   // floats per staged weight row
+  static constexpr int kSBytes = (EPI == EPI_L1) ? kBN * kSStride * 4 : 0;
+  static constexpr int kHeaderBytes = 1024;
+  static constexpr int kPhaseBytes = kStages * kStageBytes + kBarrierBytes + kSBytes;
+  static constexpr int kSmemBytes = 1024 /*align*/ + kHeaderBytes + kPhaseBytes;
+};
+
+template <int FMT, int EPI>
+__device__ __forceinline__ void gemm_phase_swap(const GemmArgs& p, const CUtensorMap* tmA, uint8_t* smem,
+                                                uint32_t tmem, volatile int* abort_flag, int cta, int ncta) {
+  using Cfg = SwapCfg<FMT, EPI>;
+  constexpr int S = Cfg::kStages;
+  constexpr int NACC = Cfg::kAccBufs;
+  constexpr int SB = Cfg::kStageBytes;
+  constexpr int BB = b_block_bytes(FMT);
+
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * SB);
+  uint64_t* empty = full + S;
+  uint64_t* acc_full = empty + S;
+  uint64_t* acc_empty = acc_full + NACC;
+  uint64_t* final_bar = acc_empty + NACC;
+  uint64_t* sbar = final_bar + 1;    // L1: [0] rows staged, [1] staged rows consumed
+  float* stage_rows = reinterpret_cast<float*>(smem + S * SB + Cfg::kBarrierBytes);  // L1: [256][kSStride]
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < NACC; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], kEpiWarps);
+    }
+    mbar_init(final_bar, 1);
+    mbar_init(&sbar[0], kEpiWarps * 32);
+    mbar_init(&sbar[1], kEpiWarps * 32);
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) prefetch_tensormap(tmA);
+  __syncthreads();
+
+  const int na = *p.num_active;
+  const int total = (na > 0) ? __ldg(p.tile_offsets + na) * p.n_tiles : 0;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      for (int T = cta; T < total; T += ncta) {
+        TileInfo t;
+        decode_tile(p, na, T, t);
+        const uint8_t* wb =
+            p.wB + (static_cast<size_t>(t.e) * p.n_tiles + t.n_tile) * p.k_stages * BB;
+        for (int ks = 0; ks < p.k_stages; ++ks) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status, 21)) goto producer_done;
+          uint8_t* st = smem + stage * SB;
+          mbar_arrive_expect_tx(&full[stage], SB);
+          tma_load_2d(st, tmA, &full[stage], ks * kBK, t.row0);
+          bulk_load(st + kTStage, wb + static_cast<size_t>(ks) * BB, BB, &full[stage]);
+          ++issued;
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    producer_done:
+      if (*abort_flag) {
+        int st = stage;
+        uint32_t ph = phase;
+        for (int i = 0; i < S && i < issued; ++i) {
+          if (--st < 0) {
+            st = S - 1;
+            ph ^= 1u;
+          }
+          mbar_drain(&full[st], ph);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdesc = (FMT == FMT_BF16) ? idesc_dense(1, 1, kNT) : idesc_dense(0, 0, kNT);
+      int stage = 0;
+      uint32_t phase = 0;
+      int ab = 0;
+      uint32_t aphase = 0;
+      bool ok = true;
+      for (int T = cta; T < total && ok; T += ncta) {
+        if (FMT != FMT_FP8) {
+          if (!mbar_wait(&acc_empty[ab], aphase ^ 1u, abort_flag, p.status, 22)) break;
+          tc_fence_after();
+        }
+        for (int ks = 0; ks < p.k_stages; ++ks) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, p.status, 23)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (FMT == FMT_FP8) {
+            if (!mbar_wait(&acc_empty[ab], aphase ^ 1u, abort_flag, p.status, 24)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+          }
+          const uint32_t d0 = tmem + ab * Cfg::kAccCols;
+          uint8_t* st = smem + stage * SB;
+          const uint64_t bdesc = sdesc_sw128(smem_u32(st));                       // routed rows
+          const uint64_t a0 = sdesc_sw128(smem_u32(st + kTStage));                // weight rows 0..127
+          const uint64_t a1 = sdesc_sw128(smem_u32(st + kTStage + kBStage / 2));  // weight rows 128..255
+#pragma unroll
+          for (int kc = 0; kc < 4; ++kc) {
+            const uint32_t acc = (FMT == FMT_FP8) ? (kc > 0) : ((ks | kc) != 0);
+            const uint64_t b = bdesc + static_cast<uint64_t>(2 * kc);
+            if (FMT == FMT_BF16) {
+              mma_f16(d0, a0 + static_cast<uint64_t>(2 * kc), b, kIdesc, acc);
+              mma_f16(d0 + kNT, a1 + static_cast<uint64_t>(2 * kc), b, kIdesc, acc);
+            } else {
+              mma_f8(d0, a0 + static_cast<uint64_t>(2 * kc), b, kIdesc, acc);
+              mma_f8(d0 + kNT, a1 + static_cast<uint64_t>(2 * kc), b, kIdesc, acc);
+            }
+          }
+          mma_commit(&empty[stage]);
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+          if (FMT == FMT_FP8) {
+            mma_commit(&acc_full[ab]);
+            if (++ab == NACC) {
+              ab = 0;
+              aphase ^= 1u;
+            }
+          }
+        }
+        if (FMT != FMT_FP8 && ok) {
+          mma_commit(&acc_full[ab]);
+          if (++ab == NACC) {
+            ab = 0;
+            aphase ^= 1u;
+          }
+        }
+      }
+      mma_commit(final_bar);
+      mbar_drain(final_bar, 0);
+    }
+  } else if (warp >= Cfg::kFirstEpiWarp) {
+    // ------------------------------------------------------------ epilogue
+    const int ew = warp - Cfg::kFirstEpiWarp;
+    const int q = warp & 3;                        // TMEM lane quarter this warp may access
+    const int half = ew >> 2;                      // weight rows 128*half ..
+    const int wr = half * 128 + q * 32 + lane;     // this thread's weight row of the tile
+    const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    int ab = 0;
+    uint32_t aphase = 0;
+    uint32_t spar = 0;
+    for (int T = cta; T < total; T += ncta) {
+      TileInfo t;
+      decode_tile_warp(p, na, T, t, lane);
+      const bool lane_row = lane < t.rows;         // routed row `lane` of the tile exists
+      // down leg: this lane's routed row -> token and router weight
+      const bool gather_wgt = EPI == EPI_L2_ACC && lane_row;
+      const int s_flat = gather_wgt ? __ldg(p.src_info + t.row0 + lane) : 0;
+      float wgt = 1.0f;
+
+      float acc[kNT];
+      if constexpr (FMT == FMT_FP8) {
+#pragma unroll
+        for (int i = 0; i < kNT; ++i) acc[i] = 0.0f;
+        // the weight block of this warp's rows (warp-uniform)
+        const int wrow = (EPI == EPI_L1) ? l1_tile_row(t.n_tile, wr, p.I) : (t.n_tile * kBN + wr);
+        const float* sbe = p.sb + (static_cast<size_t>(t.e) * p.sb_nb + (wrow >> 7)) * p.sb_kb;
+        // lane i holds routed row i's activation scale of the next K block
+        const float* sa_col = p.sa_t + t.srow0 + lane;
+        float nx_sa = sa_col[0];
+        bool ok = true;
+        for (int ks = 0; ks < p.k_stages; ++ks) {
+          const float sa = nx_sa;
+          if (ks + 1 < p.k_stages) nx_sa = sa_col[static_cast<size_t>(ks + 1) * p.sa_ld];
+          if (!mbar_wait(&acc_full[ab], aphase, abort_flag, p.status, 25)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const float sbk = __ldg(sbe + ks);
+          float v[kNT];
+          __syncwarp();
+          tmem_ld32(tmem + ab * Cfg::kAccCols + half * kNT + lane_off, v);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[ab]);
+          if (++ab == NACC) {
+            ab = 0;
+            aphase ^= 1u;
+          }
+          if (ks == 0 && gather_wgt) wgt = __ldg(p.topk_weights + s_flat);
+#pragma unroll
+          for (int i = 0; i < kNT; ++i) acc[i] = fmaf(v[i], __shfl_sync(0xFFFFFFFFu, sa, i) * sbk, acc[i]);
+        }
+        if (!ok) break;
+      } else {
+        if (!mbar_wait(&acc_full[ab], aphase, abort_flag, p.status, 26)) break;
+        tc_fence_after();
+        __syncwarp();
+        tmem_ld32(tmem + ab * Cfg::kAccCols + half * kNT + lane_off, acc);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[ab]);
+        if (++ab == NACC) {
+          ab = 0;
+          aphase ^= 1u;
+        }
+        if (gather_wgt) wgt = __ldg(p.topk_weights + s_flat);
+      }
+
+      if constexpr (EPI == EPI_L1) {
+        // stage this weight row's 32 values, then each warp finishes 4 routed rows
+#pragma unroll
+        for (int i = 0; i < kNT; ++i) stage_rows[wr * Cfg::kSStride + i] = acc[i];
+        mbar_arrive(&sbar[0]);
+        if (!mbar_wait(&sbar[0], spar, abort_flag, p.status, 27)) break;
+        const int c0 = 4 * lane;                        // intermediate columns c0..c0+3 of the tile
+        const int gate_row0 = (c0 < 64) ? c0 : 64 + c0; // weight rows of gate (c) and up (c + 64)
+        for (int j = 0; j < 4; ++j) {
+          const int tr = ew * 4 + j;                    // routed row of the tile (warp-uniform)
+          float h[4];
+          if (p.fast_math) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              h[i] = clamped_swiglu<true>(stage_rows[(gate_row0 + i) * Cfg::kSStride + tr],
+                                          stage_rows[(gate_row0 + 64 + i) * Cfg::kSStride + tr], p.clamp);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              h[i] = clamped_swiglu<false>(stage_rows[(gate_row0 + i) * Cfg::kSStride + tr],
+                                           stage_rows[(gate_row0 + 64 + i) * Cfg::kSStride + tr], p.clamp);
+          }
+          const bool row_ok = tr < t.rows;
+          uint8_t* hrow = p.h_out + static_cast<size_t>(t.row0 + tr) * p.h_row_bytes;
+          if constexpr (FMT == FMT_FP8) {
+            float amax = fmaxf(fmaxf(fabsf(h[0]), fabsf(h[1])), fmaxf(fabsf(h[2]), fabsf(h[3])));
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+            const float s = __fdiv_rn(amax, 448.0f);
+            const float inv = (s != 0.0f) ? __frcp_rn(s) : 0.0f;
+            const uint32_t lo = cvt_e4m3x2(__fmul_rn(h[0], inv), __fmul_rn(h[1], inv));
+            const uint32_t hi = cvt_e4m3x2(__fmul_rn(h[2], inv), __fmul_rn(h[3], inv));
+            if (row_ok) {
+              *reinterpret_cast<uint32_t*>(hrow + t.n_tile * 128 + c0) = (s != 0.0f) ? (lo | (hi << 16)) : 0u;
+              if (lane == 0) p.h_scale_t[static_cast<size_t>(t.n_tile) * p.h_scale_ld + t.srow0 + tr] = s;
+            }
+          } else {
+            if (row_ok)
+              *reinterpret_cast<uint2*>(hrow + (t.n_tile * 128 + c0) * 2) =
+                  make_uint2(pack_bf16x2(h[0], h[1]), pack_bf16x2(h[2], h[3]));
+          }
+        }
+        // the staging rows may be overwritten once all eight warps are done
+        mbar_arrive(&sbar[1]);
+        if (!mbar_wait(&sbar[1], spar, abort_flag, p.status, 28)) break;
+        spar ^= 1u;
+      } else {
+        // down leg: output column n of the tile for each routed row
+        const int n = t.n_tile * kBN + wr;
+        const int tok_l = gather_wgt ? s_flat / p.topk : 0;
+#pragma unroll
+        for (int i = 0; i < kNT; ++i) {
+          if (i >= t.rows) break;   // warp-uniform
+          if (EPI == EPI_L2_ACC) {
+            const int tok = __shfl_sync(0xFFFFFFFFu, tok_l, i);
+            const float w = __shfl_sync(0xFFFFFFFFu, wgt, i);
+            atomicAdd(p.out + static_cast<size_t>(tok) * p.H + n, acc[i] * w);
+          } else {
+            p.out[static_cast<size_t>(t.row0 + i) * p.H + n] = acc[i];
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+}
+
+template <int FMT, int EPI>
+__global__ void __launch_bounds__(SwapCfg<FMT, EPI>::kThreads, 1)
+    moe_gemm_swap_kernel(const __grid_constant__ GemmArgs p, const __grid_constant__ CUtensorMap tmA) {
+  uint8_t* base = smem_base_1024();
+  SmemHeader* hdr = reinterpret_cast<SmemHeader*>(base);
+  if (threadIdx.x == 0) hdr->abort = 0;
+  if ((threadIdx.x >> 5) == 1) tmem_alloc(&hdr->tmem, kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = hdr->tmem;
+  pdl_trigger();
+  pdl_wait();   // the layout, tile table, activations and accumulator come from earlier kernels
+  gemm_phase_swap<FMT, EPI>(p, &tmA, base + SwapCfg<FMT, EPI>::kHeaderBytes, tmem, &hdr->abort, blockIdx.x,
+                            gridDim.x);
+  if ((threadIdx.x >> 5) == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
+}  // namespace moe

@@ -13,6 +13,7 @@
 #include "aux_kernels.cuh"
 #include "fused.cuh"
 #include "gemm.cuh"
+#include "gemm_swap.cuh"
 
 using namespace moe;
 
@@ -35,6 +36,8 @@ moe_status_t check_problem(const moe_problem_t* p) {
   if (p->num_experts < 1 || p->num_topk < 1 || p->num_topk > p->num_experts) return MOE_ERR_INVALID_ARG;
   if (p->num_experts > 1024) return MOE_ERR_UNSUPPORTED;
   if (std::isnan(p->activation_clamp) || !(p->activation_clamp > 0.0f)) return MOE_ERR_INVALID_ARG;
+  if (p->tile_regime < MOE_TILE_AUTO || p->tile_regime > MOE_TILE_SMALL_M) return MOE_ERR_INVALID_ARG;
+  if (p->tile_regime == MOE_TILE_SMALL_M && p->format == MOE_FMT_NVFP4) return MOE_ERR_UNSUPPORTED;
   if (p->format == MOE_FMT_NVFP4 && p->intermediate_hidden % 256 != 0) return MOE_ERR_UNSUPPORTED;
   const int64_t R = p->num_tokens * p->num_topk;
   if (R > (int64_t(1) << 30)) return MOE_ERR_UNSUPPORTED;
@@ -51,7 +54,7 @@ struct WsLayout {
   int nblk;          // permute chunks
   size_t header, route_idx, route_w;
   size_t counts, starts, src_info, slot_to_row, expert_ids, num_active, a_scale_offsets, tile_offsets;
-  size_t block_counts;
+  size_t block_counts, tiles32;
   size_t x_perm, x_sf;
   size_t h, h_sf;
   size_t acc;
@@ -84,6 +87,7 @@ WsLayout make_layout(const moe_problem_t* p) {
   L.a_scale_offsets = take(size_t(E + 1) * 4);
   L.tile_offsets = take(size_t(E + 1) * 4);
   L.block_counts = take(size_t(L.nblk) * E * 4);
+  L.tiles32 = take(size_t(E + 1) * 4);
   L.x_perm = take(size_t(L.R) * x_row_bytes(fmt, H));
   L.x_sf = take(fmt == FMT_FP8 ? size_t(H / 128) * L.P * 4 : (fmt == FMT_NVFP4 ? size_t(L.P) * (H / 16) : 0));
   L.h_bytes = size_t(L.R) * h_row_bytes(fmt, I);
@@ -193,6 +197,22 @@ cudaError_t set_gemm_attr() {
                               GemmCfg<FMT, EPI>::kSmemBytes);
 }
 
+template <int FMT, int EPI>
+cudaError_t set_swap_attr() {
+  return cudaFuncSetAttribute(moe_gemm_swap_kernel<FMT, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              SwapCfg<FMT, EPI>::kSmemBytes);
+}
+
+template <int FMT>
+cudaError_t set_swap_attrs_fmt() {
+  cudaError_t e;
+  if ((e = set_swap_attr<FMT, EPI_L1>()) != cudaSuccess) return e;
+  if ((e = set_swap_attr<FMT, EPI_L2_ACC>()) != cudaSuccess) return e;
+  if ((e = set_swap_attr<FMT, EPI_L2_STAGED>()) != cudaSuccess) return e;
+  return cudaFuncSetAttribute(moe_fused_kernel<FMT, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              fused_smem_bytes<FMT, true>());
+}
+
 template <int FMT>
 cudaError_t set_attrs_fmt() {
   cudaError_t e;
@@ -203,8 +223,8 @@ cudaError_t set_attrs_fmt() {
 
 template <int FMT>
 cudaError_t set_fused_attr() {
-  return cudaFuncSetAttribute(moe_fused_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              fused_smem_bytes<FMT>());
+  return cudaFuncSetAttribute(moe_fused_kernel<FMT, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              fused_smem_bytes<FMT, false>());
 }
 
 cudaError_t set_all_attrs() {
@@ -214,7 +234,9 @@ cudaError_t set_all_attrs() {
   if ((e = set_fused_attr<FMT_NVFP4>()) != cudaSuccess) return e;
   if ((e = set_attrs_fmt<FMT_BF16>()) != cudaSuccess) return e;
   if ((e = set_attrs_fmt<FMT_FP8>()) != cudaSuccess) return e;
-  return set_attrs_fmt<FMT_NVFP4>();
+  if ((e = set_attrs_fmt<FMT_NVFP4>()) != cudaSuccess) return e;
+  if ((e = set_swap_attrs_fmt<FMT_BF16>()) != cudaSuccess) return e;
+  return set_swap_attrs_fmt<FMT_FP8>();
 }
 
 bool ensure_init() {
@@ -233,8 +255,17 @@ cudaError_t launch_gemm(const GemmArgs& a, const CUtensorMap& ta, int grid, cuda
                   st, a, ta);
 }
 
+template <int FMT, int EPI>
+cudaError_t launch_swap(const GemmArgs& a, const CUtensorMap& ta, int grid, cudaStream_t st) {
+  return launch_k(moe_gemm_swap_kernel<FMT, EPI>, grid, SwapCfg<FMT, EPI>::kThreads,
+                  SwapCfg<FMT, EPI>::kSmemBytes, st, a, ta);
+}
+
 template <int EPI>
-cudaError_t launch_gemm_fmt(int fmt, const GemmArgs& a, const CUtensorMap& ta, int grid, cudaStream_t st) {
+cudaError_t launch_gemm_fmt(int fmt, bool swap, const GemmArgs& a, const CUtensorMap& ta, int grid,
+                            cudaStream_t st) {
+  if (swap) return fmt == FMT_BF16 ? launch_swap<FMT_BF16, EPI>(a, ta, grid, st)
+                                   : launch_swap<FMT_FP8, EPI>(a, ta, grid, st);
   switch (fmt) {
     case FMT_BF16: return launch_gemm<FMT_BF16, EPI>(a, ta, grid, st);
     case FMT_FP8: return launch_gemm<FMT_FP8, EPI>(a, ta, grid, st);
@@ -302,6 +333,7 @@ struct FfnBuffers {
   const int *counts, *starts, *src_info, *slot_to_row, *expert_ids, *num_active, *a_scale_offsets, *tile_offsets;
   // scratch
   uint8_t *x_perm, *x_sf, *h, *h_sf;
+  int* tiles32;     // small-M tile table (workspace)
   int64_t P;
   int* status;
 };
@@ -312,13 +344,23 @@ struct FfnPlan {
   GemmArgs l1, l2;
   CUtensorMap ta1, ta2;
   int grid1, grid2;
+  bool swap;        // small-M (swapped-operand) GEMMs
 };
+
+// The GEMMs' tile regime for this problem (MOE_TILE_AUTO resolved).
+bool small_m_tiles(const moe_problem_t* p) {
+  if (p->tile_regime == MOE_TILE_SMALL_M) return true;
+  if (p->tile_regime == MOE_TILE_LARGE_M || p->format == FMT_NVFP4) return false;
+  return p->num_tokens * p->num_topk <= int64_t(64) * p->num_experts;
+}
 
 moe_status_t plan_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_weights_t* w, const FfnBuffers& b,
                       const float* topk_weights, float* out, FfnPlan& pl) {
   const int fmt = p->format, H = p->hidden, I = p->intermediate_hidden, E = p->num_experts, k = p->num_topk;
   const int64_t M = p->num_tokens, R = M * k;
   const int nsm = sm_count();
+  pl.swap = small_m_tiles(p);
+  const int tile_rows = pl.swap ? kNT : kBM;
 
   GatherArgs& g = pl.g;
   g = GatherArgs{};
@@ -337,9 +379,12 @@ moe_status_t plan_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_we
   g.sa_t = reinterpret_cast<float*>(b.x_sf);
   g.sfa = b.x_sf;
   g.ld = int(b.P);
+  g.expert_ids = b.expert_ids;
+  g.num_active = b.num_active;
+  g.tiles32 = pl.swap ? b.tiles32 : nullptr;
 
   // L1: gate_up
-  if (!make_map(&pl.ta1, b.x_perm, x_row_bytes(fmt, H), uint64_t(R), 128)) return MOE_ERR_CUDA;
+  if (!make_map(&pl.ta1, b.x_perm, x_row_bytes(fmt, H), uint64_t(R), uint32_t(tile_rows))) return MOE_ERR_CUDA;
   GemmArgs& a = pl.l1;
   a = GemmArgs{};
   a.k_stages = x_row_bytes(fmt, H) / 128;
@@ -355,7 +400,8 @@ moe_status_t plan_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_we
   a.num_active = b.num_active;
   a.starts = b.starts;
   a.a_scale_offsets = b.a_scale_offsets;
-  a.tile_offsets = b.tile_offsets;
+  a.tile_offsets = pl.swap ? b.tiles32 : b.tile_offsets;
+  a.tile_rows = tile_rows;
   a.src_info = b.src_info;
   a.topk_weights = topk_weights;
   a.sfa = b.x_sf;
@@ -374,11 +420,11 @@ moe_status_t plan_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_we
   a.h_scale_t = reinterpret_cast<float*>(b.h_sf);
   a.h_scale_ld = int(b.P);
   a.status = b.status;
-  const int64_t mtiles_bound = (R + 127) / 128 + std::min<int64_t>(E, R);
+  const int64_t mtiles_bound = (R + tile_rows - 1) / tile_rows + std::min<int64_t>(E, R);
   pl.grid1 = std::max(1, int(std::min<int64_t>(nsm, mtiles_bound * a.n_tiles)));
 
   // L2: down
-  if (!make_map(&pl.ta2, b.h, h_row_bytes(fmt, I), uint64_t(R), 128)) return MOE_ERR_CUDA;
+  if (!make_map(&pl.ta2, b.h, h_row_bytes(fmt, I), uint64_t(R), uint32_t(tile_rows))) return MOE_ERR_CUDA;
   GemmArgs& a2 = pl.l2;
   a2 = a;
   a2.k_stages = h_row_bytes(fmt, I) / 128;
@@ -420,7 +466,7 @@ moe_status_t run_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_wei
   }
   {
     TimScope ts(MOE_SLOT_GEMM1, st);
-    if (launch_gemm_fmt<EPI_L1>(fmt, pl.l1, pl.ta1, pl.grid1, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_gemm_fmt<EPI_L1>(fmt, pl.swap, pl.l1, pl.ta1, pl.grid1, st) != cudaSuccess) return MOE_ERR_CUDA;
   }
   if (out_mode == MOE_OUT_ACCUMULATE) {
     TimScope ts(MOE_SLOT_ZERO, st);
@@ -430,25 +476,25 @@ moe_status_t run_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_wei
   }
   TimScope ts2(MOE_SLOT_GEMM2, st);
   cudaError_t e = (out_mode == MOE_OUT_ACCUMULATE)
-                      ? launch_gemm_fmt<EPI_L2_ACC>(fmt, pl.l2, pl.ta2, pl.grid2, st)
-                      : launch_gemm_fmt<EPI_L2_STAGED>(fmt, pl.l2, pl.ta2, pl.grid2, st);
+                      ? launch_gemm_fmt<EPI_L2_ACC>(fmt, pl.swap, pl.l2, pl.ta2, pl.grid2, st)
+                      : launch_gemm_fmt<EPI_L2_STAGED>(fmt, pl.swap, pl.l2, pl.ta2, pl.grid2, st);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 // The single-launch layer: a cooperative launch of moe_fused_kernel<FMT>.
-template <int FMT>
+template <int FMT, bool SWAP>
 cudaError_t launch_fused_fmt(const FusedArgs& f, const FfnPlan& pl, int grid, cudaStream_t st) {
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
-  cfg.blockDim = dim3(GemmCfg<FMT, EPI_L1>::kThreads);
-  cfg.dynamicSmemBytes = fused_smem_bytes<FMT>();
+  cfg.blockDim = dim3(FusedShape<FMT, SWAP>::kThreads);
+  cfg.dynamicSmemBytes = fused_smem_bytes<FMT, SWAP>();
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, moe_fused_kernel<FMT>, f, pl.ta1, pl.ta2);
+  return cudaLaunchKernelEx(&cfg, moe_fused_kernel<FMT, SWAP>, f, pl.ta1, pl.ta2);
 }
 
 bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; }
@@ -531,6 +577,14 @@ moe_status_t moe_get_workspace_size(const moe_problem_t* p, size_t* bytes) {
   if (s != MOE_OK) return s;
   if (!bytes) return MOE_ERR_INVALID_ARG;
   *bytes = make_layout(p).total;
+  return MOE_OK;
+}
+
+moe_status_t moe_get_tile_regime(const moe_problem_t* p, int32_t* regime) {
+  moe_status_t s = check_problem(p);
+  if (s != MOE_OK) return s;
+  if (!regime) return MOE_ERR_INVALID_ARG;
+  *regime = small_m_tiles(p) ? MOE_TILE_SMALL_M : MOE_TILE_LARGE_M;
   return MOE_OK;
 }
 
@@ -663,6 +717,7 @@ moe_status_t moe_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_wei
   moe_get_intermediate_size(p, &isz, &so);
   b.h = intermediate ? static_cast<uint8_t*>(intermediate) : base + L.h;
   b.h_sf = intermediate ? static_cast<uint8_t*>(intermediate) + so : base + L.h_sf;
+  b.tiles32 = reinterpret_cast<int*>(base + L.tiles32);
   b.P = L.P;
   b.status = reinterpret_cast<int*>(base + L.header);
   return run_ffn(p, act, w, b, topk_weights, out_mode, static_cast<float*>(out),
@@ -740,6 +795,7 @@ moe_status_t moe_fused(const moe_problem_t* p, const moe_act_t* act, const moe_w
   b.x_sf = base + L.x_sf;
   b.h = base + L.h;
   b.h_sf = base + L.h_sf;
+  b.tiles32 = reinterpret_cast<int*>(base + L.tiles32);
   b.P = L.P;
   b.status = status;
   float* acc = reinterpret_cast<float*>(base + L.acc);
@@ -761,9 +817,13 @@ moe_status_t moe_fused(const moe_problem_t* p, const moe_act_t* act, const moe_w
   TimScope ts(MOE_SLOT_FUSED, st);
   cudaError_t e;
   switch (p->format) {
-    case FMT_BF16: e = launch_fused_fmt<FMT_BF16>(f, pl, grid, st); break;
-    case FMT_FP8: e = launch_fused_fmt<FMT_FP8>(f, pl, grid, st); break;
-    default: e = launch_fused_fmt<FMT_NVFP4>(f, pl, grid, st); break;
+    case FMT_BF16:
+      e = pl.swap ? launch_fused_fmt<FMT_BF16, true>(f, pl, grid, st) : launch_fused_fmt<FMT_BF16, false>(f, pl, grid, st);
+      break;
+    case FMT_FP8:
+      e = pl.swap ? launch_fused_fmt<FMT_FP8, true>(f, pl, grid, st) : launch_fused_fmt<FMT_FP8, false>(f, pl, grid, st);
+      break;
+    default: e = launch_fused_fmt<FMT_NVFP4, false>(f, pl, grid, st); break;
   }
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

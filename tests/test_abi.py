@@ -55,6 +55,8 @@ def _prob(**kw):
     (dict(activation_clamp=0.0), api.MOE_ERR_INVALID_ARG),
     (dict(format=7), api.MOE_ERR_INVALID_ARG),
     (dict(format="nvfp4", intermediate_hidden=384), api.MOE_ERR_UNSUPPORTED),
+    (dict(tile_regime=3), api.MOE_ERR_INVALID_ARG),
+    (dict(format="nvfp4", tile_regime="small_m"), api.MOE_ERR_UNSUPPORTED),
 ])
 def test_geometry_validation(lib, kw, code):
     n = ctypes.c_size_t(0)
@@ -118,3 +120,14 @@ def test_zero_tokens_is_ok_without_touching_memory(lib):
 def test_status_strings(lib):
     for code in range(7):
         assert api.status_string(code).startswith("MOE_")
+
+
+def test_tile_regime_resolution(lib):
+    # AUTO: swapped-operand tiles while routed rows average <= 64 per expert (BF16 / FP8)
+    assert api.tile_regime(_prob(num_tokens=256, num_experts=8, num_topk=2)) == "small_m"     # 512 <= 512
+    assert api.tile_regime(_prob(num_tokens=257, num_experts=8, num_topk=2)) == "large_m"
+    assert api.tile_regime(_prob(num_tokens=256, format="fp8", num_experts=8, num_topk=2)) == "small_m"
+    assert api.tile_regime(_prob(num_tokens=16, format="nvfp4", intermediate_hidden=256, num_experts=8,
+                                 num_topk=2)) == "large_m"
+    assert api.tile_regime(_prob(num_tokens=16, tile_regime="large_m")) == "large_m"
+    assert api.tile_regime(_prob(num_tokens=100000, tile_regime="small_m")) == "small_m"

@@ -53,10 +53,36 @@ def test_ffn_parity_small(fmt, M, H, I, E, k):
     assert np.all(S.close_bf16(a, b, 1e-2 * S.rms(a)))
 
 
-@pytest.mark.parametrize("fmt", ["bf16", "fp8", "nvfp4"])
-def test_staged_mode_and_deterministic_combine(fmt):
+@pytest.mark.parametrize("regime", ["large_m", "small_m"])
+@pytest.mark.parametrize("fmt,M,H,I,E,k", [c for c in SMALL if c[0] != "nvfp4"])
+def test_ffn_parity_both_tile_regimes(fmt, M, H, I, E, k, regime):
+    """Both GEMM tile regimes (128 routed rows x 256 weight rows, and the
+    swapped operands with 32 routed rows) on every BF16 / FP8 case, through
+    the unfused chain and the single launch."""
+    p = _small(fmt, M, H, I, E, k)
+    p["tile_regime"] = regime
+    d, host = S.make(p, seed=3)
+    L = layer.MoELayer(p, _weights(d), device=S.device())
+    assert api.tile_regime(L.problem(M)) == regime
+    lay, acc, inter, out = S.run_unfused(L, d)
+    assert L.status() == api.MOE_OK
+    lay_h = lay.host()
+    S.check_layout_exact(lay_h, O.permute(host["topk_idx"], E), M, k)
+    stats = S.check_ffn_against_oracle(p, host, lay_h, acc, inter, out, np.arange(M), label=f"{fmt}/{regime}")
+    print(fmt, regime, stats)
+    out2 = L.forward(d["x"], d.get("x_scale"), topk_idx=d["topk_idx"], topk_weights=d["topk_weights"])
+    torch.cuda.synchronize()
+    assert L.status() == api.MOE_OK
+    a, b = S.bf16_to_np(out), S.bf16_to_np(out2)
+    assert np.all(S.close_bf16(a, b, 1e-2 * S.rms(a)))
+
+
+@pytest.mark.parametrize("fmt,regime", [("bf16", "large_m"), ("fp8", "large_m"), ("nvfp4", "large_m"),
+                                        ("bf16", "small_m"), ("fp8", "small_m")])
+def test_staged_mode_and_deterministic_combine(fmt, regime):
     M, H, I, E, k = 96, 512, 256, 4, 3
     p = _small(fmt, M, H, I, E, k)
+    p["tile_regime"] = regime
     d, host = S.make(p, seed=2)
     L = layer.MoELayer(p, _weights(d), device=S.device())
     lay = L.permute(d["topk_idx"])
