@@ -437,6 +437,7 @@ def main_ours(args):
         slot = max(("gemm1", "gemm2"), key=lambda s: kern[s][0])
         work = wm[slot]
     k_ms = kern[slot][0] / max(kern[slot][1], 1)
+    gemm_name = "moe_gemm_swap_kernel" if r["regime"] == "small_m" else "moe_gemm_kernel"
     bound = BOUND.get(args.workload, "hbm")
     if bound == "tensor":
         peak = peaks["bf16_tflops"] * FMT_TENSOR_RATIO[p["format"]]
@@ -472,8 +473,8 @@ def main_ours(args):
         "tokens_per_s": job_throughput(p["num_tokens"], world, args.steps, r["t_ms"]),
         "layer_tflops": wm["layer"]["flops"] / (step_ms / 1e3) / 1e12,
         "layer_gbs": wm["layer"]["bytes"] / (step_ms / 1e3) / 1e9,
-        "roofline": {"kernel": {"fused": "moe_fused_kernel", "gemm1": "moe_gemm_kernel (gate_up)",
-                                "gemm2": "moe_gemm_kernel (down)"}[slot], "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+        "roofline": {"kernel": {"fused": "moe_fused_kernel",
+                                "gemm1": gemm_name + " (gate_up)", "gemm2": gemm_name + " (down)"}[slot], "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
                      "frac": achieved / peak,
                      "traffic": stored_traffic(args.workload, {"fused": "moe_fused_kernel", "gemm1": "gemm1",
                                                               "gemm2": "gemm2"}[slot]) if not args.set else None,
