@@ -152,7 +152,22 @@ __host__ __device__ inline bool perm_small_case(int64_t R, int E) {
 
 // Shared-memory ints of the two-pass (per chunk) and the one-block permutation.
 __host__ __device__ inline int perm_chunk_smem_ints(int E) { return 3 * E + 1 + kPermChunk; }
-__host__ __device__ inline int perm_small_smem_ints(int E, int nwarps) { return nwarps * E + 2 * E + 1; }
+// One-block problems with few experts whose experts x slots fit a 16 KB
+// bitmap take the bitmap path (perm_bitmap_block); with many experts its
+// per-expert row scans cost more than the per-warp histograms.
+constexpr int kPermBitmapWords = 4096;
+constexpr int kPermBitmapMaxE = 64;
+__host__ __device__ inline int perm_bitmap_words(int64_t R, int E) {
+  return E * static_cast<int>((R + 31) / 32);
+}
+__host__ __device__ inline bool perm_bitmap_case(int64_t R, int E) {
+  return perm_small_case(R, E) && E <= kPermBitmapMaxE && perm_bitmap_words(R, E) <= kPermBitmapWords;
+}
+__host__ __device__ inline int perm_small_smem_ints(int64_t R, int E, int nwarps) {
+  const int hist = nwarps * E + 2 * E + 1;
+  const int bitmap = 2 * perm_bitmap_words(R, E) + 2 * E + 1;
+  return perm_bitmap_case(R, E) && bitmap > hist ? bitmap : hist;
+}
 
 // Exclusive scan of v[0..n) by one warp (n <= 1024); writes out[0..n] (n+1
 // entries, out[n] = total).  Each lane owns a contiguous run of entries.
@@ -300,7 +315,69 @@ __device__ void perm_scatter_chunk(const PermArgs& a, int c, int* sm) {
 }
 
 // The whole small case in the calling block.
+// One block, bitmap form: bit s of expert e's row is set when slot s routes
+// to e.  A slot's rank inside its expert (the stable order) is the prefix
+// popcount of its expert's row below it: per-word prefix counts of each row,
+// then one popcount of the slot's own word.  Every step is a parallel pass
+// over the slots, the words or the experts.
+__device__ void perm_bitmap_block(const PermArgs& a, int* sm) {
+  const int E = a.E;
+  const int R = static_cast<int>(a.R);
+  const int W = (R + 31) >> 5;                            // words per expert row
+  uint32_t* bits = reinterpret_cast<uint32_t*>(sm);        // [E][W]
+  int* wpre = sm + E * W;                                  // [E][W] set bits of the row before word w
+  int* total = wpre + E * W;                               // [E]
+  int* start = total + E;                                  // [E+1]
+  const int nthr = blockDim.x, nw = nthr >> 5;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < E * W; i += nthr) bits[i] = 0u;
+  __syncthreads();
+  for (int s = threadIdx.x; s < R; s += nthr) {
+    const int64_t x = a.idx[s];
+    if (x >= 0 && x < E) atomicOr(&bits[static_cast<int>(x) * W + (s >> 5)], 1u << (s & 31));
+    else if (x != -1) record_error(a.status, MOE_ERR_BAD_INDEX);
+  }
+  __syncthreads();
+  // per expert row: exclusive prefix of the words' popcounts, and the total
+  const int per = (W + 31) >> 5;
+  for (int e = warp; e < E; e += nw) {
+    const int b = min(W, lane * per), w_end = min(W, b + per);
+    int sum = 0;
+    for (int w = b; w < w_end; ++w) sum += __popc(bits[e * W + w]);
+    int incl = sum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+      if (lane >= off) incl += y;
+    }
+    int run = incl - sum;
+    for (int w = b; w < w_end; ++w) {
+      wpre[e * W + w] = run;
+      run += __popc(bits[e * W + w]);
+    }
+    if (lane == 31) total[e] = incl;
+  }
+  __syncthreads();
+  if (warp == 0) expert_tables_warp(total, start, E, a.o, true, lane);
+  __syncthreads();
+  for (int s = threadIdx.x; s < R; s += nthr) {
+    const int64_t x = a.idx[s];
+    int row = -1;
+    if (x >= 0 && x < E) {
+      const int e = static_cast<int>(x), w = s >> 5;
+      row = start[e] + wpre[e * W + w] + __popc(bits[e * W + w] & ((1u << (s & 31)) - 1u));
+      a.o.src_info[row] = s;
+    }
+    a.o.slot_to_row[s] = row;
+  }
+  __syncthreads();
+}
+
 __device__ void perm_small_block(const PermArgs& a, int* sm) {
+  if (perm_bitmap_case(a.R, a.E)) {
+    perm_bitmap_block(a, sm);
+    return;
+  }
   const int E = a.E;
   const int R = static_cast<int>(a.R);
   const int nw = blockDim.x >> 5;

@@ -322,7 +322,7 @@ PermArgs perm_args(const moe_problem_t* p, const int64_t* idx, const PermOut& o,
 cudaError_t launch_permute(const PermArgs& a, cudaStream_t st) {
   TimScope ts(MOE_SLOT_PERMUTE, st);
   if (perm_small_case(a.R, a.E))
-    return launch_k(perm_small_kernel, 1, 1024, perm_small_smem_ints(a.E, 32) * sizeof(int), st, a);
+    return launch_k(perm_small_kernel, 1, 1024, perm_small_smem_ints(a.R, a.E, 32) * sizeof(int), st, a);
   cudaError_t e = launch_k(perm_count_kernel, a.nblk, 256, a.E * sizeof(int), st, a);
   if (e != cudaSuccess) return e;
   return launch_k(perm_scatter_kernel, a.nblk, 256, perm_chunk_smem_ints(a.E) * sizeof(int), st, a);
