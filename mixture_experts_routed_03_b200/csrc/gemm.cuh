@@ -34,8 +34,9 @@
 //
 // Tiles are (active expert, n tile, 128-row m tile), handed out round-robin
 // over at most one CTA per SM, in groups of n tiles (see decode_tile):
-// expert-major with m fastest for gate_up, a few output n tiles at a time for
-// down.
+// expert-major with m fastest for gate_up; for down, one output n tile at a
+// time while the intermediate fits in L2, else expert-major.  (Small
+// per-expert batches use the swapped-operand GEMMs of gemm_swap.cuh.)
 //
 // L1 epilogue: h = min(g,c) * sigmoid(min(g,c)) * clamp(u,-c,c) is formed in
 // registers, the accumulator is released, then h is re-quantised (BF16 by
@@ -43,9 +44,10 @@
 // with an E4M3 scale against the per-expert c_input_scales) and stored in
 // expert order for L2.
 // L2 epilogue: the row is read into registers, the accumulator released, and
-// the row, times its router weight, red-added (float4 atomics) into the
-// token-ordered FP32 accumulator -- no (M*k, H) staging buffer -- or, in
-// staged mode, stored per row.
+// the row, times its router weight, added into the token-ordered FP32
+// accumulator -- float4 atomics through a 32 x 32 transpose (BF16, FP8) or
+// TMA bulk reduce-adds (NVFP4); no (M*k, H) staging buffer -- or, in staged
+// mode, stored per row.
 //
 // Every wait is bounded; a wait that runs out records MOE_ERR_TIMEOUT in the
 // workspace status word, raises a CTA-wide abort flag, drains the copies and
@@ -69,7 +71,9 @@ constexpr int kSFAStage = 4 * kSFTile;        // 4 K-steps of 64 e2m1
 constexpr int kSFBStage = 2 * 4 * kSFTile;    // 2 row blocks x 4 K-steps
 constexpr int kTmemCols = 512;
 // NVFP4 scale factors in TMEM: two buffers of 48 columns after the
-// accumulator, A scales (16 columns) then B scales (32 columns).
+// accumulator, A scales (16 columns) then B scales (32 columns).  (A ring of
+// four was measured no faster: the stage's twelve tcgen05.cp take ~600
+// cycles of the tensor pipe per K step whatever the ring depth.)
 constexpr int kSFCol0 = 256;
 constexpr int kSFBufCols = 48;
 constexpr int kSFBOff = 16;
@@ -774,15 +778,6 @@ __device__ __forceinline__ void gemm_phase(const GemmArgs& p, const CUtensorMap*
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-}
-
-// The same phase as an out-of-line call: the single-launch kernel strings
-// several phases together, and separate calls keep their register
-// allocations from interfering.
-template <int FMT, int EPI>
-__device__ __noinline__ void gemm_phase_call(const GemmArgs& p, const CUtensorMap* tmA, uint8_t* smem,
-                                             uint32_t tmem, volatile int* abort_flag, int cta, int ncta) {
-  gemm_phase<FMT, EPI>(p, tmA, smem, tmem, abort_flag, cta, ncta);
 }
 
 // Shared-memory header of every kernel that runs GEMM phases.
