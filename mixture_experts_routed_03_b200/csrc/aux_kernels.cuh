@@ -507,6 +507,7 @@ struct GatherArgs {
   const int* expert_ids;
   const int* num_active;
   int* tiles32;
+  int skip_rows;             // the GEMM reads the routed rows of x itself: no row / scale copies
 };
 
 // Tile table of the small-M GEMMs: tiles32[a] = 32-row tiles of the active
@@ -614,6 +615,7 @@ __global__ void __launch_bounds__(256) gather_kernel(GatherArgs g) {
   pdl_trigger();
   pdl_wait();
   if (g.tiles32 && blockIdx.x == 0 && threadIdx.x < 32) small_tile_table(g, threadIdx.x);
+  if (g.skip_rows) return;
   const int64_t nw = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   gather_rows<1>(g, (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5, nw, threadIdx.x & 31);
 }

@@ -246,6 +246,16 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// 16-byte asynchronous copy global -> shared (any 16-byte aligned addresses),
+// and an arrive on `bar` once all of this thread's earlier cp.async have
+// landed (the barrier's expected count must include that arrive).
+__device__ __forceinline__ void cp_async16(void* sdst, const void* gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(sdst)), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 // Asynchronous bulk reduce-add (TMA engine) of `bytes` FP32 values from
 // shared memory into global memory: dst[i] += src[i].  Both addresses 16-byte
 // aligned, bytes a multiple of 16.  The calling thread's shared-memory

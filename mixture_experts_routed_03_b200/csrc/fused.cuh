@@ -152,8 +152,10 @@ __global__ void __launch_bounds__(FusedShape<FMT, SWAP>::kThreads, 1)
   stamp(f, 2);
   if (ok) {
     if (f.gather.tiles32 && blockIdx.x == 0 && threadIdx.x < 32) small_tile_table(f.gather, threadIdx.x);
-    const GridIdx g = grid_idx();
-    gather_rows<2>(f.gather, g.gw, g.tw, g.lane);
+    if (!f.gather.skip_rows) {
+      const GridIdx g = grid_idx();
+      gather_rows<2>(f.gather, g.gw, g.tw, g.lane);
+    }
     ok = grid_barrier(f.gbar, &hdr->abort, f.status);
   }
   stamp(f, 3);

@@ -158,6 +158,12 @@ struct GemmArgs {
   // L2 output
   float* out;           // accumulate: [M][H]; staged: [R][H]
   int* status;
+  // small-M gate_up reading the routed rows in place (no gather): token rows
+  // of x, row_bytes each, and FP8 activation scales [M][x_sc_ld]
+  const uint8_t* x_rows;
+  int x_row_bytes;
+  const float* x_sc;
+  int x_sc_ld;
 };
 
 struct TileInfo {

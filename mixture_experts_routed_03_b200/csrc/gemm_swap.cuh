@@ -74,9 +74,12 @@ __device__ __forceinline__ void gemm_phase_swap(const GemmArgs& p, const CUtenso
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
+  // gate_up reading the routed rows straight from x (no gather): the whole
+  // producer warp copies them, 32 arrivals more per stage
+  const bool direct = EPI == EPI_L1 && p.x_rows != nullptr;
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], direct ? 1 + 32 : 1);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < NACC; ++b) {
@@ -96,7 +99,7 @@ __device__ __forceinline__ void gemm_phase_swap(const GemmArgs& p, const CUtenso
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    if (direct || lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       int issued = 0;
@@ -105,12 +108,32 @@ __device__ __forceinline__ void gemm_phase_swap(const GemmArgs& p, const CUtenso
         decode_tile(p, na, T, t);
         const uint8_t* wb =
             p.wB + (static_cast<size_t>(t.e) * p.n_tiles + t.n_tile) * p.k_stages * BB;
+        // direct: lane l brings routed row l of the tile (row 0's token for
+        // the rows past the tile's end, whose results are never used)
+        const uint8_t* xrow = nullptr;
+        if (direct) {
+          const int r = t.row0 + (lane < t.rows ? lane : 0);
+          xrow = p.x_rows + static_cast<size_t>(__ldg(p.src_info + r) / p.topk) * p.x_row_bytes;
+        }
         for (int ks = 0; ks < p.k_stages; ++ks) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status, 21)) goto producer_done;
           uint8_t* st = smem + stage * SB;
-          mbar_arrive_expect_tx(&full[stage], SB);
-          tma_load_2d(st, tmA, &full[stage], ks * kBK, t.row0);
-          bulk_load(st + kTStage, wb + static_cast<size_t>(ks) * BB, BB, &full[stage]);
+          if (direct) {
+            // row `lane` of the 128-byte-swizzled tile: 16-byte chunk c at c ^ (lane mod 8)
+            const uint8_t* src = xrow + ks * kBK;
+            uint8_t* dst = st + lane * kBK;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) cp_async16(dst + ((c ^ (lane & 7)) << 4), src + (c << 4));
+            cp_async_arrive(&full[stage]);
+            if (lane == 0) {
+              mbar_arrive_expect_tx(&full[stage], BB);
+              bulk_load(st + kTStage, wb + static_cast<size_t>(ks) * BB, BB, &full[stage]);
+            }
+          } else {
+            mbar_arrive_expect_tx(&full[stage], SB);
+            tma_load_2d(st, tmA, &full[stage], ks * kBK, t.row0);
+            bulk_load(st + kTStage, wb + static_cast<size_t>(ks) * BB, BB, &full[stage]);
+          }
           ++issued;
           if (++stage == S) {
             stage = 0;
@@ -119,7 +142,8 @@ __device__ __forceinline__ void gemm_phase_swap(const GemmArgs& p, const CUtenso
         }
       }
     producer_done:
-      if (*abort_flag) {
+      if (direct) asm volatile("cp.async.wait_all;" ::: "memory");
+      if (*abort_flag && lane == 0) {
         int st = stage;
         uint32_t ph = phase;
         for (int i = 0; i < S && i < issued; ++i) {
@@ -151,6 +175,8 @@ __device__ __forceinline__ void gemm_phase_swap(const GemmArgs& p, const CUtenso
             break;
           }
           tc_fence_after();
+          // rows written by cp.async (generic proxy) are read by the MMA (async proxy)
+          if (direct) fence_async_smem();
           if (FMT == FMT_FP8) {
             if (!mbar_wait(&acc_empty[ab], aphase ^ 1u, abort_flag, p.status, 24)) {
               ok = false;
@@ -225,13 +251,23 @@ __device__ __forceinline__ void gemm_phase_swap(const GemmArgs& p, const CUtenso
         // the weight block of this warp's rows (warp-uniform)
         const int wrow = (EPI == EPI_L1) ? l1_tile_row(t.n_tile, wr, p.I) : (t.n_tile * kBN + wr);
         const float* sbe = p.sb + (static_cast<size_t>(t.e) * p.sb_nb + (wrow >> 7)) * p.sb_kb;
-        // lane i holds routed row i's activation scale of the next K block
-        const float* sa_col = p.sa_t + t.srow0 + lane;
+        // lane i holds routed row i's activation scale of the next K block:
+        // from x's scales by token (direct), or the gathered transposed copy
+        const float* sa_col;
+        size_t sa_step;
+        if (direct) {
+          const int r = t.row0 + (lane_row ? lane : 0);
+          sa_col = p.x_sc + static_cast<size_t>(__ldg(p.src_info + r) / p.topk) * p.x_sc_ld;
+          sa_step = 1;
+        } else {
+          sa_col = p.sa_t + t.srow0 + lane;
+          sa_step = static_cast<size_t>(p.sa_ld);
+        }
         float nx_sa = sa_col[0];
         bool ok = true;
         for (int ks = 0; ks < p.k_stages; ++ks) {
           const float sa = nx_sa;
-          if (ks + 1 < p.k_stages) nx_sa = sa_col[static_cast<size_t>(ks + 1) * p.sa_ld];
+          if (ks + 1 < p.k_stages) nx_sa = sa_col[static_cast<size_t>(ks + 1) * sa_step];
           if (!mbar_wait(&acc_full[ab], aphase, abort_flag, p.status, 25)) {
             ok = false;
             break;

@@ -382,6 +382,8 @@ moe_status_t plan_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_we
   g.expert_ids = b.expert_ids;
   g.num_active = b.num_active;
   g.tiles32 = pl.swap ? b.tiles32 : nullptr;
+  // the small-M gate_up copies its routed rows straight from x
+  g.skip_rows = pl.swap ? 1 : 0;
 
   // L1: gate_up
   if (!make_map(&pl.ta1, b.x_perm, x_row_bytes(fmt, H), uint64_t(R), uint32_t(tile_rows))) return MOE_ERR_CUDA;
@@ -402,6 +404,12 @@ moe_status_t plan_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_we
   a.a_scale_offsets = b.a_scale_offsets;
   a.tile_offsets = pl.swap ? b.tiles32 : b.tile_offsets;
   a.tile_rows = tile_rows;
+  if (pl.swap) {
+    a.x_rows = static_cast<const uint8_t*>(act->x);
+    a.x_row_bytes = x_row_bytes(fmt, H);
+    a.x_sc = static_cast<const float*>(act->x_scale);   // FP8; null for BF16
+    a.x_sc_ld = H / 128;
+  }
   a.src_info = b.src_info;
   a.topk_weights = topk_weights;
   a.sfa = b.x_sf;
@@ -427,6 +435,8 @@ moe_status_t plan_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_we
   if (!make_map(&pl.ta2, b.h, h_row_bytes(fmt, I), uint64_t(R), uint32_t(tile_rows))) return MOE_ERR_CUDA;
   GemmArgs& a2 = pl.l2;
   a2 = a;
+  a2.x_rows = nullptr;   // the down leg reads the intermediate through its TMA map
+  a2.x_sc = nullptr;
   a2.k_stages = h_row_bytes(fmt, I) / 128;
   a2.n_tiles = H / 256;
   // Output n tiles in groups: a group's slice of the FP32 accumulator
