@@ -134,6 +134,7 @@ struct PermOut {
   int* num_active;
   int* a_scale_offsets;
   int* tile_offsets;
+  int* tiles32;          // optional: the small-M GEMMs' 32-row tile table (E+1)
 };
 
 struct PermArgs {
@@ -176,13 +177,14 @@ __host__ __device__ inline int perm_small_smem_ints(int64_t R, int E, int nwarps
 // when `tables` is set, the layout arrays in global memory: expert_counts,
 // expert_start_indices, a_scale_offsets (scan of the counts padded to 128),
 // expert_ids (active experts in order, -1 after them), num_active and
-// tile_offsets (scan of the active experts' 128-row m tiles).  The four scans
-// run together: each lane takes E/32 consecutive experts, sums them, and one
-// round of shuffles scans the four sums at once.
+// tile_offsets (scan of the active experts' 128-row m tiles), and when asked
+// the small-M GEMMs' table of 32-row tiles.  The scans run together: each
+// lane takes E/32 consecutive experts, sums them, and one round of shuffles
+// scans all the sums at once.
 __device__ void expert_tables_warp(const int* total, int* start, int E, const PermOut& o, bool tables, int lane) {
   const int per = (E + 31) >> 5;
   const int b = min(E, lane * per), e_end = min(E, b + per);
-  int c = 0, pad = 0, act = 0, mt = 0;
+  int c = 0, pad = 0, act = 0, mt = 0, m32 = 0;
   for (int e = b; e < e_end; ++e) {
     const int t = total[e];
     const int m = (t + 127) >> 7;
@@ -190,23 +192,27 @@ __device__ void expert_tables_warp(const int* total, int* start, int E, const Pe
     pad += m << 7;
     act += t > 0 ? 1 : 0;
     mt += m;
+    m32 += (t + 31) >> 5;
   }
-  int ic = c, ip = pad, ia = act, im = mt;
+  int ic = c, ip = pad, ia = act, im = mt, i32 = m32;
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
     const int xc = __shfl_up_sync(0xFFFFFFFFu, ic, off);
     const int xp = __shfl_up_sync(0xFFFFFFFFu, ip, off);
     const int xa = __shfl_up_sync(0xFFFFFFFFu, ia, off);
     const int xm = __shfl_up_sync(0xFFFFFFFFu, im, off);
+    const int x32 = __shfl_up_sync(0xFFFFFFFFu, i32, off);
     if (lane >= off) {
       ic += xc;
       ip += xp;
       ia += xa;
       im += xm;
+      i32 += x32;
     }
   }
   const int na = __shfl_sync(0xFFFFFFFFu, ia, 31);
-  int rc = ic - c, rp = ip - pad, ra = ia - act, rm = im - mt;   // exclusive bases of this lane
+  // exclusive bases of this lane
+  int rc = ic - c, rp = ip - pad, ra = ia - act, rm = im - mt, r32 = i32 - m32;
   for (int e = b; e < e_end; ++e) {
     const int t = total[e];
     const int m = (t + 127) >> 7;
@@ -218,6 +224,7 @@ __device__ void expert_tables_warp(const int* total, int* start, int E, const Pe
       if (t > 0) {
         o.expert_ids[ra] = e;
         o.tile_offsets[ra] = rm;
+        if (o.tiles32) o.tiles32[ra] = r32;
       }
       if (e >= na) o.expert_ids[e] = -1;
     }
@@ -226,6 +233,7 @@ __device__ void expert_tables_warp(const int* total, int* start, int E, const Pe
     if (t > 0) {
       ++ra;
       rm += m;
+      r32 += (t + 31) >> 5;
     }
   }
   if (lane == 31) {
@@ -235,6 +243,7 @@ __device__ void expert_tables_warp(const int* total, int* start, int E, const Pe
       o.a_scale_offsets[E] = ip;
       *o.num_active = na;
       o.tile_offsets[na] = im;
+      if (o.tiles32) o.tiles32[na] = i32;
     }
   }
 }

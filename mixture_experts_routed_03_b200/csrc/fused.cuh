@@ -32,6 +32,7 @@ struct FusedArgs {
   int do_route;
   PermArgs perm;
   int perm_small;
+  int gather_phase;     // 0: the small-M GEMMs read x themselves and the permute built their tile table
   GatherArgs gather;
   float4* acc;
   int64_t acc_n4;
@@ -150,7 +151,7 @@ __global__ void __launch_bounds__(FusedShape<FMT, SWAP>::kThreads, 1)
   }
   if (ok) ok = grid_barrier(f.gbar, &hdr->abort, f.status);
   stamp(f, 2);
-  if (ok) {
+  if (ok && f.gather_phase) {
     if (f.gather.tiles32 && blockIdx.x == 0 && threadIdx.x < 32) small_tile_table(f.gather, threadIdx.x);
     if (!f.gather.skip_rows) {
       const GridIdx g = grid_idx();

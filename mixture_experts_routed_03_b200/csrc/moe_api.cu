@@ -790,6 +790,11 @@ moe_status_t moe_fused(const moe_problem_t* p, const moe_act_t* act, const moe_w
             reinterpret_cast<int*>(base + L.src_info),   reinterpret_cast<int*>(base + L.slot_to_row),
             reinterpret_cast<int*>(base + L.expert_ids), reinterpret_cast<int*>(base + L.num_active),
             reinterpret_cast<int*>(base + L.a_scale_offsets), reinterpret_cast<int*>(base + L.tile_offsets)};
+  // small-M tiles: the permutation also writes their tile table, and as the
+  // GEMMs read the routed rows of x themselves there is no gather phase
+  const bool small_m = small_m_tiles(p);
+  if (small_m) o.tiles32 = reinterpret_cast<int*>(base + L.tiles32);
+  f.gather_phase = small_m ? 0 : 1;
   f.perm = perm_args(p, idx, o, reinterpret_cast<int*>(base + L.block_counts), L.nblk, status);
   f.perm_small = perm_small_case(f.perm.R, f.perm.E) ? 1 : 0;
   FfnBuffers b{};
