@@ -2,6 +2,7 @@
 """Throughput of the routed MoE FFN layer (moe_fused) on B200 GPUs.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+                    [--chain] [--hot-l2] [--set KEY=VALUE ...]
 
 A step is one moe_fused call -- routing (when the workload routes from
 logits), permutation, the two grouped GEMMs with their fused epilogues and the
@@ -56,6 +57,8 @@ def parse():
     ap.add_argument("--chain", action="store_true",
                     help="time the multi-launch chain moe_route/moe_permute/moe_ffn/moe_combine "
                          "instead of the single moe_fused launch (per-kernel breakdown)")
+    ap.add_argument("--hot-l2", action="store_true",
+                    help="no L2 flush between steps (a hot-L2 number, reported separately)")
     ap.add_argument("--set", action="append", default=[], metavar="KEY=VALUE",
                     help="override a workload field (a smaller case for profiling)")
     return ap.parse_args()
@@ -255,6 +258,8 @@ def run_ours(args, rank, world, local_rank):
         # write 512 MiB, then read another 512 MiB: the read evicts the
         # write's dirty lines, so their write-back lands before the timed
         # interval instead of inside the step
+        if args.hot_l2:
+            return
         flush.fill_(i & 0xFF)
         torch.sum(flush_rd, dim=0, out=flush_sink)
 
@@ -469,7 +474,9 @@ def main_ours(args):
                    "num_topk": p["num_topk"], "format": p["format"], "routing": p["routing"],
                    "active_experts": r["num_active"], "gemm_tiles": r["regime"],
                    "parallelism": f"dp{world} (replicas)",
-                   "l2": "flushed before every timed step, outside the step interval: 512 MiB write, then a 512 MiB read of another buffer"},
+                   "l2": ("hot: no flush between steps" if args.hot_l2 else
+                          "flushed before every timed step, outside the step interval: 512 MiB write, "
+                          "then a 512 MiB read of another buffer")},
         "tokens_per_s": job_throughput(p["num_tokens"], world, args.steps, r["t_ms"]),
         "layer_tflops": wm["layer"]["flops"] / (step_ms / 1e3) / 1e12,
         "layer_gbs": wm["layer"]["bytes"] / (step_ms / 1e3) / 1e9,
