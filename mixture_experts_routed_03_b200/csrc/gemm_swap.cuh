@@ -12,11 +12,14 @@
 // (routed rows); per-K-block FP8 partials take 64 columns, so eight of them
 // are in flight.
 //
-// Roles as in the large-M GEMM: warp 0 lane 0 loads the stage (TMA of the
-// 32 routed rows, one bulk copy of the prepared weight block), warp 1 lane 0
-// issues the MMAs, warps 2..9 are the epilogue: warp (q, half) reads lanes
-// 32q..32q+31 of the accumulator of weight rows 128*half.., one weight row
-// per thread and 32 routed rows in its registers.
+// Roles as in the large-M GEMM: warp 0 loads the stage -- lane 0 one bulk
+// copy of the prepared weight block, and the 32 routed rows either by TMA
+// from the intermediate (down) or, for gate_up, by the whole warp straight
+// from x by token id (eight 16-byte cp.async per lane into the swizzled
+// rows, so no gather is needed) -- warp 1 lane 0 issues the MMAs, warps
+// 2..9 are the epilogue: warp (q, half) reads lanes 32q..32q+31 of the
+// accumulator of weight rows 128*half.., one weight row per thread and 32
+// routed rows in its registers.
 //
 // Gate_up epilogue: every thread stages its promoted FP32 row in shared
 // memory; after a barrier of the eight warps each warp takes four routed
