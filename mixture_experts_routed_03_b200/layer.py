@@ -1,5 +1,6 @@
 """A routed-MoE layer object over the C ABI: owns the device workspace and the
-prepared NVFP4 scale tiles, and forwards calls to ``api``.
+prepared weight blobs (the tensor-core tile layout ``moe_prepare_weights``
+writes once, NVFP4 scale tiles included), and forwards calls to ``api``.
 
 torch supplies device memory and streams only; every step runs in the
 library's kernels.
@@ -44,7 +45,8 @@ class MoELayer:
              activation_clamp, format, num_tokens = the largest batch served)
     weights: dict of device tensors w13, w13_scale, w2, w2_scale and, for
              NVFP4, gate_up_expert_scales, down_expert_scales, c_input_scales
-             (logical layouts of include/moe.h; NVFP4 scales are prepared here)
+             (logical layouts of include/moe.h; the weights are prepared here)
+    p may also carry "tile_regime" ("auto", "large_m", "small_m")
     """
 
     def __init__(self, p, weights, device=None, fast_math=1):
