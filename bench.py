@@ -383,19 +383,14 @@ def run_ours(args, rank, world, local_rank):
                 host_inputs=(d, L) if rank == 0 else None)
 
 
-def cpu_baseline(p, d, seconds):
-    """The oracle, as it stands, on a bounded sample of this workload's tokens."""
+def _oracle_sample(p, host, seconds):
+    """Runs the oracle on growing token samples until `seconds` of CPU work;
+    returns (tokens done, seconds spent)."""
     import numpy as np
-    from mixture_experts_routed_03_b200 import workloads
     from oracle import moe as O
 
-    host = workloads.to_numpy({k: v for k, v in d.items()})
-    if p["routing"] == "logits":
-        host["topk_idx"], host["topk_weights"] = O.route(host["logits"], host["bias"], p["num_topk"])
-        host["topk_weights"] = host["topk_weights"].astype(np.float32)
     M, k = p["num_tokens"], p["num_topk"]
-    rng = np.random.default_rng(0)
-    order = rng.permutation(M)
+    order = np.random.default_rng(0).permutation(M)
     n, done, t_total = 1, 0, 0.0
     while True:
         toks = np.sort(order[done: done + n])
@@ -405,20 +400,41 @@ def cpu_baseline(p, d, seconds):
         if p["routing"] == "logits":
             O.route(host["logits"][toks], host["bias"], k)
         O.moe_forward(p, host, host["topk_idx"], host["topk_weights"], tokens=toks)
-        dt = time.perf_counter() - t0
-        t_total += dt
+        t_total += time.perf_counter() - t0
         done += toks.size
         if t_total >= seconds or done >= M:
             break
         n = min(M - done, max(1, int(n * 2)))
+    return done, t_total
+
+
+def cpu_baseline(p, d, seconds):
+    """The oracle, as it stands, on a bounded sample of this workload's tokens,
+    with all host threads and with one thread."""
+    import numpy as np
+    from mixture_experts_routed_03_b200 import workloads
+    from oracle import moe as O
+
+    host = workloads.to_numpy({k: v for k, v in d.items()})
+    if p["routing"] == "logits":
+        host["topk_idx"], host["topk_weights"] = O.route(host["logits"], host["bias"], p["num_topk"])
+        host["topk_weights"] = host["topk_weights"].astype(np.float32)
+    M, k = p["num_tokens"], p["num_topk"]
+    done, t_total = _oracle_sample(p, host, seconds)
     try:
-        from threadpoolctl import threadpool_info
+        from threadpoolctl import threadpool_info, threadpool_limits
         cores = max([int(i.get("num_threads", 1)) for i in threadpool_info()] or [1])
+        with threadpool_limits(limits=1):
+            done1, t1 = _oracle_sample(p, host, seconds / 3)
+        one = dict(value=done1 * k / t1, cores=1,
+                   sample=f"{done1} of {M} tokens ({done1 * k} routed slots), {t1:.1f} s")
     except Exception:
         cores = os.cpu_count()
+        one = None
     return dict(value=done * k / t_total, unit="routed_tokens/s", cores=cores, kind="oracle",
                 sample=f"{done} of {M} tokens ({done * k} routed slots), float64 numpy oracle incl. "
-                       f"per-expert weight decode, {t_total:.1f} s")
+                       f"per-expert weight decode, {t_total:.1f} s",
+                one_thread=one)
 
 
 def main_ours(args):
