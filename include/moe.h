@@ -219,7 +219,10 @@ moe_status_t moe_prepare_weights(const moe_problem_t* problem, const moe_weights
  * Per token: score_e = logit_e + bias_e (one FP32 add); the k highest scores
  * in descending order, ties to the lower expert index, NaN scores last;
  * topk_weights = softmax over the chosen k of the UNBIASED logits.
- * Writes topk_idx int64 [M, k] and topk_weights fp32 [M, k]. */
+ * Writes topk_idx int64 [M, k] and topk_weights fp32 [M, k].  The indices
+ * are defined for any logits (NaN ranks last, +-inf compare as themselves);
+ * the weights of a token are unspecified when one of its chosen logits is
+ * not finite (+inf, -inf or NaN), since the softmax has no value there. */
 moe_status_t moe_route(const moe_problem_t* problem, const float* logits, const float* bias,
                        int64_t* topk_idx, float* topk_weights, void* stream);
 
@@ -297,6 +300,41 @@ moe_status_t moe_fused(const moe_problem_t* problem, const moe_act_t* act,
  * allocated or freed, by this library or any other. */
 moe_status_t moe_permute_noalloc(const moe_problem_t* problem, const int64_t* topk_idx,
                                  const moe_layout_t* layout, int32_t* device_status, void* stream);
+
+/* Where moe_fused leaves its working data inside the workspace, for
+ * inspection and testing: byte offsets from the workspace base for a call
+ * with this problem (the offsets depend on num_tokens, so pass the call's
+ * problem).  After a moe_fused call has completed, the regions hold
+ *   status               int32 sticky status word
+ *   topk_idx             int64 [M, k]   routing chosen in-kernel (only when
+ *   topk_weights         fp32  [M, k]   the call routed from logits)
+ *   expert_counts .. tile_offsets       the layout of moe_layout_t, int32
+ *   intermediate         the re-quantised intermediate [R, I] in expert
+ *                        order, and at intermediate_scales its scales, in
+ *                        the layout moe_ffn gives its `intermediate` buffer;
+ *                        scale_rows is P, the padded scale rows
+ *   accumulator          fp32 [M, H], the router-weighted sum before the
+ *                        BF16 rounding
+ * (Struct_mega_ffn_ep_combine_send lists these operands: expert_start_indices,
+ * expert_ids, a_scale_offsets, src_info.)  Host only; nothing is launched. */
+typedef struct {
+  size_t status;
+  size_t topk_idx;
+  size_t topk_weights;
+  size_t expert_counts;
+  size_t expert_start_indices;
+  size_t src_info;
+  size_t slot_to_row;
+  size_t expert_ids;
+  size_t num_active;
+  size_t a_scale_offsets;
+  size_t tile_offsets;
+  size_t intermediate;
+  size_t intermediate_scales;
+  int64_t scale_rows;
+  size_t accumulator;
+} moe_workspace_offsets_t;
+moe_status_t moe_get_workspace_offsets(const moe_problem_t* problem, moe_workspace_offsets_t* offsets);
 
 /* Per-kernel timing, for measurement.  moe_timing_enable(1, max_calls)
  * creates CUDA events for up to max_calls calls (once, on the current

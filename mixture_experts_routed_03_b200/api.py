@@ -39,7 +39,7 @@ EXPORTS = (
     "moe_get_prepared_weights_size",
     "moe_route", "moe_permute", "moe_ffn", "moe_get_intermediate_size", "moe_combine",
     "moe_fused", "moe_read_status", "moe_status_string", "moe_timing_enable", "moe_timing_read",
-    "moe_permute_noalloc", "moe_get_tile_regime",
+    "moe_permute_noalloc", "moe_get_tile_regime", "moe_get_workspace_offsets",
 )
 
 SLOTS = ("route", "permute", "gather", "gemm1", "zero", "gemm2", "finalize", "combine", "fused")
@@ -85,6 +85,15 @@ class Layout(ctypes.Structure):
         "expert_ids", "num_active", "a_scale_offsets", "tile_offsets")]
 
 
+WS_OFFSET_FIELDS = ("status", "topk_idx", "topk_weights", "expert_counts", "expert_start_indices",
+                    "src_info", "slot_to_row", "expert_ids", "num_active", "a_scale_offsets",
+                    "tile_offsets", "intermediate", "intermediate_scales", "scale_rows", "accumulator")
+
+
+class WorkspaceOffsets(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64 if n == "scale_rows" else ctypes.c_size_t) for n in WS_OFFSET_FIELDS]
+
+
 _lib = None
 
 
@@ -110,6 +119,7 @@ def lib():
                         vp, i32, vp, vp, vp, sz, vp],
             "moe_get_intermediate_size": [P, ctypes.POINTER(sz), ctypes.POINTER(sz)],
             "moe_get_tile_regime": [P, ctypes.POINTER(i32)],
+            "moe_get_workspace_offsets": [P, ctypes.POINTER(WorkspaceOffsets)],
             "moe_combine": [P, ctypes.POINTER(Layout), vp, vp, i32, vp, vp],
             "moe_fused": [P, ctypes.POINTER(Act), ctypes.POINTER(Weights), vp, vp, vp, vp, vp, vp, sz, vp],
             "moe_read_status": [vp, vp],
@@ -207,6 +217,14 @@ def tile_regime(prob):
     r = ctypes.c_int32(0)
     _check("moe_get_tile_regime", lib().moe_get_tile_regime(ctypes.byref(prob), ctypes.byref(r)))
     return {v: k for k, v in TILE_REGIMES.items()}[r.value]
+
+
+def workspace_offsets(prob):
+    """{region: byte offset} of moe_fused's working data in the workspace
+    (plus 'scale_rows', the padded scale rows P)."""
+    o = WorkspaceOffsets()
+    _check("moe_get_workspace_offsets", lib().moe_get_workspace_offsets(ctypes.byref(prob), ctypes.byref(o)))
+    return {n: int(getattr(o, n)) for n in WS_OFFSET_FIELDS}
 
 
 def intermediate_size(prob):

@@ -1,0 +1,245 @@
+// mma_peak.cu -- dense tensor-core throughput of this GPU, for the roofline.
+//
+// A measurement tool, not part of the layer: every CTA keeps one operand
+// stage resident in shared memory and one thread issues tcgen05.mma back to
+// back into one TMEM accumulator, the way the grouped GEMMs issue their K
+// steps, so the achieved rate is the tensor pipe's own, with no memory
+// traffic.  Shapes: M = 128 per CTA (cta_group::1) or M = 256 per CTA pair
+// (cta_group::2, each CTA holding its 128 rows of A and half of B's N rows),
+// N = 128 or 256, K = one 32-byte step per instruction (BF16 K = 16, E4M3
+// K = 32, block-scaled E2M1 K = 64).  Operands are zero, so no value can
+// slow the pipe down.  Every wait is bounded (status 6 on a time-out).
+//
+// extern "C" moe_peak_mma(kind, n, pair, iters, scratch, stream, *tflops, *cycles)
+//   kind   0 BF16 (kind::f16), 1 E4M3 (kind::f8f6f4), 2 NVFP4
+//          (kind::mxf4nvf4.block_scale.scale_vec::4X; cta_group::1 only)
+//   iters  K blocks of 4 instructions each CTA (or pair) issues
+//   scratch device buffer of at least 16 bytes x grid (status, cycles)
+// Returns 0 on success; *tflops = dense FLOPs / event time over the whole
+// grid (one CTA per SM), *cycles = SM cycles per instruction of one CTA.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace {
+
+using namespace moe;
+
+constexpr int kPeakThreads = 128;
+constexpr int kOffA = 0;            // 128 rows x 128 bytes
+constexpr int kOffB = 16384;        // up to 256 rows x 128 bytes
+constexpr int kOffSF = 49152;       // NVFP4: 12 scale tiles of 512 bytes
+constexpr int kOffBar = 55296;
+constexpr int kPeakSmem = 56320 + 1024;
+
+__device__ __forceinline__ void mma_f16_pair(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(1u)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_f8_pair(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(1u)
+      : "memory");
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+template <int KIND, int N, bool PAIR>
+__global__ void __launch_bounds__(kPeakThreads, 1) mma_peak_kernel(int iters, int* out) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base =
+      reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* done = reinterpret_cast<uint64_t*>(base + kOffBar);
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(base + kOffBar + 64);
+  int* status = reinterpret_cast<int*>(base + kOffBar + 128);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool leader = !PAIR || cluster_rank() == 0;
+
+  for (int i = threadIdx.x; i < kOffBar / 16; i += blockDim.x)
+    reinterpret_cast<uint4*>(base)[i] = make_uint4(0u, 0u, 0u, 0u);
+  fence_async_smem();
+  if (threadIdx.x == 0) {
+    mbar_init(done, 1);
+    *status = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (warp == 0) {
+    if (PAIR) {
+      asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tslot)),
+                   "r"(512)
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    } else {
+      tmem_alloc(tslot, 512);
+    }
+  }
+  tc_fence_before();
+  if (PAIR) cluster_sync(); else __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+
+  long long t0 = 0, t1 = 0;
+  if (leader && warp == 1 && lane == 0) {
+    if (KIND == 2) {
+      // scale factors of 4 K steps for A (16 columns) and B (32 columns),
+      // issued by this thread ahead of its MMAs
+      for (int t = 0; t < 12; ++t)
+        tmem_copy_sf(tmem + 256 + 4 * t, sdesc_sf_tile(smem_u32(base + kOffSF + 512 * t)));
+    }
+    constexpr uint32_t M = PAIR ? 256 : 128;
+    constexpr uint32_t idesc_m = (M >> 4) << 24;
+    const uint32_t idesc = (KIND == 0)   ? ((idesc_dense(1, 1, N) & ~(31u << 24)) | idesc_m)
+                           : (KIND == 1) ? ((idesc_dense(0, 0, N) & ~(31u << 24)) | idesc_m)
+                                         : idesc_nvf4(N);
+    const uint64_t adesc = sdesc_sw128(smem_u32(base + kOffA));
+    const uint64_t bdesc = sdesc_sw128(smem_u32(base + kOffB));
+    t0 = clock64();
+    for (int it = 0; it < iters; ++it) {
+#pragma unroll
+      for (int kc = 0; kc < 4; ++kc) {
+        const uint64_t a = adesc + static_cast<uint64_t>(2 * kc);
+        const uint64_t b = bdesc + static_cast<uint64_t>(2 * kc);
+        if (KIND == 0) {
+          if (PAIR) mma_f16_pair(tmem, a, b, idesc); else mma_f16(tmem, a, b, idesc, 1u);
+        } else if (KIND == 1) {
+          if (PAIR) mma_f8_pair(tmem, a, b, idesc); else mma_f8(tmem, a, b, idesc, 1u);
+        } else {
+          mma_nvf4(tmem, a, b, idesc, tmem + 256 + 4 * kc, tmem + 256 + 16 + 8 * kc, 1u);
+        }
+      }
+    }
+    if (PAIR) {
+      asm volatile(
+          "{\n\t.reg .b16 m;\n\tmov.b16 m, 3;\n\t"
+          "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], m;\n\t}" ::"r"(
+              smem_u32(done))
+          : "memory");
+    } else {
+      mma_commit(done);
+    }
+  }
+  // every thread waits for the MMAs to finish (bounded)
+  {
+    const unsigned long long g0 = globaltimer_ns();
+    while (!mbar_test(done, 0)) {
+      if (globaltimer_ns() - g0 > kWaitLimitNs) {
+        *status = MOE_ERR_TIMEOUT;
+        break;
+      }
+    }
+  }
+  if (leader && warp == 1 && lane == 0) {
+    t1 = clock64();
+    out[4 * blockIdx.x + 0] = *status;
+    reinterpret_cast<long long*>(out)[2 * blockIdx.x + 1] = t1 - t0;
+  } else if (!leader && threadIdx.x == 0) {
+    out[4 * blockIdx.x + 0] = *status;
+    reinterpret_cast<long long*>(out)[2 * blockIdx.x + 1] = 0;
+  }
+  tc_fence_before();
+  if (PAIR) cluster_sync(); else __syncthreads();
+  tc_fence_after();
+  if (warp == 0) {
+    if (PAIR)
+      asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512) : "memory");
+    else
+      tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int KIND, int N, bool PAIR>
+int run_peak(int iters, int* scratch, cudaStream_t st, float* tflops, float* cycles) {
+  auto kern = mma_peak_kernel<KIND, N, PAIR>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kPeakSmem) != cudaSuccess) return 4;
+  int dev = 0, nsm = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  cudaLaunchConfig_t cfg{};
+  cfg.blockDim = dim3(kPeakThreads);
+  cfg.dynamicSmemBytes = kPeakSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  int grid = nsm;
+  if (PAIR) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cfg.gridDim = dim3(2);
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess || clusters < 1) return 4;
+    grid = 2 * clusters;
+  }
+  cfg.gridDim = dim3(grid);
+  cudaEvent_t e0, e1;
+  cudaEventCreate(&e0);
+  cudaEventCreate(&e1);
+  // one short warm-up launch, then the timed one
+  if (cudaLaunchKernelEx(&cfg, kern, 64, scratch) != cudaSuccess) return 4;
+  cudaEventRecord(e0, st);
+  if (cudaLaunchKernelEx(&cfg, kern, iters, scratch) != cudaSuccess) return 4;
+  cudaEventRecord(e1, st);
+  if (cudaEventSynchronize(e1) != cudaSuccess) return 4;
+  float ms = 0.0f;
+  cudaEventElapsedTime(&ms, e0, e1);
+  cudaEventDestroy(e0);
+  cudaEventDestroy(e1);
+  int* host = new int[4 * grid];
+  cudaMemcpy(host, scratch, sizeof(int) * 4 * grid, cudaMemcpyDeviceToHost);
+  int status = 0;
+  double cyc = 0.0;
+  int n = 0;
+  for (int b = 0; b < grid; ++b) {
+    if (host[4 * b]) status = host[4 * b];
+    const long long c = reinterpret_cast<long long*>(host)[2 * b + 1];
+    if (c > 0) {
+      cyc += static_cast<double>(c);
+      ++n;
+    }
+  }
+  delete[] host;
+  const double k = (KIND == 0) ? 16.0 : (KIND == 1 ? 32.0 : 64.0);
+  const double m = PAIR ? 256.0 : 128.0;
+  const double issuers = PAIR ? grid / 2 : grid;
+  const double flops = 2.0 * m * N * k * 4.0 * iters * issuers;
+  *tflops = static_cast<float>(flops / (ms * 1e-3) / 1e12);
+  *cycles = n ? static_cast<float>(cyc / n / (4.0 * iters)) : 0.0f;
+  return status;
+}
+
+}  // namespace
+
+extern "C" int moe_peak_mma(int kind, int n, int pair, int iters, void* scratch, void* stream, float* tflops,
+                            float* cycles) {
+  if (!scratch || !tflops || !cycles || iters < 1) return 1;
+  int* s = static_cast<int*>(scratch);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (kind == 0 && n == 256 && !pair) return run_peak<0, 256, false>(iters, s, st, tflops, cycles);
+  if (kind == 0 && n == 128 && !pair) return run_peak<0, 128, false>(iters, s, st, tflops, cycles);
+  if (kind == 0 && n == 256 && pair) return run_peak<0, 256, true>(iters, s, st, tflops, cycles);
+  if (kind == 1 && n == 256 && !pair) return run_peak<1, 256, false>(iters, s, st, tflops, cycles);
+  if (kind == 1 && n == 128 && !pair) return run_peak<1, 128, false>(iters, s, st, tflops, cycles);
+  if (kind == 1 && n == 256 && pair) return run_peak<1, 256, true>(iters, s, st, tflops, cycles);
+  if (kind == 1 && n == 128 && pair) return run_peak<1, 128, true>(iters, s, st, tflops, cycles);
+  if (kind == 2 && n == 256 && !pair) return run_peak<2, 256, false>(iters, s, st, tflops, cycles);
+  if (kind == 2 && n == 128 && !pair) return run_peak<2, 128, false>(iters, s, st, tflops, cycles);
+  return 2;
+}

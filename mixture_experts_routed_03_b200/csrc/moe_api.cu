@@ -582,6 +582,29 @@ moe_status_t moe_init(int device) {
   return ok ? MOE_OK : MOE_ERR_CUDA;
 }
 
+moe_status_t moe_get_workspace_offsets(const moe_problem_t* p, moe_workspace_offsets_t* o) {
+  moe_status_t s = check_problem(p);
+  if (s != MOE_OK) return s;
+  if (!o) return MOE_ERR_INVALID_ARG;
+  const WsLayout L = make_layout(p);
+  o->status = L.header;
+  o->topk_idx = L.route_idx;
+  o->topk_weights = L.route_w;
+  o->expert_counts = L.counts;
+  o->expert_start_indices = L.starts;
+  o->src_info = L.src_info;
+  o->slot_to_row = L.slot_to_row;
+  o->expert_ids = L.expert_ids;
+  o->num_active = L.num_active;
+  o->a_scale_offsets = L.a_scale_offsets;
+  o->tile_offsets = L.tile_offsets;
+  o->intermediate = L.h;
+  o->intermediate_scales = L.h_sf;
+  o->scale_rows = L.P;
+  o->accumulator = L.acc;
+  return MOE_OK;
+}
+
 moe_status_t moe_get_workspace_size(const moe_problem_t* p, size_t* bytes) {
   moe_status_t s = check_problem(p);
   if (s != MOE_OK) return s;

@@ -125,6 +125,32 @@ class MoELayer:
                     out, stream=stream)
         return out
 
+    def workspace_views(self, M):
+        """Device views of what the last moe_fused call with M tokens left in
+        the workspace (layout arrays, in-kernel routing, the re-quantised
+        intermediate and its scales, the FP32 accumulator), for inspection.
+        Read them only after that call has completed."""
+        prob = self.problem(M)
+        off = api.workspace_offsets(prob)
+        k, E, H = self.p["num_topk"], self.p["num_experts"], self.p["hidden"]
+        R = M * k
+        n_int, so = api.intermediate_size(prob)
+        ws = self.ws
+
+        def i32(name, n):
+            return ws[off[name]: off[name] + 4 * n].view(torch.int32)
+
+        v = {name: i32(name, n) for name, n in (
+            ("expert_counts", E), ("expert_start_indices", E + 1), ("src_info", R), ("slot_to_row", R),
+            ("expert_ids", E), ("num_active", 1), ("a_scale_offsets", E + 1), ("tile_offsets", E + 1))}
+        v["topk_idx"] = ws[off["topk_idx"]: off["topk_idx"] + 8 * R].view(torch.int64).view(M, k)
+        v["topk_weights"] = ws[off["topk_weights"]: off["topk_weights"] + 4 * R].view(torch.float32).view(M, k)
+        v["intermediate"] = ws[off["intermediate"]: off["intermediate"] + so]
+        v["intermediate_scales"] = ws[off["intermediate_scales"]: off["intermediate_scales"] + (n_int - so)]
+        v["scale_rows"] = off["scale_rows"]
+        v["accumulator"] = ws[off["accumulator"]: off["accumulator"] + 4 * M * H].view(torch.float32).view(M, H)
+        return v
+
     def status(self, stream=None):
         return api.read_status(self.ws, stream=stream)
 

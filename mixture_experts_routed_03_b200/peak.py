@@ -1,0 +1,40 @@
+"""ctypes binding of the tensor-core peak probe (``libmoe_peak.so``): the
+dense tcgen05 MMA rate of this GPU per operand kind and tile shape, against
+which the benchmark states its roofline fractions.  A measurement tool, not
+part of the layer."""
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_peak.so")
+KINDS = {"bf16": 0, "fp8": 1, "nvfp4": 2}
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: run python -m mixture_experts_routed_03_b200.build")
+        L = ctypes.CDLL(LIB_PATH)
+        L.moe_peak_mma.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
+                                   ctypes.c_void_p, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_float)]
+        L.moe_peak_mma.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def mma_peak(kind, n=256, pair=False, iters=20000, stream=None):
+    """(TFLOP/s over all SMs, SM cycles per MMA instruction) of back-to-back
+    tcgen05.mma of `kind` ('bf16', 'fp8', 'nvfp4') with N = n, M = 128 per CTA
+    or 256 per CTA pair (pair=True, cta_group::2)."""
+    import torch
+    scratch = torch.zeros(4096, dtype=torch.int32, device="cuda")
+    st = torch.cuda.current_stream().cuda_stream if stream is None else stream
+    tf, cyc = ctypes.c_float(0.0), ctypes.c_float(0.0)
+    rc = lib().moe_peak_mma(KINDS[kind], int(n), int(bool(pair)), int(iters), scratch.data_ptr(), st,
+                            ctypes.byref(tf), ctypes.byref(cyc))
+    if rc != 0:
+        raise RuntimeError(f"moe_peak_mma({kind}, n={n}, pair={pair}) returned {rc}")
+    return float(tf.value), float(cyc.value)

@@ -89,8 +89,11 @@ def route(logits, bias, k):
     order = np.lexsort((ids, -key, nan), axis=-1)
     topk_idx = order[:, :k].astype(np.int64)
     chosen = np.take_along_axis(l32, topk_idx, axis=1).astype(np.float64)
-    z = np.exp(chosen - chosen.max(axis=1, keepdims=True))
-    topk_weights = z / z.sum(axis=1, keepdims=True)
+    # a token with a non-finite chosen logit has no softmax value: its
+    # weights come out NaN here and are unspecified at the boundary
+    with np.errstate(invalid="ignore"):
+        z = np.exp(chosen - chosen.max(axis=1, keepdims=True))
+        topk_weights = z / z.sum(axis=1, keepdims=True)
     return topk_idx, topk_weights
 
 
@@ -217,9 +220,12 @@ def gate_up(fmt, xhat, w13hat, alpha1, I):
 def requant(fmt, h32, G=None):
     """Re-quantise the FP32 intermediate h [rows, I] to the L2 input format.
 
-    Returns dict(codes, scales, hhat) with hhat float64 = the dequantised value
-    the down GEMM sees (for NVFP4 without the global G, which the L2 output
-    scaling carries).
+    Returns dict(codes, scales, hhat, pre, pre_scale): hhat float64 = the
+    dequantised value the down GEMM sees (for NVFP4 without the global G,
+    which the L2 output scaling carries); pre = the FP32 value each element
+    code is rounded from (h itself for BF16, h * inv for FP8 and NVFP4);
+    pre_scale = the FP32 value each NVFP4 block-scale code is rounded from
+    (amax / (6 G)), None otherwise.
 
     nvfp4, per block of 16 along I (all steps FP32, round to nearest):
         sf   = e4m3_satfinite(amax / (6 * G))
@@ -233,7 +239,7 @@ def requant(fmt, h32, G=None):
     rows, I = h32.shape
     if fmt == "bf16":
         codes = F.bf16_encode(h32)
-        return dict(codes=codes, scales=None, hhat=F.bf16_decode(codes))
+        return dict(codes=codes, scales=None, hhat=F.bf16_decode(codes), pre=h32, pre_scale=None)
     if fmt == "fp8":
         blk = h32.reshape(rows, I // 128, 128)
         amax = np.max(np.abs(blk), axis=2)                          # float32
@@ -244,13 +250,14 @@ def requant(fmt, h32, G=None):
         codes = F.e4m3_encode(v)
         codes = np.where((s == 0)[:, :, None], np.uint8(0), codes).reshape(rows, I)
         hhat = F.e4m3_decode(codes).reshape(rows, I // 128, 128) * s[:, :, None].astype(np.float64)
-        return dict(codes=codes, scales=s, hhat=hhat.reshape(rows, I))
+        return dict(codes=codes, scales=s, hhat=hhat.reshape(rows, I), pre=v.reshape(rows, I), pre_scale=None)
     if fmt == "nvfp4":
         G32 = np.float32(G)
         blk = h32.reshape(rows, I // 16, 16)
         amax = np.max(np.abs(blk), axis=2)
         denom = np.float32(np.float32(6.0) * G32)
-        sf_code = F.e4m3_encode((amax / denom).astype(np.float32))
+        sf_pre = (amax / denom).astype(np.float32)
+        sf_code = F.e4m3_encode(sf_pre)
         sf = F.e4m3_decode(sf_code).astype(np.float32)
         sg = (sf * G32).astype(np.float32)
         with np.errstate(divide="ignore"):
@@ -260,7 +267,7 @@ def requant(fmt, h32, G=None):
         q = np.where((sf == 0)[:, :, None], np.uint8(0), q).reshape(rows, I)
         hhat = (F.e2m1_decode(q).reshape(rows, I // 16, 16)
                 * sf[:, :, None].astype(np.float64)).reshape(rows, I)
-        return dict(codes=F.fp4_pack(q), scales=sf_code, hhat=hhat)
+        return dict(codes=F.fp4_pack(q), scales=sf_code, hhat=hhat, pre=v.reshape(rows, I), pre_scale=sf_pre)
     raise ValueError(fmt)
 
 
@@ -338,7 +345,9 @@ def moe_forward(problem, inputs, topk_idx, topk_weights, tokens=None,
                 key = (int(tok[ti[n]]), int(sj[n]))
                 inter[key] = dict(expert=e, h32=h32[n],
                                   codes=rq["codes"][n],
-                                  scales=None if rq["scales"] is None else rq["scales"][n])
+                                  scales=None if rq["scales"] is None else rq["scales"][n],
+                                  pre=rq["pre"][n],
+                                  pre_scale=None if rq["pre_scale"] is None else rq["pre_scale"][n])
     res = dict(out_f64=out, out_bf16=F.bf16_encode(out.astype(np.float32)))
     if keep_intermediate:
         res["intermediate"] = inter

@@ -1,4 +1,5 @@
 """Helpers shared by the GPU parity tests: run the CUDA path through the C ABI
+(the unfused chain or the single moe_fused launch), collect what it computed,
 and compare it with the oracle.  Test code only."""
 
 import numpy as np
@@ -8,7 +9,23 @@ from mixture_experts_routed_03_b200 import api, layer, workloads
 from oracle import formats as F
 from oracle import moe as O
 
+# max|err| bounds of the FFN output, relative to rms(oracle output)
 TOL = {"bf16": 5e-3, "fp8": 2e-2, "nvfp4": 2e-2}
+# An intermediate code may differ from the oracle's only where the oracle's
+# pre-rounding FP32 value lies within this relative distance of the rounding
+# midpoint between the two codes (the kernel's FP32 h differs from the
+# oracle's in its last bits, so a value that close to a midpoint may round
+# either way).
+MID_REL = 1e-4
+# FP8 block scales are FP32 amax / 448 on both sides.
+SCALE_REL = 1e-5
+# A token whose intermediate codes flipped must still be within this multiple
+# of the tolerance of the pure oracle (and within the plain tolerance of the
+# oracle recomputed from the GPU's own codes).
+FLIP_FACTOR = 3.0
+# L2 + combine recomputed by the oracle from the GPU's codes vs the GPU's
+# FP32 accumulator.
+L2_REL = 1e-3
 
 
 def device():
@@ -26,6 +43,11 @@ def make(p, seed, on_gpu_generation=False):
         host = workloads.to_numpy(h)
         d = {k: (None if v is None else v.to(dev)) for k, v in h.items()}
     return d, host
+
+
+def weights_of(d):
+    return {k: d.get(k) for k in ("w13", "w13_scale", "w2", "w2_scale", "gate_up_expert_scales",
+                                  "down_expert_scales", "c_input_scales")}
 
 
 def bf16_to_np(t):
@@ -50,6 +72,42 @@ def close_bf16(a, b, tol_abs):
     return np.abs(a - b) <= tol_abs + bf16_half_ulp(a) + bf16_half_ulp(b)
 
 
+# ------------------------------------------------------------------ code tables
+
+_TABLES = {}
+
+
+def value_table(fmt):
+    """Sorted distinct finite values of a format's codes (-0 merged with +0)."""
+    if fmt not in _TABLES:
+        if fmt == "bf16":
+            v = F.bf16_decode(np.arange(65536, dtype=np.uint32).astype(np.uint16))
+        elif fmt == "e4m3":
+            v = F.e4m3_decode(np.arange(256, dtype=np.uint8))
+        elif fmt == "e2m1":
+            v = F.e2m1_decode(np.arange(16, dtype=np.uint8))
+        else:
+            raise ValueError(fmt)
+        v = np.asarray(v, np.float64)
+        _TABLES[fmt] = np.unique(v[np.isfinite(v)] + 0.0)
+    return _TABLES[fmt]
+
+
+def midpoint_flips(table, got, ref, pre, rel=MID_REL):
+    """For elements whose decoded values differ (got != ref): True where the
+    two values are neighbours in `table` and `pre`, the oracle's value before
+    rounding, lies within `rel` of their midpoint."""
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    lo, hi = np.minimum(got, ref), np.maximum(got, ref)
+    adjacent = np.searchsorted(table, hi) == np.searchsorted(table, lo) + 1
+    mid = 0.5 * (lo + hi)
+    near = np.abs(np.asarray(pre, np.float64) - mid) <= rel * np.abs(mid)
+    return adjacent & near
+
+
+# ------------------------------------------------------------------ GPU results
+
 def row_scale_positions(lay_h, r):
     """Expert e of row r and its padded scale row."""
     starts = lay_h["expert_start_indices"]
@@ -60,40 +118,91 @@ def row_scale_positions(lay_h, r):
     return e, pr
 
 
-def decode_gpu_intermediate(p, inter, scale_off, lay_h, rows):
-    """GPU re-quantised intermediate rows -> (codes, scales-in-oracle-layout, hhat float64)."""
-    fmt, I = p["format"], p["intermediate_hidden"]
-    buf = inter.cpu().numpy()
-    R_total = p["num_tokens"] * p["num_topk"]
-    out = {}
-    if fmt == "bf16":
-        codes = buf[: R_total * I * 2].view(np.uint16).reshape(R_total, I)
-        for r in rows:
-            out[r] = dict(codes=codes[r], scales=None, hhat=F.bf16_decode(codes[r]))
-        return out
-    if fmt == "fp8":
-        codes = buf[: R_total * I].reshape(R_total, I)
-        P = int(lay_h["a_scale_offsets"][p["num_experts"]])
-        ld = (len(buf) - scale_off) // 4 // (I // 128)
-        sc = buf[scale_off: scale_off + (I // 128) * ld * 4].view(np.float32).reshape(I // 128, ld)
-        for r in rows:
-            _, pr = row_scale_positions(lay_h, r)
-            s = sc[:, pr].copy()
-            out[r] = dict(codes=codes[r], scales=s,
-                          hhat=O.dequant_intermediate("fp8", codes[r][None], s[None], I)[0])
-        return out
-    codes = buf[: R_total * I // 2].reshape(R_total, I // 2)
-    kc = I // 64
-    sfb = buf[scale_off:]
-    for r in rows:
-        _, pr = row_scale_positions(lay_h, r)
-        j = np.arange(I // 16)
-        off = ((pr >> 7) * kc + (j >> 2)) * 512 + (pr & 31) * 16 + ((pr >> 5) & 3) * 4 + (j & 3)
-        s = sfb[off].copy()
-        out[r] = dict(codes=codes[r], scales=s,
-                      hhat=O.dequant_intermediate("nvfp4", codes[r][None], s[None], I)[0])
-    return out
+class GpuResult:
+    """What one run of the CUDA path computed: the layout (host arrays), the
+    re-quantised intermediate (codes, then scales at scale_off; FP8 scales
+    [I/128][scale_rows]), the FP32 accumulator (None in staged mode) and the
+    BF16 output; route = (topk_idx, topk_weights) chosen in-kernel, if any."""
 
+    def __init__(self, lay_h, codes, scales, scale_rows, acc, out, route=None):
+        self.lay_h = lay_h
+        self.codes = codes.cpu().numpy() if torch.is_tensor(codes) else codes
+        self.scales = scales.cpu().numpy() if torch.is_tensor(scales) else scales
+        self.scale_rows = int(scale_rows)
+        self.acc = None if acc is None else acc.cpu().numpy()
+        self.out = bf16_to_np(out)
+        self.route = route
+
+    def rows(self, p, rows):
+        """GPU intermediate rows -> {row: dict(values, scales, hhat)}: values =
+        decoded element codes (unscaled), scales = block scales (FP8 float32,
+        NVFP4 E4M3 codes), hhat = dequantised row (float64, the L2 input)."""
+        fmt, I = p["format"], p["intermediate_hidden"]
+        R_total = p["num_tokens"] * p["num_topk"]
+        out = {}
+        if fmt == "bf16":
+            codes = self.codes[: R_total * I * 2].view(np.uint16).reshape(R_total, I)
+            for r in rows:
+                v = F.bf16_decode(codes[r])
+                out[r] = dict(codes=codes[r], values=v, scales=None, hhat=v)
+            return out
+        if fmt == "fp8":
+            codes = self.codes[: R_total * I].reshape(R_total, I)
+            P = self.scale_rows
+            sc = self.scales[: (I // 128) * P * 4].view(np.float32).reshape(I // 128, P)
+            for r in rows:
+                _, pr = row_scale_positions(self.lay_h, r)
+                s = sc[:, pr].copy()
+                out[r] = dict(codes=codes[r], values=F.e4m3_decode(codes[r]), scales=s,
+                              hhat=O.dequant_intermediate("fp8", codes[r][None], s[None], I)[0])
+            return out
+        codes = self.codes[: R_total * I // 2].reshape(R_total, I // 2)
+        kc = I // 64
+        j = np.arange(I // 16)
+        for r in rows:
+            _, pr = row_scale_positions(self.lay_h, r)
+            off = ((pr >> 7) * kc + (j >> 2)) * 512 + (pr & 31) * 16 + ((pr >> 5) & 3) * 4 + (j & 3)
+            s = self.scales[off].copy()
+            out[r] = dict(codes=codes[r], values=F.e2m1_decode(F.fp4_unpack(codes[r][None], I)[0]),
+                          scales=s, hhat=O.dequant_intermediate("nvfp4", codes[r][None], s[None], I)[0])
+        return out
+
+
+def run_chain(L, d, out_mode=api.MOE_OUT_ACCUMULATE):
+    """moe_permute -> moe_ffn (keeping the intermediate) -> moe_combine."""
+    M = d["x"].shape[0]
+    prob = L.problem(M)
+    lay = L.permute(d["topk_idx"])
+    y, inter = L.ffn(d["x"], d.get("x_scale"), lay, d["topk_weights"], out_mode=out_mode, keep_intermediate=True)
+    if out_mode == api.MOE_OUT_ACCUMULATE:
+        out = L.combine(lay, None, y, api.MOE_IN_ACCUMULATED, M)
+    else:
+        out = L.combine(lay, d["topk_weights"], y, api.MOE_IN_STAGED, M)
+    torch.cuda.synchronize()
+    so = api.intermediate_size(prob)[1]
+    P = api.workspace_offsets(prob)["scale_rows"]
+    return GpuResult(lay.host(), inter[:so], inter[so:], P,
+                     y if out_mode == api.MOE_OUT_ACCUMULATE else None, out)
+
+
+def run_fused(L, d, from_logits=False):
+    """moe_fused, then what it left in the workspace."""
+    M = d["x"].shape[0]
+    if from_logits:
+        out = L.forward(d["x"], d.get("x_scale"), logits=d["logits"], bias=d["bias"])
+    else:
+        out = L.forward(d["x"], d.get("x_scale"), topk_idx=d["topk_idx"], topk_weights=d["topk_weights"])
+    torch.cuda.synchronize()
+    v = L.workspace_views(M)
+    lay_h = {k: v[k].cpu().numpy() for k in ("expert_counts", "expert_start_indices", "src_info",
+                                             "slot_to_row", "expert_ids", "num_active", "a_scale_offsets",
+                                             "tile_offsets")}
+    route = (v["topk_idx"].cpu().numpy(), v["topk_weights"].cpu().numpy()) if from_logits else None
+    return GpuResult(lay_h, v["intermediate"], v["intermediate_scales"], v["scale_rows"], v["accumulator"],
+                     out, route=route)
+
+
+# ------------------------------------------------------------------ checks
 
 def check_layout_exact(lay_h, ref, M, k):
     R = int(ref["expert_start_indices"][-1])
@@ -110,77 +219,138 @@ def check_layout_exact(lay_h, ref, M, k):
     assert np.array_equal(lay_h["tile_offsets"][:na + 1], np.concatenate([[0], np.cumsum(tiles)]))
 
 
-def run_unfused(L, d, keep_intermediate=True):
-    """permute -> ffn (accumulate, keeping the intermediate) -> combine."""
-    M = d["x"].shape[0]
-    lay = L.permute(d["topk_idx"])
-    acc, inter = L.ffn(d["x"], d.get("x_scale"), lay, d["topk_weights"], keep_intermediate=keep_intermediate)
-    out = L.combine(lay, None, acc, api.MOE_IN_ACCUMULATED, M)
-    torch.cuda.synchronize()
-    return lay, acc, inter, out
+def check_route(res, host, k):
+    """In-kernel routing: indices bit-exact, weights to 1e-6 relative."""
+    ridx, rw = O.route(host["logits"], host["bias"], k)
+    gidx, gw = res.route
+    assert np.array_equal(gidx, ridx)
+    assert np.all(np.abs(gw.astype(np.float64) - rw) <= 1e-6 * rw + 1e-7)
+    return ridx, rw
 
 
-def check_ffn_against_oracle(p, host, lay_h, acc, inter, out_bf16, tokens, label=""):
-    """Split parity for the tokens in `tokens`:
-      (a) re-quantised codes equal the oracle's except near rounding midpoints,
-      (b) L2 + combine recomputed by the oracle from the GPU's own codes match
-          the GPU's FP32 accumulator to 1e-3 * rms,
-      (c) end to end against the pure oracle within the format's tolerance,
-          tokens that miss it being only ones whose codes flipped.
-    Returns a dict of statistics."""
+def _compare_codes(p, host, e, it, g, stats):
+    """Tier (a) for one routed slot: the GPU's codes against the oracle's.
+    Returns True if any code or scale differs (all at rounding midpoints)."""
+    fmt, I = p["format"], p["intermediate_hidden"]
+    pre = np.asarray(it["pre"], np.float64)
+    ref_vals = None
+    flipped = False
+    if fmt == "bf16":
+        table = value_table("bf16")
+        ref_vals = F.bf16_decode(it["codes"])
+    elif fmt == "fp8":
+        table = value_table("e4m3")
+        s_o = np.asarray(it["scales"], np.float64)
+        s_g = np.asarray(g["scales"], np.float64)
+        assert np.all(np.abs(s_g - s_o) <= SCALE_REL * np.abs(s_o)), \
+            f"FP8 block scales differ: {s_g} vs {s_o}"
+        ref_vals = F.e4m3_decode(it["codes"])
+    else:
+        table = value_table("e2m1")
+        ref_vals = F.e2m1_decode(F.fp4_unpack(np.asarray(it["codes"])[None], I)[0]).astype(np.float64)
+        sv_o = F.e4m3_decode(it["scales"])
+        sv_g = F.e4m3_decode(g["scales"])
+        sdiff = sv_o != sv_g
+        if sdiff.any():
+            ok = midpoint_flips(value_table("e4m3"), sv_g[sdiff], sv_o[sdiff], it["pre_scale"][sdiff])
+            assert ok.all(), f"NVFP4 block scale differs away from a rounding midpoint: " \
+                             f"{sv_g[sdiff][~ok]} vs {sv_o[sdiff][~ok]}"
+            stats["scale_flips"] += int(sdiff.sum())
+            flipped = True
+            # the block's codes are then those of the GPU's scale: re-derive
+            # the oracle's codes for those blocks from its h with that scale
+            G = np.float32(host["c_input_scales"][e])
+            h32 = np.asarray(it["h32"], np.float32).reshape(I // 16, 16)
+            ref_vals = ref_vals.reshape(I // 16, 16).copy()
+            pre = pre.reshape(I // 16, 16).copy()
+            for b in np.nonzero(sdiff)[0]:
+                sg = np.float32(sv_g[b])
+                if sg == 0:
+                    ref_vals[b] = 0.0
+                    pre[b] = 0.0
+                    continue
+                inv = np.float32(1.0) / np.float32(sg * G)
+                v = (h32[b] * inv).astype(np.float32)
+                ref_vals[b] = F.e2m1_decode(F.e2m1_encode(v))
+                pre[b] = v
+            ref_vals = ref_vals.reshape(I)
+            pre = pre.reshape(I)
+    got_vals = np.asarray(g["values"], np.float64)
+    diff = got_vals != ref_vals
+    stats["code_vals"] += diff.size
+    if diff.any():
+        ok = midpoint_flips(table, got_vals[diff], ref_vals[diff], pre[diff])
+        assert ok.all(), (f"{fmt} intermediate codes differ away from a rounding midpoint: GPU "
+                          f"{got_vals[diff][~ok][:8]} oracle {ref_vals[diff][~ok][:8]} "
+                          f"pre-rounding {pre[diff][~ok][:8]}")
+        stats["code_flips"] += int(diff.sum())
+        flipped = True
+    return flipped
+
+
+def oracle_reference(p, host, tokens):
+    """The pure oracle on `tokens`, keeping its intermediate (shareable between checks)."""
+    return O.moe_forward(p, host, host["topk_idx"], host["topk_weights"], tokens=np.asarray(tokens),
+                         keep_intermediate=True)
+
+
+def check_against_oracle(p, host, res, tokens, label="", ref=None):
+    """Split parity of one GPU result for the tokens in `tokens`:
+      (a) every re-quantised intermediate code (and block scale) equals the
+          oracle's, except where the oracle's pre-rounding value lies within
+          MID_REL of the rounding midpoint between the two codes;
+      (b) the oracle's L2 + combine recomputed from the GPU's own codes matches
+          the GPU's FP32 accumulator to L2_REL * rms (when there is one);
+      (c) end to end, |out - oracle| <= TOL * rms + the output's own half-ulp;
+          a token with flipped codes may exceed it only if it meets that bound
+          against the oracle recomputed from the GPU's codes AND stays within
+          FLIP_FACTOR * TOL * rms of the pure oracle.
+    Returns a dict of statistics (flip counts, errors relative to rms)."""
     fmt = p["format"]
     k = p["num_topk"]
-    I = p["intermediate_hidden"]
     tokens = np.asarray(tokens)
-    ref = O.moe_forward(p, host, host["topk_idx"], host["topk_weights"], tokens=tokens,
-                        keep_intermediate=True)
-    so = api.intermediate_size(api.problem_from_dict(p))[1]
-    slot_to_row = lay_h["slot_to_row"]
-    rows = []
-    for t in tokens:
-        for j in range(k):
-            r = int(slot_to_row[t * k + j])
-            if r >= 0:
-                rows.append(r)
-    gi = decode_gpu_intermediate(p, inter, so, lay_h, rows)
+    if ref is None:
+        ref = oracle_reference(p, host, tokens)
+    slot_to_row = res.lay_h["slot_to_row"]
+    rows = [int(slot_to_row[t * k + j]) for t in tokens for j in range(k) if slot_to_row[t * k + j] >= 0]
+    gi = res.rows(p, rows)
 
     # (a) codes
+    stats = dict(code_flips=0, scale_flips=0, code_vals=0)
     flipped_tokens = set()
-    n_vals = n_diff = 0
     for (t, j), it in ref["intermediate"].items():
         r = int(slot_to_row[t * k + j])
-        g = gi[r]
-        hh_o = O.dequant_intermediate(fmt, it["codes"][None], None if it["scales"] is None else it["scales"][None], I)[0]
-        diff = np.abs(g["hhat"] - hh_o)
-        scale = np.max(np.abs(hh_o)) + 1e-30
-        bad = diff > 1e-6 * scale
-        n_vals += bad.size
-        n_diff += int(bad.sum())
-        if bad.any():
+        assert r >= 0
+        if _compare_codes(p, host, it["expert"], it, gi[r], stats):
             flipped_tokens.add(int(t))
-    # (b) L2 + combine from the GPU codes
+    assert stats["code_flips"] <= max(8, 1e-3 * stats["code_vals"]), \
+        f"{label}: {stats['code_flips']} of {stats['code_vals']} intermediate codes differ"
+
+    # (b) L2 + combine from the GPU's codes
     def override(e, ts, js):
         return np.stack([gi[int(slot_to_row[int(a) * k + int(b)])]["hhat"] for a, b in zip(ts, js)])
     ref_g = O.moe_forward(p, host, host["topk_idx"], host["topk_weights"], tokens=tokens,
                           hhat_override=override)
-    acc_h = acc.cpu().numpy()[tokens]
-    r_ref = rms(ref_g["out_f64"])
-    err_b = float(np.max(np.abs(acc_h - ref_g["out_f64"])))
-    assert err_b <= 1e-3 * r_ref, f"{label} L2+combine from GPU codes: {err_b:.3e} > 1e-3*rms {r_ref:.3e}"
-    # (c) end to end: the GPU's BF16 output against the oracle's unrounded
-    # value, within the format's tolerance plus the output's own rounding
-    got = bf16_to_np(out_bf16)[tokens]
+    r_g = rms(ref_g["out_f64"])
+    err_b = None
+    if res.acc is not None:
+        err_b = float(np.max(np.abs(res.acc[tokens] - ref_g["out_f64"])))
+        assert err_b <= L2_REL * r_g, f"{label} L2+combine from GPU codes: {err_b:.3e} > {L2_REL}*rms {r_g:.3e}"
+
+    # (c) end to end
+    got = res.out[tokens]
     exact = ref["out_f64"]
     r = rms(exact)
-    excess = np.abs(got - exact) - bf16_half_ulp(exact)
-    per_tok = np.max(excess, axis=1)
-    over = [int(tokens[i]) for i in np.nonzero(per_tok > TOL[fmt] * r)[0]]
-    unexplained = [t for t in over if t not in flipped_tokens]
-    assert not unexplained, (f"{label} end-to-end error {per_tok.max():.3e} > {TOL[fmt]}*rms {r:.3e} "
-                             f"at tokens {unexplained} without code flips")
-    # the code differences must be rare
-    assert n_diff <= max(8, 1e-3 * n_vals), f"{label} {n_diff} of {n_vals} intermediate codes differ"
-    plain = float(np.max(np.abs(got - F.bf16_decode(ref["out_bf16"]))) / r)
-    return dict(max_err_rel=float(per_tok.max() / r), max_err_vs_bf16_oracle_rel=plain,
-                tokens_over=len(over), code_diffs=n_diff,
-                code_vals=n_vals, l2_err_rel=err_b / r_ref)
+    tol = TOL[fmt] * r
+    per_tok = np.max(np.abs(got - exact) - bf16_half_ulp(exact), axis=1)
+    over = [i for i in np.nonzero(per_tok > tol)[0]]
+    for i in over:
+        t = int(tokens[i])
+        assert t in flipped_tokens, f"{label}: token {t} error {per_tok[i] / r:.3e}*rms > {TOL[fmt]} with no code flip"
+        expl = float(np.max(np.abs(got[i] - ref_g["out_f64"][i]) - bf16_half_ulp(ref_g["out_f64"][i])))
+        assert expl <= TOL[fmt] * r_g, f"{label}: token {t} not explained by its flipped codes ({expl / r_g:.3e}*rms)"
+        assert per_tok[i] <= FLIP_FACTOR * tol, f"{label}: token {t} error {per_tok[i] / r:.3e}*rms > {FLIP_FACTOR}x tol"
+    stats.update(max_err_rel=float(per_tok.max() / r), tokens_over=len(over), tokens_flipped=len(flipped_tokens),
+                 l2_err_rel=None if err_b is None else err_b / r_g,
+                 max_err_vs_bf16_oracle_rel=float(np.max(np.abs(got - F.bf16_decode(ref["out_bf16"]))) / r))
+    return stats

@@ -43,7 +43,10 @@ def test_route_matches_oracle(M, E, k):
         ridx, rw = O.route(logits.numpy(), None if b is None else b.numpy(), k)
         assert np.array_equal(idx.cpu().numpy(), ridx)
         wg = w.cpu().numpy().astype(np.float64)
-        ok = np.isfinite(rw)
+        # weights are specified for tokens whose chosen logits are all finite
+        chosen = np.take_along_axis(logits.numpy(), ridx, axis=1)
+        ok = np.repeat(np.all(np.isfinite(chosen), axis=1, keepdims=True), k, axis=1)
+        assert ok.sum() >= 0.9 * ok.size
         assert np.all(np.abs(wg[ok] - rw[ok]) <= 1e-6 * np.abs(rw[ok]) + 1e-7)
 
 
