@@ -34,11 +34,16 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-DEFAULT_WORKLOAD = "fp8_block"
+DEFAULT_WORKLOAD = "fp8_prefill_routed"
 METRIC = "routed tokens/sec and achieved TFLOPS (% of roofline) per MoE layer, 1 B200"
 FLUSH_BYTES = 512 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FMT_TENSOR_RATIO = {"bf16": 1.0, "fp8": 2.0, "nvfp4": 4.0}   # nominal dense ratio to bf16
+# B200 datasheet dense peaks (the sparse figures halved) and the ~8 TB/s of
+# HBM the layer's roofline is stated against: time = max(FLOPs / tensor peak,
+# bytes / HBM bandwidth)
+SPEC_TFLOPS = {"bf16": 2250.0, "fp8": 4500.0, "nvfp4": 9000.0}
+SPEC_HBM_GBS = 8000.0
 ELEM_BYTES = {"bf16": 2.0, "fp8": 1.0, "nvfp4": 0.5}
 BOUND = {"tiny_bf16": "hbm", "fp8_block": "hbm", "nvfp4_decode": "hbm",
          "nvfp4_prefill": "tensor", "fp8_prefill_routed": "tensor"}
@@ -54,6 +59,8 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-mma-peak", action="store_true",
+                    help="skip the tensor-core peak probe (run after the timed steps)")
     ap.add_argument("--chain", action="store_true",
                     help="time the multi-launch chain moe_route/moe_permute/moe_ffn/moe_combine "
                          "instead of the single moe_fused launch (per-kernel breakdown)")
@@ -235,6 +242,24 @@ def work_model(p, num_active):
     return dict(gemm1=gemm1, gemm2=gemm2, layer=layer)
 
 
+def mma_probe(fmt, achieved_tflops):
+    """The dense tcgen05 rate of this GPU for the format, measured with the
+    peak probe (operands resident in shared memory, back-to-back MMAs on
+    every SM), after the timed steps; context for the roofline fraction."""
+    try:
+        from mixture_experts_routed_03_b200 import peak
+        out = {}
+        for pair in (False, True) if fmt != "nvfp4" else (False,):
+            tf, cyc = peak.mma_peak(fmt, 256, pair, iters=20000)
+            out["cta_pair" if pair else "one_cta"] = {"tflops": tf, "cycles_per_mma": cyc}
+        best = max(v["tflops"] for v in out.values())
+        out["frac_of_best"] = achieved_tflops / best
+        out["shape"] = "M128 (one CTA) / M256 (CTA pair) x N256, K 32 bytes per instruction"
+        return out
+    except Exception as e:  # the probe is context only; the line stands without it
+        return {"error": str(e)}
+
+
 # --------------------------------------------------------------------------- our arm
 
 def run_ours(args, rank, world, local_rank):
@@ -330,6 +355,7 @@ def run_ours(args, rank, world, local_rank):
     api.timing_enable(False, 0)
     L.check_status()
     t_ms = sum(per_step)
+    med_ms = statistics.median(per_step)
     launches = sum(n for _, n in kern.values())
 
     # ---- end to end through the public API, inputs from pinned host memory
@@ -377,7 +403,7 @@ def run_ours(args, rank, world, local_rank):
     # ---- max over ranks
     t_ms, e2e_ms = max_over_ranks([t_ms, e2e_ms], world, dev)
     regime = api.tile_regime(L.problem(M))
-    return dict(p=p, t_ms=t_ms, per_step=per_step, kern=kern, launches=launches, e2e_ms=e2e_ms, phases=phases,
+    return dict(p=p, t_ms=t_ms, med_ms=med_ms, per_step=per_step, kern=kern, launches=launches, e2e_ms=e2e_ms, phases=phases,
                 regime=regime,
                 h2d=h2d, d2h=d2h, num_active=num_active, clocks=clocks.summary(), R=R, M=M,
                 host_inputs=(d, L) if rank == 0 else None)
@@ -473,6 +499,12 @@ def main_ours(args):
         achieved = work["bytes"] / (k_ms / 1e3) / 1e9
         unit = "GB/s"
     total_k = sum(v[0] for v in kern.values()) or 1.0
+    # the layer's roofline as the pages' problem states it: the slower of its
+    # FLOPs at the datasheet dense tensor peak of its format and its bytes at
+    # ~8 TB/s, against the median step
+    lw = wm["layer"]
+    spec_t = max(lw["flops"] / (SPEC_TFLOPS[p["format"]] * 1e12), lw["bytes"] / (SPEC_HBM_GBS * 1e9))
+    med_ms = r["med_ms"]
     line = {
         "metric": METRIC,
         "value": value,
@@ -507,6 +539,14 @@ def main_ours(args):
                                                               "gemm2": "gemm2"}[slot]) if not args.set else None,
                      "peak_source": f"{peak_src} ({'bf16 burst x nominal ' + p['format'] + ' ratio' if bound == 'tensor' else 'hbm copy'})",
                      "kernel_ms": k_ms},
+        "ms_per_step_median": med_ms,
+        "value_median": job_throughput(r["R"], world, 1, med_ms),
+        "roofline_spec": {"time_us": spec_t * 1e6,
+                          "bound": "tensor" if lw["flops"] / (SPEC_TFLOPS[p["format"]] * 1e12) >=
+                                   lw["bytes"] / (SPEC_HBM_GBS * 1e9) else "hbm",
+                          "tensor_peak_tflops": SPEC_TFLOPS[p["format"]], "hbm_gbs": SPEC_HBM_GBS,
+                          "frac": spec_t / (med_ms / 1e3),
+                          "note": "B200 datasheet dense peak of the format and ~8 TB/s; median step"},
         "kernels_ms": {s: v[0] / max(v[1], 1) for s, v in kern.items() if v[1]},
         "fused_phases_us": r["phases"],
         "kernel_share": {s: v[0] / total_k for s, v in kern.items() if v[1]},
@@ -515,6 +555,8 @@ def main_ours(args):
                 "d2h_bytes_per_step": r["d2h"], "ms_per_step": r["e2e_ms"] / args.steps},
         "clocks": r["clocks"],
     }
+    if rank == 0 and bound == "tensor" and not args.no_mma_peak:
+        line["roofline"]["mma_probe"] = mma_probe(p["format"], achieved)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         d, _ = r["host_inputs"]
         line["cpu_baseline"] = cpu_baseline(p, d, args.cpu_seconds)

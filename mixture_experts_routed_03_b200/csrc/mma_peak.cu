@@ -225,6 +225,275 @@ int run_peak(int iters, int* scratch, cudaStream_t st, float* tflops, float* cyc
   return status;
 }
 
+// ---------------------------------------------------------------------------
+// Main-loop probe: the grouped GEMMs' operand feed without their epilogue.
+// Each CTA streams K blocks of A (128 rows x 128 bytes) and B (256 weight
+// rows x 128 bytes, or its 128-row half in a CTA pair) from an L2-resident
+// source by bulk copies into a 4-stage ring, and (mma = 1) issues the E4M3
+// MMAs of each block (M128 x N256 per CTA, or M256 x N256 per pair), or
+// (mma = 0) releases each stage as soon as it lands.  In a pair, the second
+// CTA's stages are relayed to the first CTA's MMA thread by a remote
+// mbarrier arrive, and the MMA's commit releases the stage in both CTAs.
+// ---------------------------------------------------------------------------
+constexpr int kLoopStages = 4;
+
+__device__ __forceinline__ uint32_t mapa_rank0(uint32_t saddr) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, 0;" : "=r"(r) : "r"(saddr));
+  return r;
+}
+
+__device__ __forceinline__ void remote_arrive(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_test_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait; on a time-out sets *status and returns false.
+__device__ __forceinline__ bool probe_wait(uint64_t* bar, uint32_t parity, int* status, bool cluster_scope) {
+  const unsigned long long g0 = globaltimer_ns();
+  while (!(cluster_scope ? mbar_test_cluster(bar, parity) : mbar_test(bar, parity))) {
+    if (*status) return false;
+    if (globaltimer_ns() - g0 > kWaitLimitNs) {
+      *status = MOE_ERR_TIMEOUT;
+      return false;
+    }
+  }
+  return true;
+}
+
+template <bool PAIR, bool MMA>
+__global__ void __launch_bounds__(kPeakThreads, 1)
+    mainloop_probe_kernel(int iters, const uint8_t* src, long long src_blocks, int* out) {
+  constexpr int kA = 16384;
+  constexpr int kB = PAIR ? 16384 : 32768;
+  constexpr int kStage = kA + kB;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base =
+      reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + kLoopStages * kStage);
+  uint64_t* empty = full + kLoopStages;
+  uint64_t* peer_full = empty + kLoopStages;
+  uint64_t* done = peer_full + kLoopStages;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(done + 1);
+  int* status = reinterpret_cast<int*>(tslot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = PAIR ? cluster_rank() : 0;
+  const bool leader = rank == 0;
+  const int unit = PAIR ? (blockIdx.x >> 1) : blockIdx.x;   // CTA or pair index
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kLoopStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+      mbar_init(&peer_full[i], 1);
+    }
+    mbar_init(done, 1);
+    *status = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (MMA && warp == 0) {
+    if (PAIR) {
+      asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tslot)),
+                   "r"(512)
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    } else {
+      tmem_alloc(tslot, 512);
+    }
+  }
+  tc_fence_before();
+  if (PAIR) cluster_sync(); else __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = MMA ? *tslot : 0;
+
+  long long t0 = 0, t1 = 0;
+  if (warp == 0 && lane == 0) {
+    // producer: block (unit, it) of this CTA's half comes from a spread-out,
+    // L2-resident offset
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int it = 0; it < iters; ++it) {
+      if (!probe_wait(&empty[stage], phase ^ 1u, status, false)) break;
+      const long long blk = (static_cast<long long>(unit) * 7919 + it * 13 + rank * 5) % src_blocks;
+      uint8_t* sa = base + stage * kStage;
+      mbar_arrive_expect_tx(&full[stage], kStage);
+      bulk_load(sa, src + blk * 49152, kA, &full[stage]);
+      bulk_load(sa + kA, src + blk * 49152 + kA, kB, &full[stage]);
+      if (++stage == kLoopStages) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    }
+  } else if (warp == 1 && lane == 0 && leader) {
+    // consumer: the MMAs of each stage (or an immediate release)
+    constexpr uint32_t M = PAIR ? 256 : 128;
+    const uint32_t idesc = (idesc_dense(0, 0, 256) & ~(31u << 24)) | ((M >> 4) << 24);
+    int stage = 0;
+    uint32_t phase = 0;
+    t0 = clock64();
+    for (int it = 0; it < iters; ++it) {
+      if (!probe_wait(&full[stage], phase, status, false)) break;
+      if (PAIR && !probe_wait(&peer_full[stage], phase, status, true)) break;
+      tc_fence_after();
+      uint8_t* sa = base + stage * kStage;
+      if (MMA) {
+        const uint64_t adesc = sdesc_sw128(smem_u32(sa));
+        const uint64_t bdesc = sdesc_sw128(smem_u32(sa + kA));
+#pragma unroll
+        for (int kc = 0; kc < 4; ++kc) {
+          if (PAIR) mma_f8_pair(tmem, adesc + 2 * kc, bdesc + 2 * kc, idesc);
+          else mma_f8(tmem, adesc + 2 * kc, bdesc + 2 * kc, idesc, 1u);
+        }
+        if (PAIR) {
+          asm volatile(
+              "{\n\t.reg .b16 m;\n\tmov.b16 m, 3;\n\t"
+              "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], m;\n\t}" ::"r"(
+                  smem_u32(&empty[stage]))
+              : "memory");
+        } else {
+          mma_commit(&empty[stage]);
+        }
+      } else {
+        mbar_arrive(&empty[stage]);
+        if (PAIR) {
+          // the second CTA's stage too
+          uint32_t r;
+          asm volatile("mapa.shared::cluster.u32 %0, %1, 1;" : "=r"(r) : "r"(smem_u32(&empty[stage])));
+          remote_arrive(r);
+        }
+      }
+      if (++stage == kLoopStages) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    }
+    t1 = clock64();
+    if (MMA) {
+      if (PAIR) {
+        asm volatile(
+            "{\n\t.reg .b16 m;\n\tmov.b16 m, 3;\n\t"
+            "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], m;\n\t}" ::"r"(
+                smem_u32(done))
+            : "memory");
+      } else {
+        mma_commit(done);
+      }
+    } else {
+      mbar_arrive(done);
+      if (PAIR) {
+        uint32_t r;
+        asm volatile("mapa.shared::cluster.u32 %0, %1, 1;" : "=r"(r) : "r"(smem_u32(done)));
+        remote_arrive(r);
+      }
+    }
+  } else if (PAIR && !leader && warp == 2 && lane == 0) {
+    // relay: this CTA's landed stages to the first CTA's MMA thread
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int it = 0; it < iters; ++it) {
+      if (!probe_wait(&full[stage], phase, status, false)) break;
+      remote_arrive(mapa_rank0(smem_u32(&peer_full[stage])));
+      if (++stage == kLoopStages) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    }
+  }
+  // everyone: the last stage consumed (bounded)
+  if (threadIdx.x == 64) probe_wait(done, 0, status, PAIR);
+  __syncthreads();
+  if (threadIdx.x == 32 && leader) {
+    out[4 * blockIdx.x + 0] = *status;
+    reinterpret_cast<long long*>(out)[2 * blockIdx.x + 1] = t1 - t0;
+  } else if (threadIdx.x == 0 && !leader) {
+    out[4 * blockIdx.x + 0] = *status;
+    reinterpret_cast<long long*>(out)[2 * blockIdx.x + 1] = 0;
+  }
+  tc_fence_before();
+  if (PAIR) cluster_sync(); else __syncthreads();
+  tc_fence_after();
+  if (MMA && warp == 0) {
+    if (PAIR)
+      asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512) : "memory");
+    else
+      tmem_dealloc(tmem, 512);
+  }
+}
+
+template <bool PAIR, bool MMA>
+int run_mainloop(int iters, const uint8_t* src, long long src_bytes, int* scratch, cudaStream_t st,
+                 float* cycles, float* gbs) {
+  auto kern = mainloop_probe_kernel<PAIR, MMA>;
+  constexpr int kStage = 16384 + (PAIR ? 16384 : 32768);
+  const int smem = kLoopStages * kStage + 1024 + 1024;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return 4;
+  int dev = 0, nsm = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  cudaLaunchConfig_t cfg{};
+  cfg.blockDim = dim3(kPeakThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  int grid = nsm;
+  if (PAIR) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cfg.gridDim = dim3(2);
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess || clusters < 1) return 4;
+    grid = 2 * clusters;
+  }
+  cfg.gridDim = dim3(grid);
+  const long long src_blocks = src_bytes / 49152;
+  if (src_blocks < 1) return 1;
+  cudaEvent_t e0, e1;
+  cudaEventCreate(&e0);
+  cudaEventCreate(&e1);
+  if (cudaLaunchKernelEx(&cfg, kern, 64, src, src_blocks, scratch) != cudaSuccess) return 4;
+  cudaEventRecord(e0, st);
+  if (cudaLaunchKernelEx(&cfg, kern, iters, src, src_blocks, scratch) != cudaSuccess) return 4;
+  cudaEventRecord(e1, st);
+  if (cudaEventSynchronize(e1) != cudaSuccess) return 4;
+  float ms = 0.0f;
+  cudaEventElapsedTime(&ms, e0, e1);
+  cudaEventDestroy(e0);
+  cudaEventDestroy(e1);
+  int* host = new int[4 * grid];
+  cudaMemcpy(host, scratch, sizeof(int) * 4 * grid, cudaMemcpyDeviceToHost);
+  int status = 0;
+  double cyc = 0.0;
+  int n = 0;
+  for (int b = 0; b < grid; ++b) {
+    if (host[4 * b]) status = host[4 * b];
+    const long long c = reinterpret_cast<long long*>(host)[2 * b + 1];
+    if (c > 0) {
+      cyc += static_cast<double>(c);
+      ++n;
+    }
+  }
+  delete[] host;
+  *cycles = n ? static_cast<float>(cyc / n / iters) : 0.0f;
+  *gbs = static_cast<float>(static_cast<double>(kStage) * iters * grid / (ms * 1e-3) / 1e9);
+  return status;
+}
+
 }  // namespace
 
 extern "C" int moe_peak_mma(int kind, int n, int pair, int iters, void* scratch, void* stream, float* tflops,
@@ -242,4 +511,19 @@ extern "C" int moe_peak_mma(int kind, int n, int pair, int iters, void* scratch,
   if (kind == 2 && n == 256 && !pair) return run_peak<2, 256, false>(iters, s, st, tflops, cycles);
   if (kind == 2 && n == 128 && !pair) return run_peak<2, 128, false>(iters, s, st, tflops, cycles);
   return 2;
+}
+
+// Main-loop probe (see mainloop_probe_kernel): cycles per K block of the
+// issuing CTA and the aggregate L2 -> shared memory rate.  src: device buffer
+// of src_bytes (>= 48 KB) to stream from; scratch as for moe_peak_mma.
+extern "C" int moe_peak_mainloop(int pair, int mma, int iters, const void* src, long long src_bytes, void* scratch,
+                                 void* stream, float* cycles, float* gbs) {
+  if (!src || !scratch || !cycles || !gbs || iters < 1) return 1;
+  const uint8_t* s8 = static_cast<const uint8_t*>(src);
+  int* sc = static_cast<int*>(scratch);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (pair && mma) return run_mainloop<true, true>(iters, s8, src_bytes, sc, st, cycles, gbs);
+  if (pair && !mma) return run_mainloop<true, false>(iters, s8, src_bytes, sc, st, cycles, gbs);
+  if (!pair && mma) return run_mainloop<false, true>(iters, s8, src_bytes, sc, st, cycles, gbs);
+  return run_mainloop<false, false>(iters, s8, src_bytes, sc, st, cycles, gbs);
 }

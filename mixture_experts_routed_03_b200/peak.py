@@ -38,3 +38,25 @@ def mma_peak(kind, n=256, pair=False, iters=20000, stream=None):
     if rc != 0:
         raise RuntimeError(f"moe_peak_mma({kind}, n={n}, pair={pair}) returned {rc}")
     return float(tf.value), float(cyc.value)
+
+
+def mainloop(pair=False, mma=True, iters=4000, src_bytes=32 << 20, stream=None):
+    """(SM cycles per K block, aggregate GB/s into shared memory) of the
+    grouped GEMMs' operand feed: 4-stage bulk-copy ring of 128-row A and
+    256-row B K blocks (one CTA, or halves in a CTA pair) from a src_bytes
+    source, with (mma=True) or without the E4M3 MMAs of each block."""
+    import torch
+    L = lib()
+    L.moe_peak_mainloop.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_longlong,
+                                    ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(ctypes.c_float),
+                                    ctypes.POINTER(ctypes.c_float)]
+    L.moe_peak_mainloop.restype = ctypes.c_int
+    src = torch.zeros(src_bytes, dtype=torch.uint8, device="cuda")
+    scratch = torch.zeros(4096, dtype=torch.int32, device="cuda")
+    st = torch.cuda.current_stream().cuda_stream if stream is None else stream
+    cyc, gbs = ctypes.c_float(0.0), ctypes.c_float(0.0)
+    rc = L.moe_peak_mainloop(int(bool(pair)), int(bool(mma)), int(iters), src.data_ptr(), src_bytes,
+                             scratch.data_ptr(), st, ctypes.byref(cyc), ctypes.byref(gbs))
+    if rc != 0:
+        raise RuntimeError(f"moe_peak_mainloop(pair={pair}, mma={mma}) returned {rc}")
+    return float(cyc.value), float(gbs.value)
