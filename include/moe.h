@@ -192,6 +192,20 @@ moe_status_t moe_get_workspace_size(const moe_problem_t* problem, size_t* bytes)
  * allocating a workspace and after moe_read_status reported an error. */
 moe_status_t moe_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
 
+/* Test hooks of the failure detection, stored in the workspace header
+ * (EPConfig, fuse_ffn_combine_send: incompatible options raise rather than
+ * degrade silently -- here, a CTA that never arrives must surface as an
+ * error, not as a hang).  wait_limit_us > 0 makes every bounded wait of
+ * later calls on this workspace give up after that many microseconds
+ * instead of 2 s (0 restores the default).  skip_arrival = 1 makes CTA 0 of
+ * the next moe_fused call withhold its arrival at its first grid barrier,
+ * once: the other CTAs' waits run out, the call returns, the status word
+ * reads MOE_ERR_TIMEOUT and the outputs are unspecified.  Nothing faults or
+ * hangs.  moe_workspace_init clears both hooks and the status.  Enqueued on
+ * `stream`. */
+moe_status_t moe_workspace_test_hooks(void* workspace, size_t workspace_bytes, int32_t wait_limit_us,
+                                      int32_t skip_arrival, void* stream);
+
 /* The tile regime (moe_tile_regime_t, MOE_TILE_LARGE_M or MOE_TILE_SMALL_M)
  * the grouped GEMMs of this problem use once MOE_TILE_AUTO is resolved
  * (tile regimes of the pages' prefill and decode batches; host only). */

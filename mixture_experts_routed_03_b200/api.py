@@ -40,6 +40,7 @@ EXPORTS = (
     "moe_route", "moe_permute", "moe_ffn", "moe_get_intermediate_size", "moe_combine",
     "moe_fused", "moe_read_status", "moe_status_string", "moe_timing_enable", "moe_timing_read",
     "moe_permute_noalloc", "moe_get_tile_regime", "moe_get_workspace_offsets",
+    "moe_workspace_test_hooks",
 )
 
 SLOTS = ("route", "permute", "gather", "gemm1", "zero", "gemm2", "finalize", "combine", "fused")
@@ -111,6 +112,7 @@ def lib():
             "moe_init": [ctypes.c_int],
             "moe_get_workspace_size": [P, ctypes.POINTER(sz)],
             "moe_workspace_init": [vp, sz, vp],
+            "moe_workspace_test_hooks": [vp, sz, i32, i32, vp],
             "moe_prepare_weights": [P, ctypes.POINTER(Weights), vp, vp, vp],
             "moe_get_prepared_weights_size": [P, ctypes.POINTER(sz), ctypes.POINTER(sz)],
             "moe_route": [P, vp, vp, vp, vp, vp],
@@ -236,6 +238,12 @@ def intermediate_size(prob):
 
 def workspace_init(ws, nbytes, stream=None):
     _check("moe_workspace_init", lib().moe_workspace_init(_ptr(ws), int(nbytes), _stream(stream)))
+
+
+def workspace_test_hooks(ws, nbytes, wait_limit_us=0, skip_arrival=0, stream=None):
+    """Failure-detection test hooks in the workspace header (see include/moe.h)."""
+    _check("moe_workspace_test_hooks", lib().moe_workspace_test_hooks(_ptr(ws), int(nbytes), int(wait_limit_us),
+                                                                      int(skip_arrival), _stream(stream)))
 
 
 def prepared_weights_size(prob):

@@ -18,14 +18,27 @@ struct WsHeader {
   int status;        // sticky: the first device error code, 0 if none
   int timeout_site;  // where a bounded wait gave up (diagnostics only)
   int grid_bar[2];   // single-launch layer: barrier arrivals, generation
-  int pad[12];
+  int wait_limit_us; // > 0: bounded waits give up after this many microseconds (test hook)
+  int skip_arrival;  // 1: CTA 0 skips its first grid-barrier arrival once (test hook)
+  int pad[10];
   unsigned long long phase_ns[8];  // single-launch layer: %globaltimer after each phase
   int pad2[32];
 };
 static_assert(sizeof(WsHeader) == 256, "the workspace header is 256 bytes");
 
-// A bounded wait gives up after this many nanoseconds of %globaltimer.
+// A bounded wait gives up after this many nanoseconds of %globaltimer,
+// unless the workspace header sets a shorter limit (wait_limit_us, a test
+// hook of the failure detection).
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+constexpr int kWsWaitLimitWord = 4;   // int index of WsHeader::wait_limit_us
+constexpr int kWsSkipArrivalWord = 5; // int index of WsHeader::skip_arrival
+
+// The wait limit of kernels whose `status` points at a workspace header.
+__device__ __forceinline__ unsigned long long wait_limit_ns(const int* status) {
+  if (!status) return kWaitLimitNs;
+  const int us = *reinterpret_cast<const volatile int*>(status + kWsWaitLimitWord);
+  return us > 0 ? static_cast<unsigned long long>(us) * 1000ull : kWaitLimitNs;
+}
 
 __device__ __forceinline__ void record_error(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
@@ -81,8 +94,9 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits for the phase of `bar` with parity `parity` to complete.  Gives up
-// when *abort is raised by another warp or after kWaitLimitNs; on a time-out
-// it raises *abort and records MOE_ERR_TIMEOUT.  Returns false on give-up.
+// when *abort is raised by another warp or after the wait limit (`status`
+// is the workspace header, or null); on a time-out it raises *abort and
+// records MOE_ERR_TIMEOUT.  Returns false on give-up.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           int* status, int site) {
   if (mbar_test(bar, parity)) return true;
@@ -91,7 +105,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (mbar_test(bar, parity)) return true;
     if ((spin & 127u) == 0) {
       if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > wait_limit_ns(status)) {
         *abort = 1;
         if (status) {
           if (atomicCAS(status, 0, MOE_ERR_TIMEOUT) == 0) status[1] = site;

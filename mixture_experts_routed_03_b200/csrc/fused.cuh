@@ -45,6 +45,8 @@ struct FusedArgs {
 };
 
 // Grid-wide barrier for a cooperative launch; returns false after an abort.
+// (Test hook: with the header's skip_arrival set, CTA 0 withholds its
+// arrival once -- clearing the flag -- so the others' wait runs out.)
 __device__ bool grid_barrier(int* gbar, volatile int* abort_flag, int* status) {
   asm volatile("fence.proxy.async.global;" ::: "memory");
   __threadfence();
@@ -53,7 +55,8 @@ __device__ bool grid_barrier(int* gbar, volatile int* abort_flag, int* status) {
     volatile int* gen = gbar + 1;
     const int g = *gen;
     __threadfence();
-    if (atomicAdd(gbar, 1) == static_cast<int>(gridDim.x) - 1) {
+    const bool skip = blockIdx.x == 0 && atomicExch(status + kWsSkipArrivalWord, 0) == 1;
+    if (!skip && atomicAdd(gbar, 1) == static_cast<int>(gridDim.x) - 1) {
       atomicExch(gbar, 0);
       __threadfence();
       atomicAdd(gbar + 1, 1);
@@ -61,7 +64,7 @@ __device__ bool grid_barrier(int* gbar, volatile int* abort_flag, int* status) {
       const unsigned long long t0 = globaltimer_ns();
       while (*gen == g) {
         if (*abort_flag) break;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (globaltimer_ns() - t0 > wait_limit_ns(status)) {
           *abort_flag = 1;
           if (atomicCAS(status, 0, MOE_ERR_TIMEOUT) == 0) status[1] = 100;
           break;

@@ -555,6 +555,11 @@ int* noalloc_counts_ptr() {
 
 __global__ void set_int_kernel(int* p, int v) { *p = v; }
 
+__global__ void set_hooks_kernel(int* hdr, int wait_limit_us, int skip_arrival) {
+  hdr[kWsWaitLimitWord] = wait_limit_us;
+  hdr[kWsSkipArrivalWord] = skip_arrival;
+}
+
 }  // namespace
 
 // =============================================================== C ABI
@@ -635,6 +640,15 @@ moe_status_t moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
   if (!ws || ws_bytes < sizeof(WsHeader)) return MOE_ERR_INVALID_ARG;
   zero_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<float4*>(ws),
                                                                int64_t(sizeof(WsHeader) / 16));
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status_t moe_workspace_test_hooks(void* ws, size_t ws_bytes, int32_t wait_limit_us, int32_t skip_arrival,
+                                      void* stream) {
+  if (!ws || ws_bytes < sizeof(WsHeader) || wait_limit_us < 0 || (skip_arrival != 0 && skip_arrival != 1))
+    return MOE_ERR_INVALID_ARG;
+  set_hooks_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<int*>(ws), wait_limit_us,
+                                                                    skip_arrival);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
