@@ -61,6 +61,9 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-mma-peak", action="store_true",
                     help="skip the tensor-core peak probe (run after the timed steps)")
+    ap.add_argument("--side-workloads", default="fp8_block,nvfp4_prefill,nvfp4_decode",
+                    help="other configurations timed after the main one (one GPU, rank 0), reported "
+                         "under 'workloads'; empty for none")
     ap.add_argument("--chain", action="store_true",
                     help="time the multi-launch chain moe_route/moe_permute/moe_ffn/moe_combine "
                          "instead of the single moe_fused launch (per-kernel breakdown)")
@@ -240,6 +243,62 @@ def work_model(p, num_active):
     gemm2 = dict(flops=2.0 * R * H * I, bytes=w2 + R * (I * eb + h_sc) + M * H * 4)
     layer = dict(flops=6.0 * R * H * I, bytes=w13 + w2 + x + out + (M * E * 4 if p["routing"] == "logits" else 0))
     return dict(gemm1=gemm1, gemm2=gemm2, layer=layer)
+
+
+def side_workload(name, args, dev, peaks):
+    """One more configuration, timed the same way as the main one (moe_fused,
+    L2 flushed before every step, CUDA events on the launching stream), with
+    fewer steps; its line under 'workloads'."""
+    import torch
+    from mixture_experts_routed_03_b200 import api, layer, workloads
+    p = workloads.problem(name)
+    d = workloads.make_inputs(p, seed=args.seed, device=dev)
+    L = layer.MoELayer(p, {k: d.get(k) for k in ("w13", "w13_scale", "w2", "w2_scale", "gate_up_expert_scales",
+                                                 "down_expert_scales", "c_input_scales")}, device=dev)
+    M, k = p["num_tokens"], p["num_topk"]
+    out = torch.empty((M, p["hidden"]), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_rd = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    sink = torch.empty((), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        L.forward(d["x"], d["x_scale"], topk_idx=d["topk_idx"], topk_weights=d["topk_weights"], out=out)
+
+    steps = max(5, min(args.steps, 20))
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    L.check_status()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        flush.fill_(i & 0xFF)
+        torch.sum(flush_rd, dim=0, out=sink)
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    L.check_status()
+    med = statistics.median(a.elapsed_time(b) for a, b in ev)
+    num_active = int(torch.unique(d["topk_idx"][d["topk_idx"] >= 0]).numel())
+    wm = work_model(p, num_active)["layer"]
+    bound = BOUND.get(name, "hbm")
+    if bound == "tensor":
+        achieved, peak, unit = wm["flops"] / (med / 1e3) / 1e12, peaks["bf16_tflops"] * FMT_TENSOR_RATIO[p["format"]], "TFLOP/s"
+    else:
+        achieved, peak, unit = wm["bytes"] / (med / 1e3) / 1e9, peaks["hbm_gbs"], "GB/s"
+    spec_t = max(wm["flops"] / (SPEC_TFLOPS[p["format"]] * 1e12), wm["bytes"] / (SPEC_HBM_GBS * 1e9))
+    res = {"value": M * k / (med / 1e3), "unit": "routed_tokens/s", "ms_per_step_median": med, "steps": steps,
+           "config": {"num_tokens": M, "hidden": p["hidden"], "intermediate_hidden": p["intermediate_hidden"],
+                      "num_experts": p["num_experts"], "num_topk": k, "format": p["format"],
+                      "routing": p["routing"], "active_experts": num_active,
+                      "gemm_tiles": api.tile_regime(L.problem(M))},
+           "roofline": {"kernel": "moe_fused_kernel", "bound": bound, "achieved": achieved, "peak": peak,
+                        "unit": unit, "frac": achieved / peak},
+           "roofline_spec": {"time_us": spec_t * 1e6, "frac": spec_t / (med / 1e3)}}
+    del L, d, out, flush, flush_rd
+    torch.cuda.empty_cache()
+    return res
 
 
 def mma_probe(fmt, achieved_tflops):
@@ -557,6 +616,14 @@ def main_ours(args):
     }
     if rank == 0 and bound == "tensor" and not args.no_mma_peak:
         line["roofline"]["mma_probe"] = mma_probe(p["format"], achieved)
+    if rank == 0 and world == 1 and not args.chain and not args.set and args.side_workloads:
+        dev = torch.device("cuda", local_rank)
+        line["workloads"] = {}
+        for name in [n for n in args.side_workloads.split(",") if n and n != args.workload]:
+            try:
+                line["workloads"][name] = side_workload(name, args, dev, peaks)
+            except Exception as e:  # a side line never takes the main one down
+                line["workloads"][name] = {"error": str(e)}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         d, _ = r["host_inputs"]
         line["cpu_baseline"] = cpu_baseline(p, d, args.cpu_seconds)

@@ -308,7 +308,8 @@ moe_status_t moe_fused(const moe_problem_t* problem, const moe_act_t* act,
  * one block and need no scratch.  The counts are rewritten in full by every
  * call, so nothing has to start at zero; the array keeps the last call's
  * contents.  The first call on each device looks up the array's device
- * address with that device current; make that first call before any stream
+ * address with that device current (again after a cudaDeviceReset, which
+ * gives the device a new context); make that first call before any stream
  * capture.  All calls share the one array: calls that overlap on the GPU
  * (on other streams, or from other host threads) race on it.  No memory is
  * allocated or freed, by this library or any other. */

@@ -84,13 +84,23 @@ __host__ __device__ constexpr int b_block_bytes(int fmt) {
   return kBStage + (fmt == FMT_NVFP4 ? kSFBStage : 0);
 }
 
+// Gate/up interleave of the prepared gate_up tiles: groups of G gate rows
+// followed by the G matching up rows, so that every 2G accumulator columns
+// hold matching gate and up columns (the epilogue threads read 128 columns
+// each, G = 64, in every format).
+__host__ __device__ constexpr int l1_group(int) { return 64; }
+
 // Logical weight row held by row r (0..255) of L1 tile nt: gate and up rows
-// of intermediate columns 128*nt .. 128*nt+127 in 64-row groups.
-__host__ __device__ inline int l1_tile_row(int nt, int r, int I) {
-  const int g = r >> 6, o = r & 63;
-  const int col = 128 * nt + ((g >> 1) << 6) + o;
+// of intermediate columns 128*nt .. 128*nt+127 in groups of G.
+__host__ __device__ inline int l1_tile_row(int nt, int r, int I, int G) {
+  const int g = r / G, o = r % G;
+  const int col = 128 * nt + (g >> 1) * G + o;
   return (g & 1) ? I + col : col;
 }
+
+// Tile row of the gate row of intermediate column c (0..127 within the
+// tile); the matching up row is G rows further.
+__host__ __device__ inline int l1_gate_row(int c, int G) { return (c / G) * 2 * G + c % G; }
 
 template <int FMT, int EPI>
 struct GemmCfg {
@@ -832,7 +842,7 @@ struct PrepArgs {
 };
 
 __device__ __forceinline__ int prep_row(const PrepArgs& a, int nt, int r) {
-  return a.l1 ? l1_tile_row(nt, r, a.N / 2) : nt * kBN + r;
+  return a.l1 ? l1_tile_row(nt, r, a.N / 2, l1_group(a.fmt)) : nt * kBN + r;
 }
 
 __global__ void __launch_bounds__(256) prepare_weights_kernel(PrepArgs a) {

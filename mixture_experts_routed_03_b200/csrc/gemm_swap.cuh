@@ -252,7 +252,7 @@ __device__ __forceinline__ void gemm_phase_swap(const GemmArgs& p, const CUtenso
 #pragma unroll
         for (int i = 0; i < kNT; ++i) acc[i] = 0.0f;
         // the weight block of this warp's rows (warp-uniform)
-        const int wrow = (EPI == EPI_L1) ? l1_tile_row(t.n_tile, wr, p.I) : (t.n_tile * kBN + wr);
+        const int wrow = (EPI == EPI_L1) ? l1_tile_row(t.n_tile, wr, p.I, l1_group(FMT)) : (t.n_tile * kBN + wr);
         const float* sbe = p.sb + (static_cast<size_t>(t.e) * p.sb_nb + (wrow >> 7)) * p.sb_kb;
         // lane i holds routed row i's activation scale of the next K block:
         // from x's scales by token (direct), or the gathered transposed copy
@@ -313,8 +313,9 @@ __device__ __forceinline__ void gemm_phase_swap(const GemmArgs& p, const CUtenso
         for (int i = 0; i < kNT; ++i) stage_rows[wr * Cfg::kSStride + i] = acc[i];
         mbar_arrive(&sbar[0]);
         if (!mbar_wait(&sbar[0], spar, abort_flag, p.status, 27)) break;
+        constexpr int G = l1_group(FMT);
         const int c0 = 4 * lane;                        // intermediate columns c0..c0+3 of the tile
-        const int gate_row0 = (c0 < 64) ? c0 : 64 + c0; // weight rows of gate (c) and up (c + 64)
+        const int gate_row0 = l1_gate_row(c0, G);       // weight rows of gate (c) and up (c + G)
         for (int j = 0; j < 4; ++j) {
           const int tr = ew * 4 + j;                    // routed row of the tile (warp-uniform)
           float h[4];
@@ -322,12 +323,12 @@ __device__ __forceinline__ void gemm_phase_swap(const GemmArgs& p, const CUtenso
 #pragma unroll
             for (int i = 0; i < 4; ++i)
               h[i] = clamped_swiglu<true>(stage_rows[(gate_row0 + i) * Cfg::kSStride + tr],
-                                          stage_rows[(gate_row0 + 64 + i) * Cfg::kSStride + tr], p.clamp);
+                                          stage_rows[(gate_row0 + G + i) * Cfg::kSStride + tr], p.clamp);
           } else {
 #pragma unroll
             for (int i = 0; i < 4; ++i)
               h[i] = clamped_swiglu<false>(stage_rows[(gate_row0 + i) * Cfg::kSStride + tr],
-                                           stage_rows[(gate_row0 + 64 + i) * Cfg::kSStride + tr], p.clamp);
+                                           stage_rows[(gate_row0 + G + i) * Cfg::kSStride + tr], p.clamp);
           }
           const bool row_ok = tr < t.rows;
           uint8_t* hrow = p.h_out + static_cast<size_t>(t.row0 + tr) * p.h_row_bytes;

@@ -494,6 +494,139 @@ int run_mainloop(int iters, const uint8_t* src, long long src_bytes, int* scratc
   return status;
 }
 
+// ---------------------------------------------------------------------------
+// TMEM read probe: WARPS warps (a multiple of 4, each reading the 32 lanes of
+// its quarter) repeatedly load COLS columns of FP32 with tcgen05.ld 32x32b.x16
+// chunks, waiting once per LOADS chunks, and fold them into a register sum.
+// Reports the tensor-memory to register rate of one SM.
+// ---------------------------------------------------------------------------
+template <int WARPS, int LOADS>
+__global__ void __launch_bounds__(WARPS * 32, 1) tmem_read_probe_kernel(int iters, int* out) {
+  __shared__ uint32_t tslot;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp == 0) tmem_alloc(&tslot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tslot;
+  const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+  // each warp of a quarter owns 512 / (WARPS / 4) columns
+  constexpr int kCols = 512 / (WARPS / 4);
+  const uint32_t col0 = (warp >> 2) * kCols;
+  float acc = 0.0f;
+  const long long t0 = clock64();
+  for (int it = 0; it < iters; ++it) {
+    for (int c = 0; c < kCols; c += 16 * LOADS) {
+      uint32_t r[LOADS][16];
+#pragma unroll
+      for (int l = 0; l < LOADS; ++l) {
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+            "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+            : "=r"(r[l][0]), "=r"(r[l][1]), "=r"(r[l][2]), "=r"(r[l][3]), "=r"(r[l][4]), "=r"(r[l][5]),
+              "=r"(r[l][6]), "=r"(r[l][7]), "=r"(r[l][8]), "=r"(r[l][9]), "=r"(r[l][10]), "=r"(r[l][11]),
+              "=r"(r[l][12]), "=r"(r[l][13]), "=r"(r[l][14]), "=r"(r[l][15])
+            : "r"(tmem + lane_off + col0 + c + 16 * l));
+      }
+      asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+      for (int l = 0; l < LOADS; ++l)
+#pragma unroll
+        for (int i = 0; i < 16; ++i) acc += __uint_as_float(r[l][i]);
+    }
+  }
+  const long long t1 = clock64();
+  if (acc == 1234.5f) out[3] = 1;   // keeps the loads
+  if (threadIdx.x == 0) reinterpret_cast<long long*>(out)[0] = t1 - t0;
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+// The same with one tcgen05.ld of WIDTH (32, 64 or 128) columns per wait.
+template <int WARPS, int WIDTH>
+__global__ void __launch_bounds__(WARPS * 32, 1) tmem_read_wide_kernel(int iters, int* out) {
+  __shared__ uint32_t tslot;
+  const int warp = threadIdx.x >> 5;
+  if (warp == 0) tmem_alloc(&tslot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tslot;
+  const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+  constexpr int kCols = 512 / (WARPS / 4);
+  const uint32_t col0 = (warp >> 2) * kCols;
+  float acc = 0.0f;
+  const long long t0 = clock64();
+  for (int it = 0; it < iters; ++it) {
+    for (int c = 0; c < kCols; c += WIDTH) {
+      uint32_t r[WIDTH];
+      if constexpr (WIDTH == 32) {
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+            "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+            "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+            : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+              "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+              "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+              "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+              "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+            : "r"(tmem + lane_off + col0 + c));
+      } else {
+#pragma unroll
+        for (int h = 0; h < WIDTH / 32; ++h)
+          asm volatile(
+              "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+              "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+              "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+              : "=r"(r[32 * h + 0]), "=r"(r[32 * h + 1]), "=r"(r[32 * h + 2]), "=r"(r[32 * h + 3]),
+                "=r"(r[32 * h + 4]), "=r"(r[32 * h + 5]), "=r"(r[32 * h + 6]), "=r"(r[32 * h + 7]),
+                "=r"(r[32 * h + 8]), "=r"(r[32 * h + 9]), "=r"(r[32 * h + 10]), "=r"(r[32 * h + 11]),
+                "=r"(r[32 * h + 12]), "=r"(r[32 * h + 13]), "=r"(r[32 * h + 14]), "=r"(r[32 * h + 15]),
+                "=r"(r[32 * h + 16]), "=r"(r[32 * h + 17]), "=r"(r[32 * h + 18]), "=r"(r[32 * h + 19]),
+                "=r"(r[32 * h + 20]), "=r"(r[32 * h + 21]), "=r"(r[32 * h + 22]), "=r"(r[32 * h + 23]),
+                "=r"(r[32 * h + 24]), "=r"(r[32 * h + 25]), "=r"(r[32 * h + 26]), "=r"(r[32 * h + 27]),
+                "=r"(r[32 * h + 28]), "=r"(r[32 * h + 29]), "=r"(r[32 * h + 30]), "=r"(r[32 * h + 31])
+              : "r"(tmem + lane_off + col0 + c + 32 * h));
+      }
+      asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+      for (int i = 0; i < WIDTH; i += 2) acc += __uint_as_float(r[i]) * __uint_as_float(r[i + 1]);
+    }
+  }
+  const long long t1 = clock64();
+  if (acc == 1234.5f) out[3] = 1;
+  if (threadIdx.x == 0) reinterpret_cast<long long*>(out)[0] = t1 - t0;
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+template <int WARPS, int WIDTH>
+int run_tmem_wide(int iters, int* scratch, cudaStream_t st, float* bytes_per_cycle) {
+  tmem_read_wide_kernel<WARPS, WIDTH><<<1, WARPS * 32, 0, st>>>(iters, scratch);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return 4;
+  long long cyc = 0;
+  cudaMemcpy(&cyc, scratch, sizeof(cyc), cudaMemcpyDeviceToHost);
+  const double bytes = static_cast<double>(iters) * 128.0 * 512.0 * 4.0;
+  *bytes_per_cycle = cyc > 0 ? static_cast<float>(bytes / cyc) : 0.0f;
+  return 0;
+}
+
+template <int WARPS, int LOADS>
+int run_tmem_read(int iters, int* scratch, cudaStream_t st, float* bytes_per_cycle) {
+  tmem_read_probe_kernel<WARPS, LOADS><<<1, WARPS * 32, 0, st>>>(iters, scratch);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return 4;
+  long long cyc = 0;
+  cudaMemcpy(&cyc, scratch, sizeof(cyc), cudaMemcpyDeviceToHost);
+  // every warp reads 32 lanes x 4 bytes x its columns per iteration
+  const double bytes = static_cast<double>(iters) * 128.0 * 512.0 * 4.0;
+  *bytes_per_cycle = cyc > 0 ? static_cast<float>(bytes / cyc) : 0.0f;
+  return 0;
+}
+
 }  // namespace
 
 extern "C" int moe_peak_mma(int kind, int n, int pair, int iters, void* scratch, void* stream, float* tflops,
@@ -526,4 +659,28 @@ extern "C" int moe_peak_mainloop(int pair, int mma, int iters, const void* src, 
   if (pair && !mma) return run_mainloop<true, false>(iters, s8, src_bytes, sc, st, cycles, gbs);
   if (!pair && mma) return run_mainloop<false, true>(iters, s8, src_bytes, sc, st, cycles, gbs);
   return run_mainloop<false, false>(iters, s8, src_bytes, sc, st, cycles, gbs);
+}
+
+// TMEM read probe (see tmem_read_probe_kernel): bytes per SM cycle from
+// tensor memory to registers with `warps` warps (4, 8 or 16) and `loads`
+// 16-column loads in flight per wait (1, 2 or 4).
+extern "C" int moe_peak_tmem_read(int warps, int loads, int iters, void* scratch, void* stream, float* bytes_per_cycle) {
+  if (!scratch || !bytes_per_cycle || iters < 1) return 1;
+  int* s = static_cast<int*>(scratch);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (warps == 4 && loads == 1) return run_tmem_read<4, 1>(iters, s, st, bytes_per_cycle);
+  if (warps == 4 && loads == 4) return run_tmem_read<4, 4>(iters, s, st, bytes_per_cycle);
+  if (warps == 8 && loads == 1) return run_tmem_read<8, 1>(iters, s, st, bytes_per_cycle);
+  if (warps == 8 && loads == 2) return run_tmem_read<8, 2>(iters, s, st, bytes_per_cycle);
+  if (warps == 8 && loads == 4) return run_tmem_read<8, 4>(iters, s, st, bytes_per_cycle);
+  if (warps == 16 && loads == 1) return run_tmem_read<16, 1>(iters, s, st, bytes_per_cycle);
+  if (warps == 16 && loads == 2) return run_tmem_read<16, 2>(iters, s, st, bytes_per_cycle);
+  if (warps == 16 && loads == 4) return run_tmem_read<16, 4>(iters, s, st, bytes_per_cycle);
+  // loads >= 32: one load of that many columns per wait
+  if (warps == 4 && loads == 32) return run_tmem_wide<4, 32>(iters, s, st, bytes_per_cycle);
+  if (warps == 4 && loads == 64) return run_tmem_wide<4, 64>(iters, s, st, bytes_per_cycle);
+  if (warps == 8 && loads == 32) return run_tmem_wide<8, 32>(iters, s, st, bytes_per_cycle);
+  if (warps == 8 && loads == 64) return run_tmem_wide<8, 64>(iters, s, st, bytes_per_cycle);
+  if (warps == 16 && loads == 32) return run_tmem_wide<16, 32>(iters, s, st, bytes_per_cycle);
+  return 2;
 }

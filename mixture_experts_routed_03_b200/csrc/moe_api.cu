@@ -382,10 +382,14 @@ moe_status_t plan_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_we
   g.expert_ids = b.expert_ids;
   g.num_active = b.num_active;
   g.tiles32 = pl.swap ? b.tiles32 : nullptr;
-  // the small-M gate_up copies its routed rows straight from x
-  g.skip_rows = pl.swap ? 1 : 0;
+  // the small-M gate_up copies its routed rows straight from x: no gathered
+  // copy (a large-M tile's 128 rows per K block arrive faster as one tiled
+  // copy of gathered rows than as 32 four-row gathers from x)
+  const bool direct_l1 = pl.swap;
+  g.skip_rows = direct_l1 ? 1 : 0;
 
-  // L1: gate_up
+  // L1: gate_up (its A map, over the gathered rows, is unused by the
+  // small-M tiles, which copy x rows themselves)
   if (!make_map(&pl.ta1, b.x_perm, x_row_bytes(fmt, H), uint64_t(R), uint32_t(tile_rows))) return MOE_ERR_CUDA;
   GemmArgs& a = pl.l1;
   a = GemmArgs{};
@@ -404,7 +408,7 @@ moe_status_t plan_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_we
   a.a_scale_offsets = b.a_scale_offsets;
   a.tile_offsets = pl.swap ? b.tiles32 : b.tile_offsets;
   a.tile_rows = tile_rows;
-  if (pl.swap) {
+  if (direct_l1) {
     a.x_rows = static_cast<const uint8_t*>(act->x);
     a.x_row_bytes = x_row_bytes(fmt, H);
     a.x_sc = static_cast<const float*>(act->x_scale);   // FP8; null for BF16
@@ -469,7 +473,7 @@ moe_status_t run_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_wei
   FfnPlan pl;
   moe_status_t s = plan_ffn(p, act, w, b, topk_weights, out, pl);
   if (s != MOE_OK) return s;
-  {
+  if (!pl.g.skip_rows || pl.g.tiles32) {
     TimScope ts(MOE_SLOT_GATHER, st);
     if (launch_k(gather_kernel, grid_for(R * 32, 256, 1 << 30), 256, 0, st, pl.g) != cudaSuccess)
       return MOE_ERR_CUDA;
@@ -537,18 +541,43 @@ bool layout_ok(const moe_layout_t* l) {
 constexpr int kNoAllocCountEntries = 32768;   // 128 KB
 static __device__ __align__(256) int g_noalloc_counts[kNoAllocCountEntries];
 
-// Device address of g_noalloc_counts per device, looked up once per device
-// with that device current (host code cannot use the symbol itself).
+// Device address of g_noalloc_counts per device, looked up with that device
+// current (host code cannot use the symbol itself): once per device and
+// primary context -- a cudaDeviceReset gives the device a new context, in
+// which the array has a new address, so the lookup is repeated then.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+CtxGetCurrentFn get_ctx_fn() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(ptr);
+  });
+  return fn;
+}
+
 int* noalloc_counts_ptr() {
   static int* ptrs[64] = {nullptr};
+  static CUcontext ctxs[64] = {nullptr};
   static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  CtxGetCurrentFn get_ctx = get_ctx_fn();
+  CUcontext ctx = nullptr;
+  if (!get_ctx || get_ctx(&ctx) != CUDA_SUCCESS) return nullptr;
   std::lock_guard<std::mutex> lk(mu);
-  if (!ptrs[dev]) {
+  if (!ptrs[dev] || !ctx || ctxs[dev] != ctx) {
+    // (the lookup also makes the device's context current if no runtime
+    // call of this thread has yet)
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_counts) != cudaSuccess) return nullptr;
+    if (get_ctx(&ctx) != CUDA_SUCCESS) return nullptr;
     ptrs[dev] = static_cast<int*>(p);
+    ctxs[dev] = ctx;
   }
   return ptrs[dev];
 }
@@ -831,6 +860,7 @@ moe_status_t moe_fused(const moe_problem_t* p, const moe_act_t* act, const moe_w
   // GEMMs read the routed rows of x themselves there is no gather phase
   const bool small_m = small_m_tiles(p);
   if (small_m) o.tiles32 = reinterpret_cast<int*>(base + L.tiles32);
+  // no gather phase when the gate_up GEMM reads x itself (small-M tiles)
   f.gather_phase = small_m ? 0 : 1;
   f.perm = perm_args(p, idx, o, reinterpret_cast<int*>(base + L.block_counts), L.nblk, status);
   f.perm_small = perm_small_case(f.perm.R, f.perm.E) ? 1 : 0;

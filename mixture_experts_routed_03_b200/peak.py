@@ -60,3 +60,20 @@ def mainloop(pair=False, mma=True, iters=4000, src_bytes=32 << 20, stream=None):
     if rc != 0:
         raise RuntimeError(f"moe_peak_mainloop(pair={pair}, mma={mma}) returned {rc}")
     return float(cyc.value), float(gbs.value)
+
+
+def tmem_read(warps=8, loads=1, iters=2000):
+    """Bytes per SM cycle from tensor memory to registers (one CTA, `warps`
+    warps, `loads` 16-column tcgen05.ld in flight per wait)."""
+    import torch
+    L = lib()
+    L.moe_peak_tmem_read.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+                                     ctypes.POINTER(ctypes.c_float)]
+    L.moe_peak_tmem_read.restype = ctypes.c_int
+    scratch = torch.zeros(64, dtype=torch.int32, device="cuda")
+    bpc = ctypes.c_float(0.0)
+    rc = L.moe_peak_tmem_read(int(warps), int(loads), int(iters), scratch.data_ptr(),
+                              torch.cuda.current_stream().cuda_stream, ctypes.byref(bpc))
+    if rc != 0:
+        raise RuntimeError(f"moe_peak_tmem_read returned {rc}")
+    return float(bpc.value)

@@ -38,6 +38,8 @@ def _routing(M, E, k, seed):
 
 
 @pytest.mark.parametrize("M,E,k", [(4096, 64, 8),    # 32768 slots: uses the static scratch
+                                   (64, 512, 8),     # more than 256 experts, few slots: one chunk, scratch
+                                   (8192, 512, 8),   # 64 chunks x 512 experts: the array's full 32768 entries
                                    (300, 16, 4)])    # one-block path: no scratch needed
 def test_noalloc_permute_matches_permute_twice(M, E, k):
     p, L = _layer(M, E, k)
@@ -68,8 +70,9 @@ def test_noalloc_permute_reports_bad_index_and_rejects_oversize():
     api.permute_noalloc(L.problem(M), idx, got.struct, status)
     torch.cuda.synchronize()
     assert int(status.item()) == api.MOE_ERR_BAD_INDEX
-    # more chunk x expert counts than the static array holds
-    big = api.problem(num_tokens=16384, hidden=256, intermediate_hidden=128, num_experts=512,
+    # more chunk x expert counts than the static array holds: 65 chunks x 512
+    # experts, one chunk past the limit (refused before any launch)
+    big = api.problem(num_tokens=8320, hidden=256, intermediate_hidden=128, num_experts=512,
                       num_topk=8, format="bf16")
     with pytest.raises(api.MoEError) as ei:
         api.permute_noalloc(big, idx, got.struct, status)
