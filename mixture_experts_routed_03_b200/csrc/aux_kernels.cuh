@@ -36,16 +36,17 @@ __device__ __forceinline__ uint64_t route_key(float s, int e) {
   return (static_cast<uint64_t>(ord) << 32) | static_cast<uint32_t>(0xFFFFFFFFu - e);
 }
 
-// Routes token t with the calling (full) warp.
+// Routes token t with the calling (full) warp, from its logits already in
+// registers (lane l holds experts l, l+32, ...) and the bias of those experts.
 template <int PER>
-__device__ __forceinline__ void route_token(const RouteArgs& a, int64_t t, int lane) {
-  const float* row = a.logits + t * a.E;
+__device__ __forceinline__ void route_token(const RouteArgs& a, int64_t t, const float (&lg)[PER],
+                                            const float (&bias)[PER], int lane) {
   uint64_t key[PER];
 #pragma unroll
   for (int i = 0; i < PER; ++i) {
     const int e = lane + 32 * i;
     key[i] = 0;
-    if (e < a.E) key[i] = route_key(__fadd_rn(row[e], a.bias ? a.bias[e] : 0.0f), e);
+    if (e < a.E) key[i] = route_key(__fadd_rn(lg[i], bias[i]), e);
   }
   int my_e = 0;
   for (int j = 0; j < a.k; ++j) {
@@ -69,8 +70,14 @@ __device__ __forceinline__ void route_token(const RouteArgs& a, int64_t t, int l
       if (i == bi && best == m) key[i] = 0;
     if (lane == j) my_e = e;
   }
+  // the unbiased logit of this lane's chosen expert, from the lane that holds it
   const bool mine = lane < a.k;
-  const float l = mine ? row[my_e] : -INFINITY;
+  float l = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const float v = __shfl_sync(0xFFFFFFFFu, lg[i], my_e & 31);
+    if (mine && (my_e >> 5) == i) l = v;
+  }
   float mx = l;
 #pragma unroll
   for (int off = 16; off; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
@@ -84,24 +91,63 @@ __device__ __forceinline__ void route_token(const RouteArgs& a, int64_t t, int l
   }
 }
 
-// Tokens warp_id, warp_id + nwarps, ... (all lanes of the calling warp).
-__device__ __forceinline__ void route_tokens(const RouteArgs& a, int64_t warp_id, int64_t nwarps, int lane) {
-  const int per = (a.E + 31) / 32;
-  for (int64_t t = warp_id; t < a.M; t += nwarps) {
-    if (per <= 1) route_token<1>(a, t, lane);
-    else if (per <= 2) route_token<2>(a, t, lane);
-    else if (per <= 4) route_token<4>(a, t, lane);
-    else if (per <= 8) route_token<8>(a, t, lane);
-    else if (per <= 16) route_token<16>(a, t, lane);
-    else route_token<32>(a, t, lane);
+// Tokens warp_id, warp_id + nwarps, ... (all lanes of the calling warp),
+// with the logits of B tokens loaded before any of them is routed, so their
+// memory latencies overlap.
+template <int PER>
+__device__ __forceinline__ void route_tokens_per(const RouteArgs& a, int64_t warp_id, int64_t nwarps, int lane) {
+  constexpr int B = PER <= 4 ? 4 : (PER <= 8 ? 2 : 1);
+  float bias[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int e = lane + 32 * i;
+    bias[i] = (a.bias && e < a.E) ? a.bias[e] : 0.0f;
+  }
+  for (int64_t t0 = warp_id; t0 < a.M; t0 += nwarps * B) {
+    float lg[B][PER];
+#pragma unroll
+    for (int b = 0; b < B; ++b) {
+      const int64_t t = t0 + b * nwarps;
+#pragma unroll
+      for (int i = 0; i < PER; ++i) {
+        const int e = lane + 32 * i;
+        lg[b][i] = (t < a.M && e < a.E) ? a.logits[t * a.E + e] : 0.0f;
+      }
+    }
+#pragma unroll
+    for (int b = 0; b < B; ++b) {
+      const int64_t t = t0 + b * nwarps;
+      if (t < a.M) route_token<PER>(a, t, lg[b], bias, lane);
+    }
   }
 }
 
+// Experts per lane (32-expert groups) of a routing problem.
+__host__ __device__ inline int route_per(int E) {
+  const int per = (E + 31) / 32;
+  return per <= 1 ? 1 : per <= 2 ? 2 : per <= 4 ? 4 : per <= 8 ? 8 : per <= 16 ? 16 : 32;
+}
+
+__device__ __forceinline__ void route_tokens(const RouteArgs& a, int64_t warp_id, int64_t nwarps, int lane) {
+  switch (route_per(a.E)) {
+    case 1: route_tokens_per<1>(a, warp_id, nwarps, lane); break;
+    case 2: route_tokens_per<2>(a, warp_id, nwarps, lane); break;
+    case 4: route_tokens_per<4>(a, warp_id, nwarps, lane); break;
+    case 8: route_tokens_per<8>(a, warp_id, nwarps, lane); break;
+    case 16: route_tokens_per<16>(a, warp_id, nwarps, lane); break;
+    default: route_tokens_per<32>(a, warp_id, nwarps, lane); break;
+  }
+}
+
+// One kernel per expert-group count, so the register allocation (and the
+// occupancy) is that of the problem's own width.
+template <int PER>
 __global__ void __launch_bounds__(256) route_kernel(RouteArgs a) {
   pdl_trigger();
   pdl_wait();
   const int64_t nw = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-  route_tokens(a, (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5, nw, threadIdx.x & 31);
+  route_tokens_per<PER>(a, (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5, nw,
+                        threadIdx.x & 31);
 }
 
 // ---------------------------------------------------------------------------
@@ -287,10 +333,11 @@ __device__ void perm_scatter_chunk(const PermArgs& a, int c, int* sm) {
   }
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     int tot = 0, before = 0;
+#pragma unroll 8
     for (int b = 0; b < a.nblk; ++b) {
-      const int n = a.block_counts[static_cast<size_t>(b) * E + e];
+      const int n = __ldg(a.block_counts + static_cast<size_t>(b) * E + e);
       tot += n;
-      if (b < c) before += n;
+      before += (b < c) ? n : 0;
     }
     total[e] = tot;
     cursor[e] = before;
@@ -545,16 +592,15 @@ __device__ void small_tile_table(const GatherArgs& g, int lane) {
   if (lane == 31) g.tiles32[na] = incl;
 }
 
-// Token and padded scale row of routed row r.
-__device__ __forceinline__ void gather_locate(const GatherArgs& g, int64_t r, int64_t& t, int& pr) {
-  t = g.src_info[r] / g.topk;
-  // the expert owning row r: starts[e] <= r < starts[e+1]
+// The expert owning row r: the largest e with starts[e] <= r (empty experts
+// before it have smaller ids, those after it start past r).
+__device__ __forceinline__ int gather_expert_of(const GatherArgs& g, int64_t r) {
   int lo = 0, hi = g.E;
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
     if (g.starts[mid] <= r) lo = mid; else hi = mid;
   }
-  pr = g.a_scale_offsets[lo] + static_cast<int>(r - g.starts[lo]);
+  return lo;
 }
 
 // Copies rows r0 and r1 (r1 < 0: none) of x into expert order with all of a
@@ -603,20 +649,58 @@ __device__ __forceinline__ void gather_scales(const GatherArgs& g, int64_t t, in
   }
 }
 
-// Rows warp_id, warp_id + nwarps, ... below the number of valid slots, ROWS
-// rows per step (2 when few warps per SM must keep enough bytes in flight).
-template <int ROWS>
+// The calling warp's contiguous run of rows (an equal share of the valid
+// slots, warp_id-th of nwarps), two rows per step.  Consecutive rows share
+// their expert, so its search runs once per run and the expert then only
+// advances; each row's token comes from src_info.
 __device__ __forceinline__ void gather_rows(const GatherArgs& g, int64_t warp_id, int64_t nwarps, int lane) {
   const int64_t valid = g.starts[g.E];
-  for (int64_t r0 = warp_id; r0 < valid; r0 += ROWS * nwarps) {
-    const int64_t r1 = (ROWS == 2 && r0 + nwarps < valid) ? r0 + nwarps : -1;
-    int64_t t0, t1 = 0;
-    int p0, p1 = 0;
-    gather_locate(g, r0, t0, p0);
-    if (r1 >= 0) gather_locate(g, r1, t1, p1);
+  const int64_t per = (valid + nwarps - 1) / nwarps;
+  const int64_t rb = warp_id * per;
+  const int64_t re = min(valid, rb + per);
+  if (rb >= re) return;
+  int e = gather_expert_of(g, rb);
+  int64_t e_end = g.starts[e + 1];
+  int64_t sbase = g.a_scale_offsets[e] - g.starts[e];   // padded scale row = sbase + r
+  for (int64_t r0 = rb; r0 < re; r0 += 2) {
+    const int64_t r1 = (r0 + 1 < re) ? r0 + 1 : -1;
+    while (r0 >= e_end) {
+      ++e;
+      e_end = g.starts[e + 1];
+      sbase = g.a_scale_offsets[e] - g.starts[e];
+    }
+    const int p0 = static_cast<int>(sbase + r0);
+    int p1 = 0;
+    if (r1 >= 0) {
+      while (r1 >= e_end) {
+        ++e;
+        e_end = g.starts[e + 1];
+        sbase = g.a_scale_offsets[e] - g.starts[e];
+      }
+      p1 = static_cast<int>(sbase + r1);
+    }
+    const int64_t t0 = g.src_info[r0] / g.topk;
+    const int64_t t1 = (r1 >= 0) ? g.src_info[r1] / g.topk : 0;
     gather_copy2(g, r0, t0, r1, t1, lane);
-    gather_scales(g, t0, p0, lane);
-    if (r1 >= 0) gather_scales(g, t1, p1, lane);
+    if (g.fmt == 2) {
+      gather_scales(g, t0, p0, lane);
+      if (r1 >= 0) gather_scales(g, t1, p1, lane);
+    }
+  }
+  if (g.fmt == 1) {
+    // FP8 scales, transposed [H/128][padded rows]: lane l takes row r + l of
+    // each 32-row group, so every K block's 32 scales are written as
+    // consecutive padded rows
+    const int kbs = g.H / 128;
+    int le = gather_expert_of(g, rb);
+    for (int64_t r = rb + lane; r - lane < re; r += 32) {
+      if (r < re) {
+        while (r >= g.starts[le + 1]) ++le;
+        const size_t pr = static_cast<size_t>(g.a_scale_offsets[le] + (r - g.starts[le]));
+        const float* xs = static_cast<const float*>(g.x_scale) + static_cast<int64_t>(g.src_info[r] / g.topk) * kbs;
+        for (int kb = 0; kb < kbs; ++kb) g.sa_t[static_cast<size_t>(kb) * g.ld + pr] = __ldg(xs + kb);
+      }
+    }
   }
 }
 
@@ -626,7 +710,7 @@ __global__ void __launch_bounds__(256) gather_kernel(GatherArgs g) {
   if (g.tiles32 && blockIdx.x == 0 && threadIdx.x < 32) small_tile_table(g, threadIdx.x);
   if (g.skip_rows) return;
   const int64_t nw = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-  gather_rows<1>(g, (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5, nw, threadIdx.x & 31);
+  gather_rows(g, (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5, nw, threadIdx.x & 31);
 }
 
 __device__ __forceinline__ void zero_range(float4* __restrict__ p, int64_t n4, int64_t i0, int64_t stride) {

@@ -33,10 +33,13 @@ constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 constexpr int kWsWaitLimitWord = 4;   // int index of WsHeader::wait_limit_us
 constexpr int kWsSkipArrivalWord = 5; // int index of WsHeader::skip_arrival
 
-// The wait limit of kernels whose `status` points at a workspace header.
-__device__ __forceinline__ unsigned long long wait_limit_ns(const int* status) {
-  if (!status) return kWaitLimitNs;
-  const int us = *reinterpret_cast<const volatile int*>(status + kWsWaitLimitWord);
+// The wait limit set in a workspace header (`status` points at it), read
+// once per kernel phase: wait loops use the copy that the phase keeps next to
+// its abort flag in shared memory (see mbar_wait), never a global load.
+__device__ __forceinline__ int wait_limit_us(const int* status) {
+  return status ? *reinterpret_cast<const volatile int*>(status + kWsWaitLimitWord) : 0;
+}
+__device__ __forceinline__ unsigned long long limit_ns_of(int us) {
   return us > 0 ? static_cast<unsigned long long>(us) * 1000ull : kWaitLimitNs;
 }
 
@@ -94,9 +97,11 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits for the phase of `bar` with parity `parity` to complete.  Gives up
-// when *abort is raised by another warp or after the wait limit (`status`
-// is the workspace header, or null); on a time-out it raises *abort and
-// records MOE_ERR_TIMEOUT.  Returns false on give-up.
+// when *abort is raised by another warp or after the wait limit, whose
+// microseconds (0: the default) the caller keeps in abort[1] (the abort flag
+// and the limit are adjacent words of the kernel's shared-memory header); on
+// a time-out it raises *abort and records MOE_ERR_TIMEOUT in `status`.
+// Returns false on give-up.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           int* status, int site) {
   if (mbar_test(bar, parity)) return true;
@@ -105,7 +110,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (mbar_test(bar, parity)) return true;
     if ((spin & 127u) == 0) {
       if (*abort) return false;
-      if (globaltimer_ns() - t0 > wait_limit_ns(status)) {
+      if (globaltimer_ns() - t0 > limit_ns_of(abort[1])) {
         *abort = 1;
         if (status) {
           if (atomicCAS(status, 0, MOE_ERR_TIMEOUT) == 0) status[1] = site;

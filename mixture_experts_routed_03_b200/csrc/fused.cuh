@@ -56,6 +56,7 @@ __device__ bool grid_barrier(int* gbar, volatile int* abort_flag, int* status) {
     const int g = *gen;
     __threadfence();
     const bool skip = blockIdx.x == 0 && atomicExch(status + kWsSkipArrivalWord, 0) == 1;
+    const unsigned long long limit = limit_ns_of(abort_flag[1]);
     if (!skip && atomicAdd(gbar, 1) == static_cast<int>(gridDim.x) - 1) {
       atomicExch(gbar, 0);
       __threadfence();
@@ -64,7 +65,7 @@ __device__ bool grid_barrier(int* gbar, volatile int* abort_flag, int* status) {
       const unsigned long long t0 = globaltimer_ns();
       while (*gen == g) {
         if (*abort_flag) break;
-        if (globaltimer_ns() - t0 > wait_limit_ns(status)) {
+        if (globaltimer_ns() - t0 > limit) {
           *abort_flag = 1;
           if (atomicCAS(status, 0, MOE_ERR_TIMEOUT) == 0) status[1] = 100;
           break;
@@ -127,7 +128,10 @@ __global__ void __launch_bounds__(FusedShape<FMT, SWAP>::kThreads, 1)
                      const __grid_constant__ CUtensorMap tmA2) {
   constexpr int kHdr = FusedShape<FMT, SWAP>::kHeaderBytes;
   SmemHeader* hdr = reinterpret_cast<SmemHeader*>(smem_base_1024());
-  if (threadIdx.x == 0) hdr->abort = 0;
+  if (threadIdx.x == 0) {
+    hdr->abort = 0;
+    hdr->wait_us = wait_limit_us(f.status);
+  }
   if ((threadIdx.x >> 5) == 1) tmem_alloc(&hdr->tmem, kTmemCols);
   tc_fence_before();
   __syncthreads();
@@ -158,7 +162,7 @@ __global__ void __launch_bounds__(FusedShape<FMT, SWAP>::kThreads, 1)
     if (f.gather.tiles32 && blockIdx.x == 0 && threadIdx.x < 32) small_tile_table(f.gather, threadIdx.x);
     if (!f.gather.skip_rows) {
       const GridIdx g = grid_idx();
-      gather_rows<2>(f.gather, g.gw, g.tw, g.lane);
+      gather_rows(f.gather, g.gw, g.tw, g.lane);
     }
     ok = grid_barrier(f.gbar, &hdr->abort, f.status);
   }

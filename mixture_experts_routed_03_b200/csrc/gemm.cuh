@@ -796,10 +796,13 @@ __device__ __forceinline__ void gemm_phase(const GemmArgs& p, const CUtensorMap*
   tc_fence_after();
 }
 
-// Shared-memory header of every kernel that runs GEMM phases.
+// Shared-memory header of every kernel that runs GEMM phases: the TMEM
+// address, the CTA's abort flag and, in the word after it, the bounded
+// waits' limit in microseconds (0: the default; mbar_wait reads it there).
 struct SmemHeader {
   uint32_t tmem;
   int abort;
+  int wait_us;
 };
 
 __device__ __forceinline__ uint8_t* smem_base_1024() {
@@ -814,12 +817,13 @@ __global__ void __launch_bounds__(GemmCfg<FMT, EPI>::kThreads, 1)
   SmemHeader* hdr = reinterpret_cast<SmemHeader*>(base);
   if (threadIdx.x == 0) hdr->abort = 0;
   if ((threadIdx.x >> 5) == 1) tmem_alloc(&hdr->tmem, kTmemCols);
+  pdl_trigger();
+  pdl_wait();   // the layout, activations, accumulator and header come from earlier kernels
+  if (threadIdx.x == 0) hdr->wait_us = wait_limit_us(p.status);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = hdr->tmem;
-  pdl_trigger();
-  pdl_wait();   // the layout, activations and accumulator come from earlier kernels
   gemm_phase<FMT, EPI>(p, &tmA, base + GemmCfg<FMT, EPI>::kHeaderBytes, tmem, &hdr->abort, blockIdx.x,
                        gridDim.x);
   if ((threadIdx.x >> 5) == 1) tmem_dealloc(tmem, kTmemCols);

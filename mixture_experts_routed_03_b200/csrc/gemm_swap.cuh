@@ -385,12 +385,13 @@ __global__ void __launch_bounds__(SwapCfg<FMT, EPI>::kThreads, 1)
   SmemHeader* hdr = reinterpret_cast<SmemHeader*>(base);
   if (threadIdx.x == 0) hdr->abort = 0;
   if ((threadIdx.x >> 5) == 1) tmem_alloc(&hdr->tmem, kTmemCols);
+  pdl_trigger();
+  pdl_wait();   // the layout, tile table, activations, accumulator and header come from earlier kernels
+  if (threadIdx.x == 0) hdr->wait_us = wait_limit_us(p.status);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = hdr->tmem;
-  pdl_trigger();
-  pdl_wait();   // the layout, tile table, activations and accumulator come from earlier kernels
   gemm_phase_swap<FMT, EPI>(p, &tmA, base + SwapCfg<FMT, EPI>::kHeaderBytes, tmem, &hdr->abort, blockIdx.x,
                             gridDim.x);
   if ((threadIdx.x >> 5) == 1) tmem_dealloc(tmem, kTmemCols);

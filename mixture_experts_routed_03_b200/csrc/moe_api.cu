@@ -303,7 +303,15 @@ RouteArgs route_args(const moe_problem_t* p, const float* logits, const float* b
 
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t st) {
   TimScope ts(MOE_SLOT_ROUTE, st);
-  return launch_k(route_kernel, grid_for(a.M * 32, 256, 1 << 30), 256, 0, st, a);
+  const int grid = grid_for(a.M * 32, 256, 1 << 30);
+  switch (route_per(a.E)) {
+    case 1: return launch_k(route_kernel<1>, grid, 256, 0, st, a);
+    case 2: return launch_k(route_kernel<2>, grid, 256, 0, st, a);
+    case 4: return launch_k(route_kernel<4>, grid, 256, 0, st, a);
+    case 8: return launch_k(route_kernel<8>, grid, 256, 0, st, a);
+    case 16: return launch_k(route_kernel<16>, grid, 256, 0, st, a);
+    default: return launch_k(route_kernel<32>, grid, 256, 0, st, a);
+  }
 }
 
 PermArgs perm_args(const moe_problem_t* p, const int64_t* idx, const PermOut& o, int* block_counts, int nblk,
@@ -475,7 +483,8 @@ moe_status_t run_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_wei
   if (s != MOE_OK) return s;
   if (!pl.g.skip_rows || pl.g.tiles32) {
     TimScope ts(MOE_SLOT_GATHER, st);
-    if (launch_k(gather_kernel, grid_for(R * 32, 256, 1 << 30), 256, 0, st, pl.g) != cudaSuccess)
+    // eight 256-thread blocks per SM: each warp copies a run of rows
+    if (launch_k(gather_kernel, grid_for(R * 32, 256, sm_count() * 8), 256, 0, st, pl.g) != cudaSuccess)
       return MOE_ERR_CUDA;
   }
   {
