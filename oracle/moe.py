@@ -151,17 +151,20 @@ def permute(topk_idx, num_experts, scale_block_rows=128):
 # Decoding of activations and expert weights
 # ----------------------------------------------------------------------------
 
-def decode_x(fmt, x, x_scale, H, rows=None):
+def decode_x(fmt, x, x_scale, H, rows=None, row_scale=None):
     """Activations [M, H] -> float64.
 
     fp8: E4M3 codes times the FP32 per-128 block scale of the token.
-    nvfp4: e2m1 codes times the E4M3 per-16 block scale (no global scale; the
-    per-expert L1 output scaling carries it).
+    nvfp4: e2m1 codes times the E4M3 per-16 block scale, times the token's
+    BF16 rowwise scale when the activations were quantised per token
+    (``row_scale``, see quantize_nvfp4_rowwise); the static global scale is
+    carried by the per-expert L1 output scaling instead.
     """
     x = np.asarray(x)
     if rows is not None:
         x = x[rows]
         x_scale = None if x_scale is None else np.asarray(x_scale)[rows]
+        row_scale = None if row_scale is None else np.asarray(row_scale)[rows]
     if fmt == "bf16":
         return F.bf16_decode(x)
     if fmt == "fp8":
@@ -170,8 +173,49 @@ def decode_x(fmt, x, x_scale, H, rows=None):
     if fmt == "nvfp4":
         codes = F.fp4_unpack(x, H)
         s = F.e4m3_decode(x_scale)
-        return F.e2m1_decode(codes) * np.repeat(s, 16, axis=1)
+        v = F.e2m1_decode(codes) * np.repeat(s, 16, axis=1)
+        if row_scale is not None:
+            v = v * F.bf16_decode(np.asarray(row_scale, np.uint16))[:, None]
+        return v
     raise ValueError(fmt)
+
+
+# The largest E4M3 block scale times the largest E2M1 code: a token whose
+# largest magnitude is rowmax is quantised against 2688 / rowmax.
+NVFP4_ROW_RANGE = 448.0 * 6.0
+
+
+def quantize_nvfp4_rowwise(x):
+    """Per-token dynamic NVFP4 quantisation of activations (EPConfig,
+    ``nvfp4_dyn_global_scales``): each token is quantised against its own
+    global scale 2688 / rowmax instead of a static one, and the scale's BF16
+    inverse travels with the token as its rowwise scale, so a row dequantises
+    as e2m1 * block_scale * rowwise_scale.
+
+    x: float activations [M, H] (FP32 values, e.g. decoded BF16).  Per token:
+      rowmax = max |x[t]|;  G = fp32(rowmax / 2688), the dequant multiplier;
+      blocks of 16 then follow the same steps as the intermediate's re-quant
+      (``requant`` with G): sf = e4m3(amax_b / (6 G)), q = e2m1(x / (sf G));
+      rowwise scale = bf16_rn(G).  An all-zero token gives zero codes, scales
+      and rowwise scale.
+    Returns dict(codes uint8 [M, H/2], scales uint8 E4M3 [M, H/16],
+    rowwise uint16 BF16 [M]).
+    """
+    x32 = np.asarray(x, np.float32)
+    M, H = x32.shape
+    codes = np.zeros((M, H // 2), np.uint8)
+    scales = np.zeros((M, H // 16), np.uint8)
+    rowwise = np.zeros(M, np.uint16)
+    for t in range(M):
+        rowmax = np.float32(np.max(np.abs(x32[t]))) if H else np.float32(0)
+        if rowmax == 0:
+            continue
+        G = np.float32(rowmax / np.float32(NVFP4_ROW_RANGE))
+        rq = requant("nvfp4", x32[t:t + 1], G)
+        codes[t] = rq["codes"][0]
+        scales[t] = rq["scales"][0]
+        rowwise[t] = F.bf16_encode(np.array([G], np.float32))[0]
+    return dict(codes=codes, scales=scales, rowwise=rowwise)
 
 
 def decode_weight(fmt, w, w_scale, e, n_rows, k_cols):
@@ -304,7 +348,8 @@ def moe_forward(problem, inputs, topk_idx, topk_weights, tokens=None,
     problem: dict(hidden, intermediate_hidden, num_experts, num_topk,
                   activation_clamp, format)
     inputs:  dict(x, x_scale, w13, w13_scale, w2, w2_scale,
-                  gate_up_expert_scales, down_expert_scales, c_input_scales)
+                  gate_up_expert_scales, down_expert_scales, c_input_scales,
+                  and for NVFP4 quantised per token, x_row_scale: BF16 [M])
     tokens:  optional subset of token indices (every quantity here is per
              token, so a subset is computed exactly as in the full problem).
     hhat_override: optional callable (e, t_array, j_array) -> float64 rows
@@ -325,7 +370,7 @@ def moe_forward(problem, inputs, topk_idx, topk_weights, tokens=None,
     tok = np.arange(idx.shape[0]) if tokens is None else np.asarray(tokens, np.int64)
     idx_t = idx[tok]
     w_t = w[tok]
-    xhat = decode_x(fmt, inputs["x"], inputs.get("x_scale"), H, rows=tok)
+    xhat = decode_x(fmt, inputs["x"], inputs.get("x_scale"), H, rows=tok, row_scale=inputs.get("x_row_scale"))
     out = np.zeros((tok.shape[0], H), np.float64)
     inter = {} if keep_intermediate else None
     for e in range(E):
