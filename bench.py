@@ -46,7 +46,7 @@ SPEC_TFLOPS = {"bf16": 2250.0, "fp8": 4500.0, "nvfp4": 9000.0}
 SPEC_HBM_GBS = 8000.0
 ELEM_BYTES = {"bf16": 2.0, "fp8": 1.0, "nvfp4": 0.5}
 BOUND = {"tiny_bf16": "hbm", "fp8_block": "hbm", "nvfp4_decode": "hbm",
-         "nvfp4_prefill": "tensor", "fp8_prefill_routed": "tensor"}
+         "nvfp4_prefill": "tensor", "fp8_prefill_routed": "tensor", "nvfp4_prefill_rowwise": "tensor"}
 
 
 def parse():
@@ -61,7 +61,7 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-mma-peak", action="store_true",
                     help="skip the tensor-core peak probe (run after the timed steps)")
-    ap.add_argument("--side-workloads", default="fp8_block,nvfp4_prefill,nvfp4_decode",
+    ap.add_argument("--side-workloads", default="fp8_block,nvfp4_prefill,nvfp4_decode,nvfp4_prefill_rowwise",
                     help="other configurations timed after the main one (one GPU, rank 0), reported "
                          "under 'workloads'; empty for none")
     ap.add_argument("--chain", action="store_true",
@@ -262,8 +262,17 @@ def side_workload(name, args, dev, peaks):
     sink = torch.empty((), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
 
-    def step():
-        L.forward(d["x"], d["x_scale"], topk_idx=d["topk_idx"], topk_weights=d["topk_weights"], out=out)
+    if p.get("act") == "bf16":
+        # BF16 activations: the per-token NVFP4 quantiser, then the layer
+        xb = d["x_bf16"].view(torch.bfloat16)
+
+        def step():
+            codes, scales, rowwise = L.quantize_rowwise(xb)
+            L.forward(codes, scales, topk_idx=d["topk_idx"], topk_weights=d["topk_weights"], out=out,
+                      x_rowwise_scale=rowwise)
+    else:
+        def step():
+            L.forward(d["x"], d["x_scale"], topk_idx=d["topk_idx"], topk_weights=d["topk_weights"], out=out)
 
     steps = max(5, min(args.steps, 20))
     for _ in range(3):
@@ -282,7 +291,9 @@ def side_workload(name, args, dev, peaks):
     med = statistics.median(a.elapsed_time(b) for a, b in ev)
     num_active = int(torch.unique(d["topk_idx"][d["topk_idx"] >= 0]).numel())
     wm = work_model(p, num_active)["layer"]
-    bound = BOUND.get(name, "hbm")
+    if p.get("act") == "bf16":   # the step reads BF16 activations instead of NVFP4 ones
+        wm = dict(wm, bytes=wm["bytes"] + M * p["hidden"] * (2.0 - 0.5 - 1.0 / 16))
+    bound = BOUND.get(name, "tensor" if p["format"] == "nvfp4" and M * k > 8 * p["num_experts"] * 64 else "hbm")
     if bound == "tensor":
         achieved, peak, unit = wm["flops"] / (med / 1e3) / 1e12, peaks["bf16_tflops"] * FMT_TENSOR_RATIO[p["format"]], "TFLOP/s"
     else:

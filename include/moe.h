@@ -119,10 +119,15 @@ typedef enum {
   MOE_TILE_SMALL_M = 2
 } moe_tile_regime_t;
 
-/* Activations (device).  x_scale is NULL for BF16. */
+/* Activations (device).  x_scale is NULL for BF16.  x_rowwise_scale is
+ * NULL, or for NVFP4 activations quantised per token (EPConfig,
+ * nvfp4_dyn_global_scales; moe_quantize_nvfp4_rowwise) the BF16 [M] rowwise
+ * scales: row t dequantises as e2m1 * block scale * x_rowwise_scale[t], and
+ * gate_up_expert_scales then carry the weights' global scales alone. */
 typedef struct {
   const void* x;
   const void* x_scale;
+  const void* x_rowwise_scale;
 } moe_act_t;
 
 /* Expert weights (device).  moe_prepare_weights takes them in the logical
@@ -239,6 +244,20 @@ moe_status_t moe_prepare_weights(const moe_problem_t* problem, const moe_weights
  * not finite (+inf, -inf or NaN), since the softmax has no value there. */
 moe_status_t moe_route(const moe_problem_t* problem, const float* logits, const float* bias,
                        int64_t* topk_idx, float* topk_weights, void* stream);
+
+/* Per-token dynamic NVFP4 quantisation of BF16 activations (EPConfig,
+ * nvfp4_dyn_global_scales: each token is quantised against its own global
+ * scale 2688 / rowmax -- 448 * 6, the largest block scale times the largest
+ * e2m1 code -- and the scale's BF16 inverse travels with the token).  Per
+ * token t of x_bf16 [M, H]: rowmax = max |x[t]|, G = rowmax / 2688 (FP32);
+ * per 16 values: scale = e4m3(amax / (6 G)), code = e2m1(x / (scale * G))
+ * (0 where the scale is 0); rowwise_scale[t] = bf16(G).  All steps FP32,
+ * round to nearest even, saturating; an all-zero token gives zeros.
+ * Writes codes uint8 [M, H/2] (element 2i in the low nibble), block_scales
+ * E4M3 [M, H/16] and rowwise_scales BF16 [M] -- the moe_act_t of an NVFP4
+ * problem with x_rowwise_scale set.  Uses problem->num_tokens and ->hidden. */
+moe_status_t moe_quantize_nvfp4_rowwise(const moe_problem_t* problem, const void* x_bf16, void* codes,
+                                        void* block_scales, void* rowwise_scales, void* stream);
 
 /* Expert-contiguous layout of the routed slots (see moe_layout_t).
  * topk_idx int64 [M, k], values in [-1, E).  Out-of-range ids set

@@ -40,7 +40,7 @@ EXPORTS = (
     "moe_route", "moe_permute", "moe_ffn", "moe_get_intermediate_size", "moe_combine",
     "moe_fused", "moe_read_status", "moe_status_string", "moe_timing_enable", "moe_timing_read",
     "moe_permute_noalloc", "moe_get_tile_regime", "moe_get_workspace_offsets",
-    "moe_workspace_test_hooks",
+    "moe_workspace_test_hooks", "moe_quantize_nvfp4_rowwise",
 )
 
 SLOTS = ("route", "permute", "gather", "gemm1", "zero", "gemm2", "finalize", "combine", "fused")
@@ -67,7 +67,7 @@ class Problem(ctypes.Structure):
 
 
 class Act(ctypes.Structure):
-    _fields_ = [("x", ctypes.c_void_p), ("x_scale", ctypes.c_void_p)]
+    _fields_ = [("x", ctypes.c_void_p), ("x_scale", ctypes.c_void_p), ("x_rowwise_scale", ctypes.c_void_p)]
 
 
 class Weights(ctypes.Structure):
@@ -113,6 +113,7 @@ def lib():
             "moe_get_workspace_size": [P, ctypes.POINTER(sz)],
             "moe_workspace_init": [vp, sz, vp],
             "moe_workspace_test_hooks": [vp, sz, i32, i32, vp],
+            "moe_quantize_nvfp4_rowwise": [P, vp, vp, vp, vp, vp],
             "moe_prepare_weights": [P, ctypes.POINTER(Weights), vp, vp, vp],
             "moe_get_prepared_weights_size": [P, ctypes.POINTER(sz), ctypes.POINTER(sz)],
             "moe_route": [P, vp, vp, vp, vp, vp],
@@ -186,8 +187,8 @@ def problem_from_dict(d, num_tokens=None, fast_math=1):
                    d.get("activation_clamp", 10.0), d["format"], fast_math, d.get("tile_regime", "auto"))
 
 
-def act(x, x_scale=None):
-    return Act(_ptr(x), _ptr(x_scale))
+def act(x, x_scale=None, x_rowwise_scale=None):
+    return Act(_ptr(x), _ptr(x_scale), _ptr(x_rowwise_scale))
 
 
 def weights(w13, w13_scale, w2, w2_scale, gate_up_expert_scales=None, down_expert_scales=None,
@@ -261,6 +262,12 @@ def prepare_weights(prob, logical, out_w13, out_w2, stream=None):
 def route(prob, logits, bias, topk_idx, topk_weights, stream=None):
     _check("moe_route", lib().moe_route(ctypes.byref(prob), _ptr(logits), _ptr(bias), _ptr(topk_idx),
                                         _ptr(topk_weights), _stream(stream)))
+
+
+def quantize_nvfp4_rowwise(prob, x_bf16, codes, block_scales, rowwise_scales, stream=None):
+    """Per-token dynamic NVFP4 quantisation of BF16 activations (see include/moe.h)."""
+    _check("moe_quantize_nvfp4_rowwise", lib().moe_quantize_nvfp4_rowwise(
+        ctypes.byref(prob), _ptr(x_bf16), _ptr(codes), _ptr(block_scales), _ptr(rowwise_scales), _stream(stream)))
 
 
 def permute(prob, topk_idx, lay, ws, ws_bytes, stream=None):

@@ -151,6 +151,78 @@ __global__ void __launch_bounds__(256) route_kernel(RouteArgs a) {
 }
 
 // ---------------------------------------------------------------------------
+// Per-token dynamic NVFP4 quantisation of BF16 activations (EPConfig,
+// nvfp4_dyn_global_scales): one warp per token; lane l owns the 16-value
+// blocks l, l+32, ...  Pass 1 finds the token's largest magnitude, pass 2
+// re-reads each block and quantises it against G = rowmax / 2688 with the
+// same FP32 steps as the intermediate's NVFP4 re-quant.
+// ---------------------------------------------------------------------------
+struct QuantRowArgs {
+  const uint16_t* x;     // BF16 [M][H]
+  int64_t M;
+  int H;
+  uint8_t* codes;        // [M][H/2]
+  uint8_t* scales;       // E4M3 [M][H/16]
+  uint16_t* rowwise;     // BF16 [M]
+};
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __uint_as_float(b << 16); }
+
+__global__ void __launch_bounds__(256) quantize_rowwise_kernel(QuantRowArgs a) {
+  pdl_trigger();
+  pdl_wait();
+  const int lane = threadIdx.x & 31;
+  const int64_t nw = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  const int nblk = a.H / 16;
+  for (int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; t < a.M; t += nw) {
+    const uint4* row = reinterpret_cast<const uint4*>(a.x + t * a.H);
+    float rowmax = 0.0f;
+    for (int b = lane; b < nblk; b += 32) {
+      const uint4 u0 = __ldg(row + 2 * b), u1 = __ldg(row + 2 * b + 1);
+      const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        rowmax = fmaxf(rowmax, fmaxf(fabsf(bf16_bits_to_f32(w[i] & 0xFFFFu)), fabsf(bf16_bits_to_f32(w[i] >> 16))));
+    }
+#pragma unroll
+    for (int off = 16; off; off >>= 1) rowmax = fmaxf(rowmax, __shfl_xor_sync(0xFFFFFFFFu, rowmax, off));
+    const float G = __fdiv_rn(rowmax, 2688.0f);
+    const float denom6 = __fmul_rn(6.0f, G);
+    uint32_t* crow = reinterpret_cast<uint32_t*>(a.codes + t * (a.H / 2));
+    for (int b = lane; b < nblk; b += 32) {
+      const uint4 u0 = __ldg(row + 2 * b), u1 = __ldg(row + 2 * b + 1);
+      const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+      float v[16];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        v[2 * i] = bf16_bits_to_f32(w[i] & 0xFFFFu);
+        v[2 * i + 1] = bf16_bits_to_f32(w[i] >> 16);
+      }
+      uint32_t c0 = 0, c1 = 0, sf_code = 0;
+      if (rowmax > 0.0f) {
+        float amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+        sf_code = cvt_e4m3x2(__fdiv_rn(amax, denom6), 0.0f) & 0xFFu;
+        const float sf = e4m3_to_f32(sf_code);
+        if (sf != 0.0f) {
+          const float inv = __frcp_rn(__fmul_rn(sf, G));
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            c0 |= cvt_e2m1x2(__fmul_rn(v[2 * j], inv), __fmul_rn(v[2 * j + 1], inv)) << (8 * j);
+            c1 |= cvt_e2m1x2(__fmul_rn(v[8 + 2 * j], inv), __fmul_rn(v[9 + 2 * j], inv)) << (8 * j);
+          }
+        }
+      }
+      crow[2 * b] = c0;
+      crow[2 * b + 1] = c1;
+      a.scales[t * nblk + b] = static_cast<uint8_t>(sf_code);
+    }
+    if (lane == 0) a.rowwise[t] = rowmax > 0.0f ? static_cast<uint16_t>(pack_bf16x2(G, 0.0f) & 0xFFFFu) : 0;
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Permutation (Struct_mega_ffn_ep_combine_send: expert_start_indices,
 // expert_ids, a_scale_offsets, src_info, num_active_experts): a stable
 // counting sort of the flat slots s = t*k + j by expert.

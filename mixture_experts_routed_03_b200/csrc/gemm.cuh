@@ -157,6 +157,7 @@ struct GemmArgs {
   int sb_nb, sb_kb;
   // NVFP4 per-expert scalars
   const float* alpha;   // gate_up_expert_scales (L1) or down_expert_scales (L2)
+  const uint16_t* x_row_scale;   // NVFP4 L1: BF16 per-token rowwise scales of x, or null
   const float* c_in;    // c_input_scales (L1 re-quant)
   // L1 output: the re-quantised intermediate, expert order
   uint8_t* h_out;
@@ -544,9 +545,11 @@ __device__ __forceinline__ void gemm_phase(const GemmArgs& p, const CUtensorMap*
       const int pr = t.srow0 + row_local;
       // Down leg: the row's flat slot is loaded now and its router weight
       // once the first partial has been taken, so neither load's latency
-      // falls on the epilogue's tail.
+      // falls on the epilogue's tail (and, likewise, the NVFP4 gate_up's
+      // per-token rowwise scale of x).
       const bool gather_wgt = EPI == EPI_L2_ACC && valid;
-      const int s_flat = gather_wgt ? __ldg(p.src_info + r) : 0;
+      const bool row_scaled = EPI == EPI_L1 && FMT == FMT_NVFP4 && p.x_row_scale != nullptr;
+      const int s_flat = (gather_wgt || (row_scaled && valid)) ? __ldg(p.src_info + r) : 0;
       float wgt = 1.0f;
 
       // acc[0..127]: this thread's row, columns 128*half .. 128*half+127 of
@@ -633,7 +636,9 @@ __device__ __forceinline__ void gemm_phase(const GemmArgs& p, const CUtensorMap*
           aphase ^= 1u;
         }
         if (FMT == FMT_NVFP4) {
-          const float alpha = __ldg(p.alpha + t.e);
+          float alpha = __ldg(p.alpha + t.e);
+          if (row_scaled && valid)
+            alpha = __fmul_rn(alpha, __uint_as_float(static_cast<uint32_t>(__ldg(p.x_row_scale + s_flat / p.topk)) << 16));
 #pragma unroll
           for (int i = 0; i < 128; ++i) acc[i] = __fmul_rn(acc[i], alpha);
         }

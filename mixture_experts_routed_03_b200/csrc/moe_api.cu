@@ -432,6 +432,7 @@ moe_status_t plan_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_we
   a.sb_nb = 2 * I / 128;
   a.sb_kb = H / 128;
   a.alpha = w->gate_up_expert_scales;
+  a.x_row_scale = static_cast<const uint16_t*>(act->x_rowwise_scale);
   a.c_in = w->c_input_scales;
   a.h_out = b.h;
   a.h_row_bytes = h_row_bytes(fmt, I);
@@ -449,6 +450,7 @@ moe_status_t plan_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_we
   a2 = a;
   a2.x_rows = nullptr;   // the down leg reads the intermediate through its TMA map
   a2.x_sc = nullptr;
+  a2.x_row_scale = nullptr;
   a2.k_stages = h_row_bytes(fmt, I) / 128;
   a2.n_tiles = H / 256;
   // Output n tiles in groups: a group's slice of the FP32 accumulator
@@ -530,6 +532,8 @@ moe_status_t check_act_weights(const moe_problem_t* p, const moe_act_t* act, con
   if (p->format == MOE_FMT_NVFP4 &&
       (!w->gate_up_expert_scales || !w->down_expert_scales || !w->c_input_scales))
     return MOE_ERR_INVALID_ARG;
+  // rowwise activation scales exist for NVFP4 only
+  if (act->x_rowwise_scale && p->format != MOE_FMT_NVFP4) return MOE_ERR_INVALID_ARG;
   return MOE_OK;
 }
 
@@ -751,6 +755,26 @@ moe_status_t moe_route(const moe_problem_t* p, const float* logits, const float*
   if (!logits || !topk_idx || !topk_weights) return MOE_ERR_INVALID_ARG;
   return launch_route(route_args(p, logits, bias, topk_idx, topk_weights), static_cast<cudaStream_t>(stream)) ==
                  cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
+}
+
+moe_status_t moe_quantize_nvfp4_rowwise(const moe_problem_t* p, const void* x_bf16, void* codes, void* block_scales,
+                                        void* rowwise_scales, void* stream) {
+  moe_status_t s = check_problem(p);
+  if (s != MOE_OK) return s;
+  if (p->num_tokens == 0) return MOE_OK;
+  if (!x_bf16 || !codes || !block_scales || !rowwise_scales || !aligned16(x_bf16) || !aligned16(codes))
+    return MOE_ERR_INVALID_ARG;
+  QuantRowArgs a{};
+  a.x = static_cast<const uint16_t*>(x_bf16);
+  a.M = p->num_tokens;
+  a.H = p->hidden;
+  a.codes = static_cast<uint8_t*>(codes);
+  a.scales = static_cast<uint8_t*>(block_scales);
+  a.rowwise = static_cast<uint16_t*>(rowwise_scales);
+  return launch_k(quantize_rowwise_kernel, grid_for(a.M * 32, 256, sm_count() * 16), 256, 0,
+                  static_cast<cudaStream_t>(stream), a) == cudaSuccess
              ? MOE_OK
              : MOE_ERR_CUDA;
 }

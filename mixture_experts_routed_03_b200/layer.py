@@ -80,14 +80,25 @@ class MoELayer:
         return api.problem_from_dict(self.p, num_tokens=M, fast_math=self.fast_math)
 
     def forward(self, x, x_scale=None, topk_idx=None, topk_weights=None, logits=None, bias=None,
-                out=None, stream=None):
+                out=None, stream=None, x_rowwise_scale=None):
         """moe_fused: the whole layer, BF16 out [M, H]."""
         M = x.shape[0]
         if out is None:
             out = torch.empty((M, self.p["hidden"]), dtype=torch.bfloat16, device=self.device)
-        api.fused(self.problem(M), api.act(x, x_scale), self.weights, out, self.ws, self.ws_bytes,
-                  topk_idx=topk_idx, topk_weights=topk_weights, logits=logits, bias=bias, stream=stream)
+        api.fused(self.problem(M), api.act(x, x_scale, x_rowwise_scale), self.weights, out, self.ws,
+                  self.ws_bytes, topk_idx=topk_idx, topk_weights=topk_weights, logits=logits, bias=bias,
+                  stream=stream)
         return out
+
+    def quantize_rowwise(self, x_bf16, stream=None):
+        """Per-token dynamic NVFP4 quantisation of BF16 activations [M, H]:
+        (codes uint8 [M, H/2], block scales E4M3 [M, H/16], rowwise BF16 [M])."""
+        M, H = x_bf16.shape
+        codes = torch.empty((M, H // 2), dtype=torch.uint8, device=self.device)
+        scales = torch.empty((M, H // 16), dtype=torch.uint8, device=self.device)
+        rowwise = torch.empty((M,), dtype=torch.int16, device=self.device)
+        api.quantize_nvfp4_rowwise(self.problem(M), x_bf16, codes, scales, rowwise, stream=stream)
+        return codes, scales, rowwise
 
     def route(self, logits, bias=None, stream=None):
         M = logits.shape[0]
@@ -104,7 +115,7 @@ class MoELayer:
         return lay
 
     def ffn(self, x, x_scale, lay, topk_weights, out_mode=api.MOE_OUT_ACCUMULATE, keep_intermediate=False,
-            stream=None):
+            stream=None, x_rowwise_scale=None):
         """moe_ffn; returns (out fp32, intermediate bytes or None)."""
         M = x.shape[0]
         prob = self.problem(M)
@@ -115,7 +126,7 @@ class MoELayer:
         if keep_intermediate:
             n, _ = api.intermediate_size(prob)
             inter = torch.empty(n, dtype=torch.uint8, device=self.device)
-        api.ffn(prob, api.act(x, x_scale), self.weights, lay.struct, topk_weights, out_mode, out,
+        api.ffn(prob, api.act(x, x_scale, x_rowwise_scale), self.weights, lay.struct, topk_weights, out_mode, out,
                 self.ws, self.ws_bytes, intermediate=inter, stream=stream)
         return out, inter
 

@@ -18,6 +18,8 @@ activation encodings and FromLogits routing):
   nvfp4_prefill    M=4096  H=7168 I=2048 E=32  k=8  NVFP4, uniform routing
   nvfp4_decode     M=64    H=7168 I=2048 E=256 k=8  NVFP4, Zipf(1.2) routing
   fp8_prefill_routed M=16384 H=4096 I=1536 E=128 k=8 E4M3, routing from logits
+  nvfp4_prefill_rowwise  as nvfp4_prefill, with BF16 activations [M, H]
+                     (x_bf16) for the per-token quantiser
 """
 
 import math
@@ -35,6 +37,11 @@ WORKLOADS = {
                          num_experts=256, num_topk=8, format="nvfp4", routing="zipf"),
     "fp8_prefill_routed": dict(num_tokens=16384, hidden=4096, intermediate_hidden=1536,
                                num_experts=128, num_topk=8, format="fp8", routing="logits"),
+    # the NVFP4 prefill with BF16 activations quantised per token by the
+    # layer (EPConfig nvfp4_dyn_global_scales) instead of arriving quantised
+    "nvfp4_prefill_rowwise": dict(num_tokens=4096, hidden=7168, intermediate_hidden=2048,
+                                  num_experts=32, num_topk=8, format="nvfp4", routing="uniform",
+                                  act="bf16"),
 }
 
 # Typical magnitudes of the drawn values.
@@ -164,6 +171,9 @@ def make_inputs(p, seed=0, device="cpu"):
         d["c_input_scales"] = c_in.to(torch.float32)
     else:
         raise ValueError(fmt)
+    if p.get("act") == "bf16":
+        # raw activations for the per-token quantiser
+        d["x_bf16"] = _bf16_codes((M, H), X_STD, g, device)
     d.update(_routing(p, g, device))
     return d
 

@@ -174,7 +174,8 @@ def run_chain(L, d, out_mode=api.MOE_OUT_ACCUMULATE):
     M = d["x"].shape[0]
     prob = L.problem(M)
     lay = L.permute(d["topk_idx"])
-    y, inter = L.ffn(d["x"], d.get("x_scale"), lay, d["topk_weights"], out_mode=out_mode, keep_intermediate=True)
+    y, inter = L.ffn(d["x"], d.get("x_scale"), lay, d["topk_weights"], out_mode=out_mode, keep_intermediate=True,
+                     x_rowwise_scale=d.get("x_row_scale"))
     if out_mode == api.MOE_OUT_ACCUMULATE:
         out = L.combine(lay, None, y, api.MOE_IN_ACCUMULATED, M)
     else:
@@ -192,7 +193,8 @@ def run_fused(L, d, from_logits=False):
     if from_logits:
         out = L.forward(d["x"], d.get("x_scale"), logits=d["logits"], bias=d["bias"])
     else:
-        out = L.forward(d["x"], d.get("x_scale"), topk_idx=d["topk_idx"], topk_weights=d["topk_weights"])
+        out = L.forward(d["x"], d.get("x_scale"), topk_idx=d["topk_idx"], topk_weights=d["topk_weights"],
+                        x_rowwise_scale=d.get("x_row_scale"))
     torch.cuda.synchronize()
     v = L.workspace_views(M)
     lay_h = {k: v[k].cpu().numpy() for k in ("expert_counts", "expert_start_indices", "src_info",
