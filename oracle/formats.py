@@ -17,6 +17,10 @@ reference by name only):
   per byte, element 2i in the low nibble (reading: the pages do not state
   the nibble order).
 * BF16 -- flashinfer.fused_moe.MoEActivationPack, "BF16: raw bfloat16".
+* UE8M0 -- flashinfer.fused_moe.MoEActivationPack, MXFP8 "token-major uint8
+  [M, H/32] UE8M0 scales"; Struct_mega_ffn_ep_combine_send names the E8M0
+  sibling.  An unsigned power of two: code c is 2**(c - 127), code 255 is
+  NaN (the OCP microscaling scale format).
 
 Encoders round to nearest, ties to even, and saturate to the largest finite
 magnitude ("satfinite"), the reading taken where the pages are silent.
@@ -160,6 +164,17 @@ def fp4_pack(codes):
     """Pack nibble codes [..., n] (n even) into uint8 [..., n/2]; element 2i -> low nibble."""
     c = np.asarray(codes, dtype=np.uint8)
     return (c[..., 0::2] & 0xF) | ((c[..., 1::2] & 0xF) << 4)
+
+
+# ----------------------------------------------------------------------------
+# UE8M0 (MX block scale)
+# ----------------------------------------------------------------------------
+
+def ue8m0_decode(codes):
+    """uint8 UE8M0 codes -> float64: 2**(code - 127); code 255 is NaN."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    v = np.ldexp(1.0, c - 127)
+    return np.where(c == 255, np.nan, v)
 
 
 # ----------------------------------------------------------------------------

@@ -63,7 +63,7 @@ import numpy as np
 
 from . import formats as F
 
-FORMATS = ("bf16", "fp8", "nvfp4")
+FORMATS = ("bf16", "fp8", "nvfp4", "mxfp8")
 
 
 # ----------------------------------------------------------------------------
@@ -155,6 +155,7 @@ def decode_x(fmt, x, x_scale, H, rows=None, row_scale=None):
     """Activations [M, H] -> float64.
 
     fp8: E4M3 codes times the FP32 per-128 block scale of the token.
+    mxfp8: E4M3 codes times the UE8M0 per-32 block scale of the token.
     nvfp4: e2m1 codes times the E4M3 per-16 block scale, times the token's
     BF16 rowwise scale when the activations were quantised per token
     (``row_scale``, see quantize_nvfp4_rowwise); the static global scale is
@@ -170,6 +171,8 @@ def decode_x(fmt, x, x_scale, H, rows=None, row_scale=None):
     if fmt == "fp8":
         s = np.asarray(x_scale, np.float32).astype(np.float64)
         return F.e4m3_decode(x) * np.repeat(s, 128, axis=1)
+    if fmt == "mxfp8":
+        return F.e4m3_decode(x) * np.repeat(F.ue8m0_decode(x_scale), 32, axis=1)
     if fmt == "nvfp4":
         codes = F.fp4_unpack(x, H)
         s = F.e4m3_decode(x_scale)
@@ -221,7 +224,8 @@ def quantize_nvfp4_rowwise(x):
 def decode_weight(fmt, w, w_scale, e, n_rows, k_cols):
     """Expert e's weight [n_rows, k_cols] (K-major, as stored) -> float64.
 
-    fp8 scales are per 128 x 128 block; nvfp4 scales per 1 x 16 block.
+    fp8 scales are per 128 x 128 block; mxfp8 (UE8M0) scales per 1 x 32
+    block; nvfp4 scales per 1 x 16 block.
     """
     if fmt == "bf16":
         return F.bf16_decode(np.asarray(w)[e])
@@ -229,6 +233,8 @@ def decode_weight(fmt, w, w_scale, e, n_rows, k_cols):
         s = np.asarray(w_scale, np.float32)[e].astype(np.float64)
         full = np.repeat(np.repeat(s, 128, axis=0), 128, axis=1)
         return F.e4m3_decode(np.asarray(w)[e]) * full
+    if fmt == "mxfp8":
+        return F.e4m3_decode(np.asarray(w)[e]) * np.repeat(F.ue8m0_decode(np.asarray(w_scale)[e]), 32, axis=1)
     if fmt == "nvfp4":
         codes = F.fp4_unpack(np.asarray(w)[e], k_cols)
         s = F.e4m3_decode(np.asarray(w_scale)[e])
@@ -278,6 +284,12 @@ def requant(fmt, h32, G=None):
         s    = amax / 448
         q    = e4m3_satfinite(h * (1 / s))             (q = 0, s = 0 where amax == 0)
     bf16:  q = bf16_rn(h)
+    mxfp8, per block of 32 along I (the OCP microscaling rule; E8M0 scales
+    carry no per-expert input scale):
+        X    = floor(log2(amax)) - 8, clamped to [-127, 127]  (8: the largest
+               E4M3 exponent; X = -127 where amax == 0)
+        q    = e4m3_satfinite(h * 2**-X)      (exact power-of-two scaling)
+        scale code = X + 127
     """
     h32 = np.asarray(h32, np.float32)
     rows, I = h32.shape
@@ -295,6 +307,18 @@ def requant(fmt, h32, G=None):
         codes = np.where((s == 0)[:, :, None], np.uint8(0), codes).reshape(rows, I)
         hhat = F.e4m3_decode(codes).reshape(rows, I // 128, 128) * s[:, :, None].astype(np.float64)
         return dict(codes=codes, scales=s, hhat=hhat.reshape(rows, I), pre=v.reshape(rows, I), pre_scale=None)
+    if fmt == "mxfp8":
+        blk = h32.reshape(rows, I // 32, 32)
+        amax = np.max(np.abs(blk), axis=2).astype(np.float64)
+        with np.errstate(divide="ignore"):
+            X = np.where(amax > 0, np.floor(np.log2(np.where(amax > 0, amax, 1.0))) - 8, -127)
+        X = np.clip(X, -127, 127).astype(np.int64)
+        v = blk.astype(np.float64) * np.ldexp(1.0, -X)[:, :, None]   # exact
+        codes = F.e4m3_encode(v).reshape(rows, I)
+        sc = (X + 127).astype(np.uint8)
+        hhat = F.e4m3_decode(codes).reshape(rows, I // 32, 32) * F.ue8m0_decode(sc)[:, :, None]
+        return dict(codes=codes, scales=sc, hhat=hhat.reshape(rows, I), pre=v.reshape(rows, I).astype(np.float32),
+                    pre_scale=None)
     if fmt == "nvfp4":
         G32 = np.float32(G)
         blk = h32.reshape(rows, I // 16, 16)
@@ -322,6 +346,8 @@ def dequant_intermediate(fmt, codes, scales, I):
     if fmt == "fp8":
         s = np.asarray(scales, np.float32).astype(np.float64)
         return F.e4m3_decode(codes) * np.repeat(s, 128, axis=1)
+    if fmt == "mxfp8":
+        return F.e4m3_decode(codes) * np.repeat(F.ue8m0_decode(scales), 32, axis=1)
     if fmt == "nvfp4":
         q = F.fp4_unpack(codes, I)
         return F.e2m1_decode(q) * np.repeat(F.e4m3_decode(scales), 16, axis=1)
