@@ -38,15 +38,16 @@ DEFAULT_WORKLOAD = "fp8_prefill_routed"
 METRIC = "routed tokens/sec and achieved TFLOPS (% of roofline) per MoE layer, 1 B200"
 FLUSH_BYTES = 512 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-FMT_TENSOR_RATIO = {"bf16": 1.0, "fp8": 2.0, "nvfp4": 4.0}   # nominal dense ratio to bf16
+FMT_TENSOR_RATIO = {"bf16": 1.0, "fp8": 2.0, "nvfp4": 4.0, "mxfp8": 2.0}   # nominal dense ratio to bf16
 # B200 datasheet dense peaks (the sparse figures halved) and the ~8 TB/s of
 # HBM the layer's roofline is stated against: time = max(FLOPs / tensor peak,
 # bytes / HBM bandwidth)
-SPEC_TFLOPS = {"bf16": 2250.0, "fp8": 4500.0, "nvfp4": 9000.0}
+SPEC_TFLOPS = {"bf16": 2250.0, "fp8": 4500.0, "nvfp4": 9000.0, "mxfp8": 4500.0}
 SPEC_HBM_GBS = 8000.0
-ELEM_BYTES = {"bf16": 2.0, "fp8": 1.0, "nvfp4": 0.5}
+ELEM_BYTES = {"bf16": 2.0, "fp8": 1.0, "nvfp4": 0.5, "mxfp8": 1.0}
 BOUND = {"tiny_bf16": "hbm", "fp8_block": "hbm", "nvfp4_decode": "hbm",
-         "nvfp4_prefill": "tensor", "fp8_prefill_routed": "tensor", "nvfp4_prefill_rowwise": "tensor"}
+         "nvfp4_prefill": "tensor", "fp8_prefill_routed": "tensor", "nvfp4_prefill_rowwise": "tensor",
+         "mxfp8_prefill_routed": "tensor"}
 
 
 def parse():
@@ -61,7 +62,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-mma-peak", action="store_true",
                     help="skip the tensor-core peak probe (run after the timed steps)")
-    ap.add_argument("--side-workloads", default="fp8_block,nvfp4_prefill,nvfp4_decode,nvfp4_prefill_rowwise",
+    ap.add_argument("--side-workloads",
+                    default="fp8_block,nvfp4_prefill,nvfp4_decode,nvfp4_prefill_rowwise,mxfp8_prefill_routed",
                     help="other configurations timed after the main one (one GPU, rank 0), reported "
                          "under 'workloads'; empty for none")
     ap.add_argument("--chain", action="store_true",
@@ -233,6 +235,9 @@ def work_model(p, num_active):
     elif fmt == "nvfp4":
         w13_sc, w2_sc = 2 * I * H // 16, H * I // 16
         x_sc, h_sc = H // 16, I // 16
+    elif fmt == "mxfp8":
+        w13_sc, w2_sc = 2 * I * H // 32, H * I // 32
+        x_sc, h_sc = H // 32, I // 32
     else:
         w13_sc = w2_sc = x_sc = h_sc = 0
     w13 = num_active * (2 * I * H * eb + w13_sc)
@@ -270,6 +275,10 @@ def side_workload(name, args, dev, peaks):
             codes, scales, rowwise = L.quantize_rowwise(xb)
             L.forward(codes, scales, topk_idx=d["topk_idx"], topk_weights=d["topk_weights"], out=out,
                       x_rowwise_scale=rowwise)
+    elif p["routing"] == "logits":
+        # routing from logits inside the single launch, as the main line
+        def step():
+            L.forward(d["x"], d["x_scale"], logits=d["logits"], bias=d["bias"], out=out)
     else:
         def step():
             L.forward(d["x"], d["x_scale"], topk_idx=d["topk_idx"], topk_weights=d["topk_weights"], out=out)
@@ -289,7 +298,8 @@ def side_workload(name, args, dev, peaks):
     torch.cuda.synchronize()
     L.check_status()
     med = statistics.median(a.elapsed_time(b) for a, b in ev)
-    num_active = int(torch.unique(d["topk_idx"][d["topk_idx"] >= 0]).numel())
+    idx = L.route(d["logits"], d["bias"])[0] if p["routing"] == "logits" else d["topk_idx"]
+    num_active = int(torch.unique(idx[idx >= 0]).numel())
     wm = work_model(p, num_active)["layer"]
     if p.get("act") == "bf16":   # the step reads BF16 activations instead of NVFP4 ones
         wm = dict(wm, bytes=wm["bytes"] + M * p["hidden"] * (2.0 - 0.5 - 1.0 / 16))
@@ -587,7 +597,8 @@ def main_ours(args):
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": {"bf16": "bf16", "fp8": "e4m3+f32 scales (f32 accumulate)",
-                  "nvfp4": "e2m1+e4m3 scales (f32 accumulate)"}[p["format"]],
+                  "nvfp4": "e2m1+e4m3 scales (f32 accumulate)",
+                  "mxfp8": "e4m3+ue8m0 scales per 32 (f32 accumulate)"}[p["format"]],
         "data": "synthetic (seeded torch generators; random-init experts of the workload's shapes)",
         "config": {"workload": args.workload + ("" if not args.set else " (" + ",".join(args.set) + ")"),
                    "path": "multi-launch chain" if args.chain else "moe_fused (one launch)",

@@ -57,6 +57,13 @@
  *                   gate_up_expert_scales fp32 [E]  L1 output multiplier
  *                   down_expert_scales    fp32 [E]  L2 output multiplier
  *                   c_input_scales        fp32 [E]  re-quant dequant multiplier G
+ *  format MXFP8     x  e4m3 [M, H], x_scale ue8m0 uint8 [M, H/32] (code c
+ *                   is 2^(c-127); flashinfer.fused_moe.MoEActivationPack,
+ *                   MXFP8 activations; the OCP MX block format)
+ *                   w13 e4m3 [E, 2I, H], w13_scale ue8m0 [E, 2I, H/32]
+ *                   w2  e4m3 [E, H, I],  w2_scale  ue8m0 [E, H, I/32]
+ *                   the intermediate is re-quantised per 32 columns with
+ *                   scale 2^(floor(log2 amax) - 8), clamped to 2^[-127, 127]
  *  topk_idx int64 [M, k]; topk_weights fp32 [M, k]; output bf16 [M, H].
  *
  *  Geometry (flashinfer.megamoe.MegaMoESymmBuffer, Parameters): hidden is a
@@ -87,7 +94,8 @@ typedef enum {
 typedef enum {
   MOE_FMT_BF16 = 0,
   MOE_FMT_FP8_E4M3_B128 = 1,  /* E4M3 with FP32 per-128 block scales */
-  MOE_FMT_NVFP4 = 2           /* e2m1 with E4M3 per-16 block scales + per-expert FP32 */
+  MOE_FMT_NVFP4 = 2,          /* e2m1 with E4M3 per-16 block scales + per-expert FP32 */
+  MOE_FMT_MXFP8 = 3           /* E4M3 with UE8M0 (power-of-two) per-32 block scales */
 } moe_format_t;
 
 /* The problem statement, after flashinfer.megamoe.MegaMoESymmBuffer
@@ -111,7 +119,7 @@ typedef struct {
  * 64*num_experts), else LARGE_M.  LARGE_M: 128 routed rows x 256 weight rows
  * per tile.  SMALL_M: the operands swapped, 256 weight rows x 32 routed rows
  * per tile, so the tensor work follows the routed rows that exist; BF16 and
- * FP8 only (MOE_ERR_UNSUPPORTED for NVFP4).  Results agree between regimes
+ * FP8 only (MOE_ERR_UNSUPPORTED for NVFP4 and MXFP8).  Results agree between regimes
  * up to FP32 summation order. */
 typedef enum {
   MOE_TILE_AUTO = 0,
@@ -134,8 +142,8 @@ typedef struct {
  * layouts listed above.  Every other call takes w13 and w2 as the PREPARED
  * blobs that moe_prepare_weights wrote (Struct_mega_ffn_ep_combine_send:
  * "pre-permuted gate/up weights", "pre-permuted W13 scale tile"); for NVFP4
- * the block scales are inside those blobs and w13_scale / w2_scale are
- * ignored; for FP8 w13_scale / w2_scale are the logical FP32 block scales.
+ * and MXFP8 the block scales are inside those blobs and w13_scale / w2_scale
+ * are ignored; for FP8 w13_scale / w2_scale are the logical FP32 block scales.
  * The three per-expert FP32 arrays are used by NVFP4 only and may be NULL
  * otherwise. */
 typedef struct {
@@ -222,13 +230,13 @@ moe_status_t moe_get_prepared_weights_size(const moe_problem_t* problem, size_t*
 
 /* One-time re-layout of the expert weights for the GEMM kernels (per weight
  * set; "pre-permuted" weights of Struct_mega_ffn_ep_combine_send).  Reads
- * `logical` (w13 / w2 and, for NVFP4, w13_scale / w2_scale in the logical
+ * `logical` (w13 / w2 and, for NVFP4 and MXFP8, w13_scale / w2_scale in the logical
  * layouts above) and writes out_w13 / out_w2 (device, sizes from
  * moe_get_prepared_weights_size, 16-byte aligned).  The blobs hold, for
  * every (expert, n tile, 128-byte K slice), the 256 weight rows the tile
  * multiplies (gate_up tiles: 64 gate rows, the 64 matching up rows, then
  * the next 64 of each) in the 128-byte-swizzled order the tensor cores read,
- * followed for NVFP4 by the slice's E4M3 scales in 512-byte tiles, so each
+ * followed for NVFP4 / MXFP8 by the slice's scales in 512-byte tiles, so each
  * pipeline stage streams one contiguous block. */
 moe_status_t moe_prepare_weights(const moe_problem_t* problem, const moe_weights_t* logical,
                                  void* out_w13, void* out_w2, void* stream);
@@ -272,10 +280,11 @@ moe_status_t moe_permute(const moe_problem_t* problem, const int64_t* topk_idx,
  * scatter-reduces w * y into `out` (MOE_OUT_ACCUMULATE) or stores y per row
  * (MOE_OUT_STAGED).  topk_weights fp32 [M, k] (read in accumulate mode).
  * If `intermediate` is not NULL the re-quantised intermediate is ALSO kept
- * there for inspection: codes [R, I] (BF16: 2 bytes, FP8: 1, NVFP4: 1/2
- * byte per element) at byte 0, followed at byte offset
- * moe_intermediate_scale_offset() by its scales (FP8: fp32 [I/128][P];
- * NVFP4: 512-byte tiles [P/128][I/64]; P = padded rows, a_scale_offsets[E]).
+ * there for inspection: codes [R, I] (BF16: 2 bytes, FP8 and MXFP8: 1,
+ * NVFP4: 1/2 byte per element) at byte 0, followed at the byte offset
+ * `scale_offset` of moe_get_intermediate_size by its scales (FP8: fp32 [I/128][P];
+ * NVFP4: 512-byte tiles [P/128][I/64]; MXFP8: 512-byte tiles [P/128][I/128];
+ * P = padded rows, a_scale_offsets[E]).
  * Size it with moe_get_intermediate_size. */
 moe_status_t moe_ffn(const moe_problem_t* problem, const moe_act_t* act,
                      const moe_weights_t* weights, const moe_layout_t* layout,

@@ -617,7 +617,7 @@ __global__ void __launch_bounds__(1024) perm_small_kernel(PermArgs a) {
 // ---------------------------------------------------------------------------
 struct GatherArgs {
   const uint8_t* x;          // [M][row_bytes]
-  const void* x_scale;       // FP8: fp32 [M][H/128]; NVFP4: e4m3 [M][H/16]
+  const void* x_scale;       // FP8: fp32 [M][H/128]; NVFP4: e4m3 [M][H/16]; MXFP8: ue8m0 [M][H/32]
   const int* src_info;
   const int* starts;
   const int* a_scale_offsets;
@@ -629,7 +629,7 @@ struct GatherArgs {
   int fmt;                   // FMT_*
   uint8_t* x_perm;           // [R][row_bytes]
   float* sa_t;               // FP8: [H/128][ld]
-  uint8_t* sfa;              // NVFP4: tiles [P/128][H/64]
+  uint8_t* sfa;              // NVFP4 / MXFP8: tiles [P/128][H/64 | H/128]
   int ld;                    // padded rows allocated
   // small-M GEMMs: their tile table (32-row tiles), built here; null otherwise
   const int* expert_ids;
@@ -710,10 +710,12 @@ __device__ __forceinline__ void gather_scales(const GatherArgs& g, int64_t t, in
   if (g.fmt == 1) {
     const float* xs = static_cast<const float*>(g.x_scale) + t * (g.H / 128);
     for (int kb = lane; kb < g.H / 128; kb += 32) g.sa_t[static_cast<size_t>(kb) * g.ld + pr] = xs[kb];
-  } else if (g.fmt == 2) {
-    const uint8_t* xs = static_cast<const uint8_t*>(g.x_scale) + t * (g.H / 16);
-    const int kc = g.H / 64;
-    for (int j = lane; j < g.H / 16; j += 32) {
+  } else if (g.fmt >= 2) {
+    // one byte per 16 (NVFP4) or 32 (MXFP8) elements, four per tile row
+    const int cols = g.fmt == 2 ? g.H / 16 : g.H / 32;
+    const uint8_t* xs = static_cast<const uint8_t*>(g.x_scale) + t * cols;
+    const int kc = cols / 4;
+    for (int j = lane; j < cols; j += 32) {
       const size_t off = (static_cast<size_t>(pr >> 7) * kc + (j >> 2)) * 512 + (pr & 31) * 16 +
                          ((pr >> 5) & 3) * 4 + (j & 3);
       g.sfa[off] = xs[j];
@@ -754,7 +756,7 @@ __device__ __forceinline__ void gather_rows(const GatherArgs& g, int64_t warp_id
     const int64_t t0 = g.src_info[r0] / g.topk;
     const int64_t t1 = (r1 >= 0) ? g.src_info[r1] / g.topk : 0;
     gather_copy2(g, r0, t0, r1, t1, lane);
-    if (g.fmt == 2) {
+    if (g.fmt >= 2) {
       gather_scales(g, t0, p0, lane);
       if (r1 >= 0) gather_scales(g, t1, p1, lane);
     }

@@ -203,6 +203,24 @@ __host__ __device__ constexpr uint32_t idesc_nvf4(uint32_t n) {
   return (1u << 7) | (1u << 10) | ((n >> 3) << 17) | ((128u >> 4) << 24);
 }
 
+// kind::mxf8f6f4 block-scaled: A = B = E4M3, UE8M0 scale factors (one per
+// 32 K elements, i.e. per instruction), M = 128, N = n; the scale factors of
+// instruction k of a 128-element K block are byte `sf_id` of their TMEM
+// words (one word per row holds the block's four scales).
+__host__ __device__ constexpr uint32_t idesc_mxf8(uint32_t n, uint32_t sf_id) {
+  return ((sf_id & 3u) << 4) | ((n >> 3) << 17) | (1u << 23) | ((128u >> 4) << 24) | ((sf_id & 3u) << 29);
+}
+
+__device__ __forceinline__ void mma_mxf8(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa,
+                                         uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale.scale_vec::1X"
+      " [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
 __device__ __forceinline__ void mma_f16(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
                                         uint32_t accumulate) {
   asm volatile(

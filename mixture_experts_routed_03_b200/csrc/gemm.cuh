@@ -12,6 +12,10 @@
 //          128-wide K block into a TMEM partial; the epilogue warps promote
 //          it, partial * (a_scale[row, kb] * b_scale[n_blk, kb]), into FP32
 //          registers (the per-128 FP32 block scales have no hardware form)
+//   MXFP8  tcgen05.mma kind::mxf8f6f4 block_scale scale_vec::1X: E4M3
+//          operands, UE8M0 scale per 32 elements (one per MMA instruction,
+//          picked by the descriptor's scale-factor id), copied to TMEM with
+//          tcgen05.cp; FP32 accumulation over all of K in TMEM
 //
 // Operands.  A (routed rows in expert order) comes by TMA, 128 rows x 128
 // bytes per stage, 128-byte swizzle.  B (expert weights) is PREPARED once
@@ -19,14 +23,14 @@
 // send): every (expert, n tile, K stage) block of 256 rows x 128 bytes is
 // stored contiguously, already in the 128-byte-swizzled order the MMA reads
 // (16-byte chunk c of row r at chunk c ^ (r mod 8)), followed for NVFP4 by its
-// 4 KB of scale tiles, so one bulk copy per stage streams it sequentially
+// 4 KB (MXFP8: 1 KB) of scale tiles, so one bulk copy per stage streams it sequentially
 // from HBM.  L1 B tiles interleave gate and up rows as [gate j0..j0+63 |
 // up j0..j0+63 | gate j0+64..j0+127 | up j0+64..j0+127], so each 128-column
 // half of the accumulator holds matching gate and up columns.
 //
 // Roles: warp 0 lane 0 issues the copies into a 4-stage ring guarded by
 // mbarriers; warp 1 lane 0 issues the MMAs (M = 128, N = 256, four 32-byte K
-// steps per stage) and commits them; for NVFP4, warp 2 lane 0 moves each
+// steps per stage) and commits them; for NVFP4 and MXFP8, warp 2 lane 0 moves each
 // stage's scale factors from shared memory into one of two TMEM scale
 // buffers (tcgen05.cp), so their issue cost overlaps the MMAs; the last 8
 // warps are the epilogue, two per 32-lane TMEM quarter, one per 128-column
@@ -41,11 +45,12 @@
 // L1 epilogue: h = min(g,c) * sigmoid(min(g,c)) * clamp(u,-c,c) is formed in
 // registers, the accumulator is released, then h is re-quantised (BF16 by
 // rounding; FP8 per 128 columns with scale amax/448; NVFP4 per 16 columns
-// with an E4M3 scale against the per-expert c_input_scales) and stored in
-// expert order for L2.
+// with an E4M3 scale against the per-expert c_input_scales; MXFP8 per 32
+// columns with the power-of-two scale 2^(floor(log2 amax) - 8)) and stored
+// in expert order for L2.
 // L2 epilogue: the row is read into registers, the accumulator released, and
 // the row, times its router weight, added into the token-ordered FP32
-// accumulator -- float4 atomics through a 32 x 32 transpose (BF16, FP8) or
+// accumulator -- float4 atomics through a 32 x 32 transpose (BF16, FP8, MXFP8) or
 // TMA bulk reduce-adds (NVFP4); no (M*k, H) staging buffer -- or, in staged
 // mode, stored per row.
 //
@@ -58,7 +63,7 @@
 
 namespace moe {
 
-enum { FMT_BF16 = 0, FMT_FP8 = 1, FMT_NVFP4 = 2 };
+enum { FMT_BF16 = 0, FMT_FP8 = 1, FMT_NVFP4 = 2, FMT_MXFP8 = 3 };
 enum { EPI_L1 = 0, EPI_L2_ACC = 1, EPI_L2_STAGED = 2 };
 
 constexpr int kBM = 128;          // MMA M: rows of A (routed rows) per tile
@@ -69,9 +74,12 @@ constexpr int kBStage = kBN * kBK;            // 32 KB
 constexpr int kSFTile = 512;                  // 128 rows x 4 scale bytes
 constexpr int kSFAStage = 4 * kSFTile;        // 4 K-steps of 64 e2m1
 constexpr int kSFBStage = 2 * 4 * kSFTile;    // 2 row blocks x 4 K-steps
+constexpr int kMxSFAStage = kSFTile;          // MXFP8: 4 scales (128 E4M3) per row
+constexpr int kMxSFBStage = 2 * kSFTile;      // MXFP8: 2 row blocks
 constexpr int kTmemCols = 512;
 // NVFP4 scale factors in TMEM: two buffers of 48 columns after the
-// accumulator, A scales (16 columns) then B scales (32 columns).  (A ring of
+// accumulator, A scales (16 columns) then B scales (32 columns).  MXFP8 uses
+// the same buffers: A in columns 0..3, B in columns 16..23 of each.  (A ring of
 // four was measured no faster: the stage's twelve tcgen05.cp take ~600
 // cycles of the tensor pipe per K step whatever the ring depth.)
 constexpr int kSFCol0 = 256;
@@ -81,8 +89,11 @@ constexpr int kEpiWarps = 8;
 
 // Bytes of one prepared B block (one stage of one tile).
 __host__ __device__ constexpr int b_block_bytes(int fmt) {
-  return kBStage + (fmt == FMT_NVFP4 ? kSFBStage : 0);
+  return kBStage + (fmt == FMT_NVFP4 ? kSFBStage : fmt == FMT_MXFP8 ? kMxSFBStage : 0);
 }
+
+// Formats whose block scales the tensor cores apply from TMEM.
+__host__ __device__ constexpr bool hw_scaled(int fmt) { return fmt == FMT_NVFP4 || fmt == FMT_MXFP8; }
 
 // Gate/up interleave of the prepared gate_up tiles: groups of G gate rows
 // followed by the G matching up rows, so that every 2G accumulator columns
@@ -107,12 +118,18 @@ struct GemmCfg {
   // L2 gives 36 KB of shared memory to the epilogue's transpose buffers
   static constexpr int kStages = (EPI == EPI_L1) ? 4 : 3;
   // accumulator (BF16/NVFP4) or partial (FP8) buffers of 256 TMEM columns
-  static constexpr int kAccBufs = (FMT == FMT_NVFP4) ? 1 : 2;
-  static constexpr int kStageBytes =
-      kAStage + kBStage + ((FMT == FMT_NVFP4) ? (kSFBStage + kSFAStage) : 0);
-  // warp 0 producer, warp 1 MMA issuer, (NVFP4) warp 2 scale-factor copier,
-  // then the epilogue warps
-  static constexpr int kFirstEpiWarp = (FMT == FMT_NVFP4) ? 3 : 2;
+  static constexpr int kAccBufs = hw_scaled(FMT) ? 1 : 2;
+  // bytes one stage's copies bring in
+  static constexpr int kStageLoadBytes =
+      kAStage + kBStage + ((FMT == FMT_NVFP4)   ? (kSFBStage + kSFAStage)
+                           : (FMT == FMT_MXFP8) ? (kMxSFBStage + kMxSFAStage)
+                                                : 0);
+  // stage stride: every stage's A tile starts on a 1024-byte boundary (the
+  // 128-byte swizzle's period)
+  static constexpr int kStageBytes = (kStageLoadBytes + 1023) / 1024 * 1024;
+  // warp 0 producer, warp 1 MMA issuer, (NVFP4, MXFP8) warp 2 scale-factor
+  // copier, then the epilogue warps
+  static constexpr int kFirstEpiWarp = hw_scaled(FMT) ? 3 : 2;
   static constexpr int kThreads = (kFirstEpiWarp + kEpiWarps) * 32;
   static constexpr int kBarrierBytes = 4096;
   static constexpr int kXposeStride = 36;   // floats per row of a 32 x 32 transpose buffer
@@ -147,7 +164,7 @@ struct GemmArgs {
   const float* topk_weights;
   // prepared weights: [E][n_tiles][k_stages] blocks of b_block_bytes(FMT)
   const uint8_t* wB;
-  // NVFP4 A scales: 512-byte tiles [row block][K/64]
+  // NVFP4 / MXFP8 A scales: 512-byte tiles [row block][K/64 | K/128]
   const uint8_t* sfa;
   int sfa_kc;
   // FP8 scales: A transposed [K/128][sa_ld] (padded rows), B [E][N/128][K/128]
@@ -162,7 +179,7 @@ struct GemmArgs {
   // L1 output: the re-quantised intermediate, expert order
   uint8_t* h_out;
   int h_row_bytes;
-  uint8_t* h_sf;        // NVFP4 scale tiles [P/128][I/64]
+  uint8_t* h_sf;        // NVFP4 / MXFP8 scale tiles [P/128][I/64 | I/128]
   int h_sf_kc;
   float* h_scale_t;     // FP8 scales transposed [I/128][h_scale_ld]
   int h_scale_ld;
@@ -373,13 +390,16 @@ __device__ __forceinline__ void gemm_phase(const GemmArgs& p, const CUtensorMap*
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status, 1)) goto producer_done;
           uint8_t* sa = smem + stage * SB;
           uint8_t* sbp = sa + kAStage;
-          mbar_arrive_expect_tx(&full[stage], SB);
+          mbar_arrive_expect_tx(&full[stage], Cfg::kStageLoadBytes);
           tma_load_2d(sa, tmA, &full[stage], ks * kBK, t.row0);
           bulk_load(sbp, wb + static_cast<size_t>(ks) * BB, BB, &full[stage]);
           if (FMT == FMT_NVFP4) {
             bulk_load(sbp + BB,
                       p.sfa + (static_cast<size_t>(t.srow0 >> 7) * p.sfa_kc + ks * 4) * kSFTile,
                       kSFAStage, &full[stage]);
+          } else if (FMT == FMT_MXFP8) {
+            bulk_load(sbp + BB, p.sfa + (static_cast<size_t>(t.srow0 >> 7) * p.sfa_kc + ks) * kSFTile,
+                      kMxSFAStage, &full[stage]);
           }
           ++issued;
           if (++stage == S) {
@@ -405,9 +425,10 @@ __device__ __forceinline__ void gemm_phase(const GemmArgs& p, const CUtensorMap*
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t kIdesc = (FMT == FMT_BF16)  ? idesc_dense(1, 1, kBN)
-                                  : (FMT == FMT_FP8) ? idesc_dense(0, 0, kBN)
-                                                     : idesc_nvf4(kBN);
+      constexpr uint32_t kIdesc = (FMT == FMT_BF16)    ? idesc_dense(1, 1, kBN)
+                                  : (FMT == FMT_FP8)   ? idesc_dense(0, 0, kBN)
+                                  : (FMT == FMT_NVFP4) ? idesc_nvf4(kBN)
+                                                       : idesc_mxf8(kBN, 0);
       int stage = 0;
       uint32_t phase = 0;
       int ab = 0;
@@ -439,7 +460,7 @@ __device__ __forceinline__ void gemm_phase(const GemmArgs& p, const CUtensorMap*
           const uint64_t adesc = sdesc_sw128(smem_u32(sa));
           const uint64_t bdesc = sdesc_sw128(smem_u32(sbp));
           const uint32_t sfa_t = tmem + kSFCol0 + kSFBufCols * sb;
-          if (FMT == FMT_NVFP4) {
+          if (hw_scaled(FMT)) {
             if (!mbar_wait(&sf_full[sb], sphase, abort_flag, p.status, 8)) {
               ok = false;
               break;
@@ -453,10 +474,12 @@ __device__ __forceinline__ void gemm_phase(const GemmArgs& p, const CUtensorMap*
             const uint64_t b = bdesc + static_cast<uint64_t>(2 * kc);
             if (FMT == FMT_BF16) mma_f16(d, a, b, kIdesc, acc);
             else if (FMT == FMT_FP8) mma_f8(d, a, b, kIdesc, acc);
-            else mma_nvf4(d, a, b, kIdesc, sfa_t + 4 * kc, sfa_t + kSFBOff + 8 * kc, acc);
+            else if (FMT == FMT_NVFP4) mma_nvf4(d, a, b, kIdesc, sfa_t + 4 * kc, sfa_t + kSFBOff + 8 * kc, acc);
+            // one UE8M0 scale per 32-wide K step: byte kc of the stage's scale words
+            else mma_mxf8(d, a, b, idesc_mxf8(kBN, kc), sfa_t, sfa_t + kSFBOff, acc);
           }
           mma_commit(&empty[stage]);
-          if (FMT == FMT_NVFP4) {
+          if (hw_scaled(FMT)) {
             mma_commit(&sf_empty[sb]);
             if (++sb == 2) {
               sb = 0;
@@ -487,7 +510,7 @@ __device__ __forceinline__ void gemm_phase(const GemmArgs& p, const CUtensorMap*
       mma_commit(final_bar);
       mbar_drain(final_bar, 0);
     }
-  } else if (FMT == FMT_NVFP4 && warp == 2) {
+  } else if (hw_scaled(FMT) && warp == 2) {
     // ------------------------------------------------------------ scale copier
     if (lane == 0) {
       int stage = 0;
@@ -504,13 +527,20 @@ __device__ __forceinline__ void gemm_phase(const GemmArgs& p, const CUtensorMap*
           }
           tc_fence_after();
           const uint32_t sfb_s = smem_u32(smem + stage * SB + kAStage + kBStage);
-          const uint32_t sfa_s = sfb_s + kSFBStage;
           const uint32_t dst = tmem + kSFCol0 + kSFBufCols * sb;
+          if (FMT == FMT_NVFP4) {
+            const uint32_t sfa_s = sfb_s + kSFBStage;
 #pragma unroll
-          for (int kc = 0; kc < 4; ++kc) {
-            tmem_copy_sf(dst + 4 * kc, sdesc_sf_tile(sfa_s + kc * kSFTile));
-            tmem_copy_sf(dst + kSFBOff + 8 * kc, sdesc_sf_tile(sfb_s + kc * kSFTile));
-            tmem_copy_sf(dst + kSFBOff + 8 * kc + 4, sdesc_sf_tile(sfb_s + 4 * kSFTile + kc * kSFTile));
+            for (int kc = 0; kc < 4; ++kc) {
+              tmem_copy_sf(dst + 4 * kc, sdesc_sf_tile(sfa_s + kc * kSFTile));
+              tmem_copy_sf(dst + kSFBOff + 8 * kc, sdesc_sf_tile(sfb_s + kc * kSFTile));
+              tmem_copy_sf(dst + kSFBOff + 8 * kc + 4, sdesc_sf_tile(sfb_s + 4 * kSFTile + kc * kSFTile));
+            }
+          } else {
+            // MXFP8: one tile per 128 rows covers the stage's four K steps
+            tmem_copy_sf(dst, sdesc_sf_tile(sfb_s + kMxSFBStage));
+            tmem_copy_sf(dst + kSFBOff, sdesc_sf_tile(sfb_s));
+            tmem_copy_sf(dst + kSFBOff + 4, sdesc_sf_tile(sfb_s + kSFTile));
           }
           mma_commit(&sf_full[sb]);
           if (++sb == 2) {
@@ -603,7 +633,7 @@ __device__ __forceinline__ void gemm_phase(const GemmArgs& p, const CUtensorMap*
         }
         if (!ok) break;
       } else {
-        // BF16 / NVFP4: the whole K sum is in TMEM; read it, release it.
+        // BF16 / NVFP4 / MXFP8: the whole K sum is in TMEM; read it, release it.
         if (!mbar_wait(&acc_full[ab], aphase, abort_flag, p.status, 6)) break;
         tc_fence_after();
         if (gather_wgt) wgt = __ldg(p.topk_weights + s_flat);
@@ -691,6 +721,38 @@ __device__ __forceinline__ void gemm_phase(const GemmArgs& p, const CUtensorMap*
             const uint4 v = *reinterpret_cast<const uint4*>(stg + row * Cfg::kHStageStride + c16 * 16);
             if (row < rows_here)
               *reinterpret_cast<uint4*>(hbase + static_cast<size_t>(row) * p.h_row_bytes + c16 * 16) = v;
+          }
+        } else if constexpr (FMT == FMT_MXFP8) {
+          // two 32-column blocks: scale 2^X, X = floor(log2 amax) - 8 clamped
+          // to [-127, 127] (read off amax's exponent field; a zero or
+          // subnormal amax gives -127), codes e4m3(h * 2^-X) saturating --
+          // the scaling by a power of two is exact
+          uint32_t w[16];
+          uint32_t sfw = 0;
+#pragma unroll
+          for (int b = 0; b < 2; ++b) {
+            float amax = 0.0f;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(h[32 * b + j]));
+            const int ex = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFFu);
+            const int X = ex == 0 ? -127 : max(ex - 135, -127);
+            const float inv = __uint_as_float(static_cast<uint32_t>(127 - X) << 23);   // 2^-X
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const uint32_t lo = cvt_e4m3x2(__fmul_rn(h[32 * b + 4 * i], inv), __fmul_rn(h[32 * b + 4 * i + 1], inv));
+              const uint32_t hi =
+                  cvt_e4m3x2(__fmul_rn(h[32 * b + 4 * i + 2], inv), __fmul_rn(h[32 * b + 4 * i + 3], inv));
+              w[8 * b + i] = lo | (hi << 16);
+            }
+            sfw |= static_cast<uint32_t>(X + 127) << (8 * b);
+          }
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(hrow + hcol0);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+            // scale columns hcol0/32 and hcol0/32 + 1 (even) share a 4-byte group
+            *reinterpret_cast<uint16_t*>(p.h_sf + sf_tile_offset(pr, hcol0 >> 5, p.h_sf_kc)) =
+                static_cast<uint16_t>(sfw);
           }
         } else if constexpr (FMT == FMT_BF16) {
           if (valid) {
@@ -836,15 +898,16 @@ __global__ void __launch_bounds__(GemmCfg<FMT, EPI>::kThreads, 1)
 
 // ---------------------------------------------------------------------------
 // Weight preparation: logical K-major weights [E][N][Kb] (+ NVFP4 scales
-// [E][N][K/16]) -> blocks [E][n_tiles][k_stages] of b_block_bytes(fmt).
-// One thread per 16-byte chunk of block data; the NVFP4 scale tiles follow.
+// [E][N][K/16], MXFP8 scales [E][N][K/32]) -> blocks [E][n_tiles][k_stages]
+// of b_block_bytes(fmt).  One thread per 16-byte chunk of block data; the
+// scale tiles follow.
 // ---------------------------------------------------------------------------
 struct PrepArgs {
   const uint8_t* w;        // logical weights
-  const uint8_t* sf;       // NVFP4 logical scales, else null
+  const uint8_t* sf;       // NVFP4 / MXFP8 logical scales, else null
   uint8_t* out;
   int E, N, Kb;            // experts, rows per expert, bytes per row
-  int ksf;                 // NVFP4 scale columns per row (K/16)
+  int ksf;                 // scale columns per row (NVFP4 K/16, MXFP8 K/32)
   int n_tiles, k_stages;
   int l1;                  // 1: gate/up interleaved L1 tiles (N = 2I)
   int fmt;
@@ -875,20 +938,23 @@ __global__ void __launch_bounds__(256) prepare_weights_kernel(PrepArgs a) {
         a.w + (static_cast<size_t>(e) * a.N + row) * a.Kb + static_cast<size_t>(ks) * kBK + 16 * c);
     *reinterpret_cast<uint4*>(a.out + blk * bb + within * 16) = *src;
   }
-  if (a.fmt != FMT_NVFP4) return;
-  const int64_t nsf = blocks * kSFBStage;
+  if (!hw_scaled(a.fmt)) return;
+  // per row block: NVFP4 four tiles (K steps kc), MXFP8 one
+  const int tiles_per_rb = a.fmt == FMT_NVFP4 ? 4 : 1;
+  const int sf_block = bb - kBStage;
+  const int64_t nsf = blocks * sf_block;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nsf;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t blk = i / kSFBStage;
-    const int o = static_cast<int>(i - blk * kSFBStage);
-    const int rb = o / (4 * kSFTile), kc = (o / kSFTile) & 3, b = o & (kSFTile - 1);
+    const int64_t blk = i / sf_block;
+    const int o = static_cast<int>(i - blk * sf_block);
+    const int rb = o / (tiles_per_rb * kSFTile), kc = (o / kSFTile) % tiles_per_rb, b = o & (kSFTile - 1);
     const int ks = static_cast<int>(blk % a.k_stages);
     const int64_t et = blk / a.k_stages;
     const int nt = static_cast<int>(et % a.n_tiles);
     const int e = static_cast<int>(et / a.n_tiles);
     const int tile_row = 128 * rb + ((b & 15) >> 2) * 32 + (b >> 4);
     const int row = prep_row(a, nt, tile_row);
-    const int col = ks * 16 + kc * 4 + (b & 3);
+    const int col = ks * 4 * tiles_per_rb + kc * 4 + (b & 3);
     a.out[blk * bb + kBStage + o] = a.sf[(static_cast<size_t>(e) * a.N + row) * a.ksf + col];
   }
 }

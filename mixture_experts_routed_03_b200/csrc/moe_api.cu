@@ -24,20 +24,26 @@ constexpr size_t kAlign = 256;
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // ---------------------------------------------------------------- validation
-int x_row_bytes(int fmt, int H) { return fmt == FMT_BF16 ? 2 * H : (fmt == FMT_FP8 ? H : H / 2); }
-int h_row_bytes(int fmt, int I) { return fmt == FMT_BF16 ? 2 * I : (fmt == FMT_FP8 ? I : I / 2); }
+int x_row_bytes(int fmt, int H) { return fmt == FMT_BF16 ? 2 * H : (fmt == FMT_NVFP4 ? H / 2 : H); }
+int h_row_bytes(int fmt, int I) { return fmt == FMT_BF16 ? 2 * I : (fmt == FMT_NVFP4 ? I / 2 : I); }
+
+// Bytes of the block scales of one padded row of K elements.
+size_t scale_row_bytes(int fmt, int K) {
+  return fmt == FMT_FP8 ? size_t(K / 128) * 4 : fmt == FMT_NVFP4 ? size_t(K / 16) : fmt == FMT_MXFP8 ? size_t(K / 32) : 0;
+}
 
 moe_status_t check_problem(const moe_problem_t* p) {
   if (!p) return MOE_ERR_INVALID_ARG;
   if (p->num_tokens < 0) return MOE_ERR_INVALID_ARG;
-  if (p->format < MOE_FMT_BF16 || p->format > MOE_FMT_NVFP4) return MOE_ERR_INVALID_ARG;
+  if (p->format < MOE_FMT_BF16 || p->format > MOE_FMT_MXFP8) return MOE_ERR_INVALID_ARG;
   if (p->hidden <= 0 || p->hidden % 256 != 0) return MOE_ERR_INVALID_ARG;
   if (p->intermediate_hidden <= 0 || p->intermediate_hidden % 128 != 0) return MOE_ERR_INVALID_ARG;
   if (p->num_experts < 1 || p->num_topk < 1 || p->num_topk > p->num_experts) return MOE_ERR_INVALID_ARG;
   if (p->num_experts > 1024) return MOE_ERR_UNSUPPORTED;
   if (std::isnan(p->activation_clamp) || !(p->activation_clamp > 0.0f)) return MOE_ERR_INVALID_ARG;
   if (p->tile_regime < MOE_TILE_AUTO || p->tile_regime > MOE_TILE_SMALL_M) return MOE_ERR_INVALID_ARG;
-  if (p->tile_regime == MOE_TILE_SMALL_M && p->format == MOE_FMT_NVFP4) return MOE_ERR_UNSUPPORTED;
+  if (p->tile_regime == MOE_TILE_SMALL_M && (p->format == MOE_FMT_NVFP4 || p->format == MOE_FMT_MXFP8))
+    return MOE_ERR_UNSUPPORTED;
   if (p->format == MOE_FMT_NVFP4 && p->intermediate_hidden % 256 != 0) return MOE_ERR_UNSUPPORTED;
   const int64_t R = p->num_tokens * p->num_topk;
   if (R > (int64_t(1) << 30)) return MOE_ERR_UNSUPPORTED;
@@ -89,9 +95,9 @@ WsLayout make_layout(const moe_problem_t* p) {
   L.block_counts = take(size_t(L.nblk) * E * 4);
   L.tiles32 = take(size_t(E + 1) * 4);
   L.x_perm = take(size_t(L.R) * x_row_bytes(fmt, H));
-  L.x_sf = take(fmt == FMT_FP8 ? size_t(H / 128) * L.P * 4 : (fmt == FMT_NVFP4 ? size_t(L.P) * (H / 16) : 0));
+  L.x_sf = take(size_t(L.P) * scale_row_bytes(fmt, H));
   L.h_bytes = size_t(L.R) * h_row_bytes(fmt, I);
-  L.h_sf_bytes = fmt == FMT_FP8 ? size_t(I / 128) * L.P * 4 : (fmt == FMT_NVFP4 ? size_t(L.P) * (I / 16) : 0);
+  L.h_sf_bytes = size_t(L.P) * scale_row_bytes(fmt, I);
   L.h = take(L.h_bytes);
   L.h_sf = take(L.h_sf_bytes);
   L.acc = take(size_t(L.M) * H * 4);
@@ -232,9 +238,11 @@ cudaError_t set_all_attrs() {
   if ((e = set_fused_attr<FMT_BF16>()) != cudaSuccess) return e;
   if ((e = set_fused_attr<FMT_FP8>()) != cudaSuccess) return e;
   if ((e = set_fused_attr<FMT_NVFP4>()) != cudaSuccess) return e;
+  if ((e = set_fused_attr<FMT_MXFP8>()) != cudaSuccess) return e;
   if ((e = set_attrs_fmt<FMT_BF16>()) != cudaSuccess) return e;
   if ((e = set_attrs_fmt<FMT_FP8>()) != cudaSuccess) return e;
   if ((e = set_attrs_fmt<FMT_NVFP4>()) != cudaSuccess) return e;
+  if ((e = set_attrs_fmt<FMT_MXFP8>()) != cudaSuccess) return e;
   if ((e = set_swap_attrs_fmt<FMT_BF16>()) != cudaSuccess) return e;
   return set_swap_attrs_fmt<FMT_FP8>();
 }
@@ -269,6 +277,7 @@ cudaError_t launch_gemm_fmt(int fmt, bool swap, const GemmArgs& a, const CUtenso
   switch (fmt) {
     case FMT_BF16: return launch_gemm<FMT_BF16, EPI>(a, ta, grid, st);
     case FMT_FP8: return launch_gemm<FMT_FP8, EPI>(a, ta, grid, st);
+    case FMT_MXFP8: return launch_gemm<FMT_MXFP8, EPI>(a, ta, grid, st);
     default: return launch_gemm<FMT_NVFP4, EPI>(a, ta, grid, st);
   }
 }
@@ -358,7 +367,7 @@ struct FfnPlan {
 // The GEMMs' tile regime for this problem (MOE_TILE_AUTO resolved).
 bool small_m_tiles(const moe_problem_t* p) {
   if (p->tile_regime == MOE_TILE_SMALL_M) return true;
-  if (p->tile_regime == MOE_TILE_LARGE_M || p->format == FMT_NVFP4) return false;
+  if (p->tile_regime == MOE_TILE_LARGE_M || p->format == FMT_NVFP4 || p->format == FMT_MXFP8) return false;
   return p->num_tokens * p->num_topk <= int64_t(64) * p->num_experts;
 }
 
@@ -425,7 +434,7 @@ moe_status_t plan_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_we
   a.src_info = b.src_info;
   a.topk_weights = topk_weights;
   a.sfa = b.x_sf;
-  a.sfa_kc = H / 64;
+  a.sfa_kc = fmt == FMT_MXFP8 ? H / 128 : H / 64;   // scale tiles per 128-row block
   a.sa_t = reinterpret_cast<const float*>(b.x_sf);
   a.sa_ld = int(b.P);
   a.sb = static_cast<const float*>(w->w13_scale);
@@ -437,7 +446,7 @@ moe_status_t plan_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_we
   a.h_out = b.h;
   a.h_row_bytes = h_row_bytes(fmt, I);
   a.h_sf = b.h_sf;
-  a.h_sf_kc = I / 64;
+  a.h_sf_kc = fmt == FMT_MXFP8 ? I / 128 : I / 64;
   a.h_scale_t = reinterpret_cast<float*>(b.h_sf);
   a.h_scale_ld = int(b.P);
   a.status = b.status;
@@ -464,7 +473,7 @@ moe_status_t plan_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_we
   a2.n_group = (size_t(R) * h_row_bytes(fmt, I) <= kL2Budget) ? 1 : a2.n_tiles;
   a2.wB = static_cast<const uint8_t*>(w->w2);
   a2.sfa = b.h_sf;
-  a2.sfa_kc = I / 64;
+  a2.sfa_kc = a.h_sf_kc;
   a2.sa_t = reinterpret_cast<const float*>(b.h_sf);
   a2.sb = static_cast<const float*>(w->w2_scale);
   a2.sb_nb = H / 128;
@@ -710,7 +719,8 @@ moe_status_t moe_prepare_weights(const moe_problem_t* p, const moe_weights_t* lo
   if (!logical || !logical->w13 || !logical->w2 || !out_w13 || !out_w2) return MOE_ERR_INVALID_ARG;
   if (!aligned16(logical->w13) || !aligned16(logical->w2) || !aligned16(out_w13) || !aligned16(out_w2))
     return MOE_ERR_INVALID_ARG;
-  if (p->format == MOE_FMT_NVFP4 && (!logical->w13_scale || !logical->w2_scale)) return MOE_ERR_INVALID_ARG;
+  if ((p->format == MOE_FMT_NVFP4 || p->format == MOE_FMT_MXFP8) && (!logical->w13_scale || !logical->w2_scale))
+    return MOE_ERR_INVALID_ARG;
   if (!ensure_init()) return MOE_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int fmt = p->format, E = p->num_experts, H = p->hidden, I = p->intermediate_hidden;
@@ -723,7 +733,7 @@ moe_status_t moe_prepare_weights(const moe_problem_t* p, const moe_weights_t* lo
   a.out = static_cast<uint8_t*>(out_w13);
   a.N = 2 * I;
   a.Kb = x_row_bytes(fmt, H);
-  a.ksf = H / 16;
+  a.ksf = fmt == FMT_MXFP8 ? H / 32 : H / 16;
   a.n_tiles = I / 128;
   a.k_stages = a.Kb / 128;
   a.l1 = 1;
@@ -736,7 +746,7 @@ moe_status_t moe_prepare_weights(const moe_problem_t* p, const moe_weights_t* lo
   a.out = static_cast<uint8_t*>(out_w2);
   a.N = H;
   a.Kb = h_row_bytes(fmt, I);
-  a.ksf = I / 16;
+  a.ksf = fmt == FMT_MXFP8 ? I / 32 : I / 16;
   a.n_tiles = H / 256;
   a.k_stages = a.Kb / 128;
   a.l1 = 0;
@@ -938,6 +948,7 @@ moe_status_t moe_fused(const moe_problem_t* p, const moe_act_t* act, const moe_w
     case FMT_FP8:
       e = pl.swap ? launch_fused_fmt<FMT_FP8, true>(f, pl, grid, st) : launch_fused_fmt<FMT_FP8, false>(f, pl, grid, st);
       break;
+    case FMT_MXFP8: e = launch_fused_fmt<FMT_MXFP8, false>(f, pl, grid, st); break;
     default: e = launch_fused_fmt<FMT_NVFP4, false>(f, pl, grid, st); break;
   }
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;

@@ -60,7 +60,7 @@ class MoELayer:
         self.alpha1 = w.get("gate_up_expert_scales")
         self.alpha2 = w.get("down_expert_scales")
         self.c_in = w.get("c_input_scales")
-        # FP8 block scales stay logical; NVFP4 scales go into the prepared blobs
+        # FP8 block scales stay logical; NVFP4 and MXFP8 scales go into the prepared blobs
         self.w13_scale = w.get("w13_scale") if self.p["format"] == "fp8" else None
         self.w2_scale = w.get("w2_scale") if self.p["format"] == "fp8" else None
         n13, n2 = api.prepared_weights_size(self.prob)

@@ -8,7 +8,7 @@ Gaussian draws for E4M3, torch's bfloat16 cast for BF16) and scales are drawn
 as plain positive numbers.  Both the CUDA path and the CPU oracle consume
 what it returns; neither is imported here.
 
-The five workloads follow the shapes and value structure of the routed-MoE
+The workloads follow the shapes and value structure of the routed-MoE
 API pages (flashinfer.megamoe.MegaMoESymmBuffer staging views; Struct_mega_
 ffn_ep_combine_send operands; flashinfer.fused_moe.MoEActivationPack
 activation encodings and FromLogits routing):
@@ -20,6 +20,8 @@ activation encodings and FromLogits routing):
   fp8_prefill_routed M=16384 H=4096 I=1536 E=128 k=8 E4M3, routing from logits
   nvfp4_prefill_rowwise  as nvfp4_prefill, with BF16 activations [M, H]
                      (x_bf16) for the per-token quantiser
+  mxfp8_prefill_routed   the fp8_prefill_routed shapes in MXFP8: E4M3 with
+                     UE8M0 scales per 32 (MoEActivationPack MXFP8)
 """
 
 import math
@@ -42,6 +44,10 @@ WORKLOADS = {
     "nvfp4_prefill_rowwise": dict(num_tokens=4096, hidden=7168, intermediate_hidden=2048,
                                   num_experts=32, num_topk=8, format="nvfp4", routing="uniform",
                                   act="bf16"),
+    # the FP8 prefill's shapes with the microscaling format's power-of-two
+    # scales per 32 elements, which the tensor cores apply themselves
+    "mxfp8_prefill_routed": dict(num_tokens=16384, hidden=4096, intermediate_hidden=1536,
+                                 num_experts=128, num_topk=8, format="mxfp8", routing="logits"),
 }
 
 # Typical magnitudes of the drawn values.
@@ -81,6 +87,11 @@ def _e4m3_codes(shape, g, device):
 
 def _e4m3_positive(shape, lo, hi, g, device):
     return _uniform(shape, lo, hi, g, device).to(torch.float8_e4m3fn).view(torch.uint8)
+
+
+def _ue8m0_codes(shape, lo, hi, g, device):
+    """UE8M0 scale codes drawn uniformly from the integers lo..hi (code c is 2^(c-127))."""
+    return torch.randint(lo, hi + 1, shape, generator=g, device=device, dtype=torch.int32).to(torch.uint8)
 
 
 def _fp4_bytes(shape, g, device):
@@ -124,9 +135,9 @@ def make_inputs(p, seed=0, device="cpu"):
       topk_idx, topk_weights          (precomputed routing), or
       logits, bias                    (routing from logits).
     Layouts: x [M, H] (BF16 / E4M3) or [M, H/2] packed e2m1; x_scale
-    FP32 [M, H/128] or E4M3 [M, H/16]; w13 [E, 2I, H(/2)] with gate rows
-    first; w2 [E, H, I(/2)]; weight scales FP32 [E, N/128, K/128] or E4M3
-    [E, N, K/16].
+    FP32 [M, H/128], E4M3 [M, H/16] or UE8M0 [M, H/32]; w13 [E, 2I, H(/2)]
+    with gate rows first; w2 [E, H, I(/2)]; weight scales FP32
+    [E, N/128, K/128], E4M3 [E, N, K/16] or UE8M0 [E, N, K/32].
     """
     device = torch.device(device)
     g = _gen(device, seed)
@@ -169,6 +180,18 @@ def make_inputs(p, seed=0, device="cpu"):
         d["gate_up_expert_scales"] = (w13_global * x_global).to(torch.float32)
         d["down_expert_scales"] = (w2_global * c_in).to(torch.float32)
         d["c_input_scales"] = c_in.to(torch.float32)
+    elif fmt == "mxfp8":
+        # power-of-two scales around X_STD / FP8_CODE_STD = 2^-6 (codes
+        # 120..122) and W_STD / FP8_CODE_STD ~ 2^-11.6 (codes 115..117)
+        d["x"] = _e4m3_codes((M, H), g, device)
+        d["x_scale"] = _ue8m0_codes((M, H // 32), 120, 122, g, device)
+        d["w13"] = torch.empty((E, 2 * I, H), dtype=torch.uint8, device=device)
+        d["w2"] = torch.empty((E, H, I), dtype=torch.uint8, device=device)
+        for e in range(E):
+            d["w13"][e] = _e4m3_codes((2 * I, H), g, device)
+            d["w2"][e] = _e4m3_codes((H, I), g, device)
+        d["w13_scale"] = _ue8m0_codes((E, 2 * I, H // 32), 115, 117, g, device)
+        d["w2_scale"] = _ue8m0_codes((E, H, I // 32), 115, 117, g, device)
     else:
         raise ValueError(fmt)
     if p.get("act") == "bf16":

@@ -10,7 +10,7 @@ from oracle import formats as F
 from oracle import moe as O
 
 # max|err| bounds of the FFN output, relative to rms(oracle output)
-TOL = {"bf16": 5e-3, "fp8": 2e-2, "nvfp4": 2e-2}
+TOL = {"bf16": 5e-3, "fp8": 2e-2, "nvfp4": 2e-2, "mxfp8": 2e-2}
 # An intermediate code may differ from the oracle's only if it is the correct
 # rounding of a value within this distance of the oracle's pre-rounding FP32
 # value, relative to that value (the kernel's FP32 h differs from the
@@ -137,7 +137,8 @@ class GpuResult:
     def rows(self, p, rows):
         """GPU intermediate rows -> {row: dict(values, scales, hhat)}: values =
         decoded element codes (unscaled), scales = block scales (FP8 float32,
-        NVFP4 E4M3 codes), hhat = dequantised row (float64, the L2 input)."""
+        NVFP4 E4M3 codes, MXFP8 UE8M0 codes), hhat = dequantised row (float64,
+        the L2 input)."""
         fmt, I = p["format"], p["intermediate_hidden"]
         R_total = p["num_tokens"] * p["num_topk"]
         out = {}
@@ -156,6 +157,17 @@ class GpuResult:
                 s = sc[:, pr].copy()
                 out[r] = dict(codes=codes[r], values=F.e4m3_decode(codes[r]), scales=s,
                               hhat=O.dequant_intermediate("fp8", codes[r][None], s[None], I)[0])
+            return out
+        if fmt == "mxfp8":
+            codes = self.codes[: R_total * I].reshape(R_total, I)
+            kc = I // 128
+            j = np.arange(I // 32)
+            for r in rows:
+                _, pr = row_scale_positions(self.lay_h, r)
+                off = ((pr >> 7) * kc + (j >> 2)) * 512 + (pr & 31) * 16 + ((pr >> 5) & 3) * 4 + (j & 3)
+                s = self.scales[off].copy()
+                out[r] = dict(codes=codes[r], values=F.e4m3_decode(codes[r]), scales=s,
+                              hhat=O.dequant_intermediate("mxfp8", codes[r][None], s[None], I)[0])
             return out
         codes = self.codes[: R_total * I // 2].reshape(R_total, I // 2)
         kc = I // 64
@@ -248,6 +260,32 @@ def _compare_codes(p, host, e, it, g, stats):
         assert np.all(np.abs(s_g - s_o) <= SCALE_REL * np.abs(s_o)), \
             f"FP8 block scales differ: {s_g} vs {s_o}"
         ref_vals = F.e4m3_decode(it["codes"])
+    elif fmt == "mxfp8":
+        table = "e4m3"
+        ref_vals = F.e4m3_decode(it["codes"]).astype(np.float64)
+        sc_o = np.asarray(it["scales"], np.int64)
+        sc_g = np.asarray(g["scales"], np.int64)
+        sdiff = sc_o != sc_g
+        if sdiff.any():
+            # a scale may differ only by one step, where the block's amax is
+            # within MID_REL of the power of two that separates the two
+            amax = np.max(np.abs(np.asarray(it["h32"], np.float64).reshape(I // 32, 32)), axis=1)
+            edge = np.ldexp(1.0, np.maximum(sc_o, sc_g) - 127 + 8)
+            ok = (np.abs(sc_g - sc_o) == 1) & (np.abs(amax - edge) <= MID_REL * edge)
+            ok = ok[sdiff]
+            assert ok.all(), f"MXFP8 block scale differs beyond a power-of-two edge: {sc_g[sdiff][~ok]} vs {sc_o[sdiff][~ok]}"
+            stats["scale_flips"] += int(sdiff.sum())
+            flipped = True
+            # the block's codes follow the GPU's scale: re-derive the oracle's
+            h32 = np.asarray(it["h32"], np.float64).reshape(I // 32, 32)
+            ref_vals = ref_vals.reshape(I // 32, 32).copy()
+            pre = pre.reshape(I // 32, 32).copy()
+            for b in np.nonzero(sdiff)[0]:
+                v = h32[b] * np.ldexp(1.0, 127 - int(sc_g[b]))
+                ref_vals[b] = F.e4m3_decode(F.e4m3_encode(v))
+                pre[b] = v
+            ref_vals = ref_vals.reshape(I)
+            pre = pre.reshape(I)
     else:
         table = "e2m1"
         ref_vals = F.e2m1_decode(F.fp4_unpack(np.asarray(it["codes"])[None], I)[0]).astype(np.float64)
@@ -282,8 +320,8 @@ def _compare_codes(p, host, e, it, g, stats):
     diff = got_vals != ref_vals
     stats["code_vals"] += diff.size
     if diff.any():
-        # quantisation blocks: the whole row (BF16), 128 (FP8) or 16 (NVFP4) values
-        scale = block_max(pre, {"bf16": I, "fp8": 128, "nvfp4": 16}[fmt])
+        # quantisation blocks: the whole row (BF16), 128 (FP8), 16 (NVFP4) or 32 (MXFP8) values
+        scale = block_max(pre, {"bf16": I, "fp8": 128, "nvfp4": 16, "mxfp8": 32}[fmt])
         ok = rounding_of_nearby(table, got_vals[diff], pre[diff], scale[diff])
         assert ok.all(), (f"{fmt} intermediate codes are not a rounding of the oracle's value: GPU "
                           f"{got_vals[diff][~ok][:8]} oracle {ref_vals[diff][~ok][:8]} "

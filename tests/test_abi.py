@@ -57,6 +57,8 @@ def _prob(**kw):
     (dict(format="nvfp4", intermediate_hidden=384), api.MOE_ERR_UNSUPPORTED),
     (dict(tile_regime=3), api.MOE_ERR_INVALID_ARG),
     (dict(format="nvfp4", tile_regime="small_m"), api.MOE_ERR_UNSUPPORTED),
+    (dict(format="mxfp8", tile_regime="small_m"), api.MOE_ERR_UNSUPPORTED),
+    (dict(format=4), api.MOE_ERR_INVALID_ARG),
 ])
 def test_geometry_validation(lib, kw, code):
     n = ctypes.c_size_t(0)
@@ -65,12 +67,13 @@ def test_geometry_validation(lib, kw, code):
 
 
 def test_valid_geometry_and_sizes(lib):
-    for fmt, eb in (("bf16", 2.0), ("fp8", 1.0), ("nvfp4", 0.5)):
+    for fmt, eb in (("bf16", 2.0), ("fp8", 1.0), ("nvfp4", 0.5), ("mxfp8", 1.0)):
         p = _prob(format=fmt, hidden=512, intermediate_hidden=256)
         assert api.workspace_size(p) > 0
         a, b = api.prepared_weights_size(p)
-        # the prepared blobs hold exactly the weights (+ NVFP4 scales, 1/16 byte per element... 1 per 16)
-        extra = 1.0 / 16 if fmt == "nvfp4" else 0.0
+        # the prepared blobs hold exactly the weights plus their block scales:
+        # one byte per 16 elements (NVFP4) or per 32 (MXFP8)
+        extra = {"nvfp4": 1.0 / 16, "mxfp8": 1.0 / 32}.get(fmt, 0.0)
         assert a == int(8 * 2 * 256 * 512 * (eb + extra))
         assert b == int(8 * 512 * 256 * (eb + extra))
         n, off = api.intermediate_size(p)
@@ -129,5 +132,6 @@ def test_tile_regime_resolution(lib):
     assert api.tile_regime(_prob(num_tokens=256, format="fp8", num_experts=8, num_topk=2)) == "small_m"
     assert api.tile_regime(_prob(num_tokens=16, format="nvfp4", intermediate_hidden=256, num_experts=8,
                                  num_topk=2)) == "large_m"
+    assert api.tile_regime(_prob(num_tokens=16, format="mxfp8", num_experts=8, num_topk=2)) == "large_m"
     assert api.tile_regime(_prob(num_tokens=16, tile_regime="large_m")) == "large_m"
     assert api.tile_regime(_prob(num_tokens=100000, tile_regime="small_m")) == "small_m"

@@ -3,7 +3,7 @@ unfused chain (moe_permute / moe_ffn / moe_combine) and through the single
 moe_fused launch -- whose layout, intermediate codes, FP32 accumulator and
 output are read back from its workspace and held to the same split-parity
 checks -- on small problems that span several tiles with ragged tails, and on
-the five full-size workloads in the launch configuration the benchmark times
+the full-size workloads in the launch configuration the benchmark times
 (sampled tokens, plus whole-problem layout and routing checks)."""
 
 import numpy as np
@@ -48,6 +48,8 @@ SMALL = [
     ("fp8", 700, 1024, 384, 3, 2),     # several m and n tiles, ragged
     ("nvfp4", 200, 512, 256, 6, 3),
     ("nvfp4", 333, 1024, 512, 5, 2),
+    ("mxfp8", 200, 512, 256, 6, 3),
+    ("mxfp8", 700, 1024, 384, 3, 2),   # several m and n tiles, ragged
 ]
 
 
@@ -60,7 +62,7 @@ def test_ffn_parity_small(fmt, M, H, I, E, k):
 
 
 @pytest.mark.parametrize("regime", ["large_m", "small_m"])
-@pytest.mark.parametrize("fmt,M,H,I,E,k", [c for c in SMALL if c[0] != "nvfp4"])
+@pytest.mark.parametrize("fmt,M,H,I,E,k", [c for c in SMALL if c[0] in ("bf16", "fp8")])
 def test_ffn_parity_both_tile_regimes(fmt, M, H, I, E, k, regime):
     """Both GEMM tile regimes (128 routed rows x 256 weight rows, and the
     swapped operands with 32 routed rows) on every BF16 / FP8 case, through
@@ -73,7 +75,7 @@ def test_ffn_parity_both_tile_regimes(fmt, M, H, I, E, k, regime):
 
 
 @pytest.mark.parametrize("fmt,regime", [("bf16", "large_m"), ("fp8", "large_m"), ("nvfp4", "large_m"),
-                                        ("bf16", "small_m"), ("fp8", "small_m")])
+                                        ("mxfp8", "large_m"), ("bf16", "small_m"), ("fp8", "small_m")])
 def test_staged_mode_and_deterministic_combine(fmt, regime):
     """Staged rows + the deterministic gather-combine meet the format's own
     tolerance; the combine gives the same bytes twice."""
@@ -93,7 +95,7 @@ def test_staged_mode_and_deterministic_combine(fmt, regime):
     assert torch.equal(o1, o2)
 
 
-@pytest.mark.parametrize("fmt", ["bf16", "fp8", "nvfp4"])
+@pytest.mark.parametrize("fmt", ["bf16", "fp8", "nvfp4", "mxfp8"])
 def test_clamp_active(fmt):
     """Weights scaled up so that more than 20% of g and u pass +-c: the clamp
     is exercised in every format, chain and single launch."""
@@ -106,6 +108,9 @@ def test_clamp_active(fmt):
         host["w13"] = d["w13"].cpu().view(torch.int16).numpy().view(np.uint16)
     elif fmt == "fp8":
         d["w13_scale"] = d["w13_scale"] * 60
+        host["w13_scale"] = d["w13_scale"].cpu().numpy()
+    elif fmt == "mxfp8":
+        d["w13_scale"] = d["w13_scale"] + 6        # x 64
         host["w13_scale"] = d["w13_scale"].cpu().numpy()
     else:
         d["gate_up_expert_scales"] = d["gate_up_expert_scales"] * 60
@@ -121,7 +126,7 @@ def test_clamp_active(fmt):
     _check_both_paths(p, d, host, L, np.arange(M), f"clamp/{fmt}")
 
 
-@pytest.mark.parametrize("fmt", ["bf16", "fp8", "nvfp4"])
+@pytest.mark.parametrize("fmt", ["bf16", "fp8", "nvfp4", "mxfp8"])
 def test_skipped_and_duplicate_slots(fmt):
     M, H, I, E, k = 40, 512, 256, 3, 3
     p = _small(fmt, M, H, I, E, k)
@@ -135,7 +140,7 @@ def test_skipped_and_duplicate_slots(fmt):
     _check_both_paths(p, d, host, L, np.arange(M), f"skip/dup/{fmt}")
 
 
-@pytest.mark.parametrize("fmt", ["bf16", "fp8", "nvfp4"])
+@pytest.mark.parametrize("fmt", ["bf16", "fp8", "nvfp4", "mxfp8"])
 def test_all_tokens_one_expert_and_single_expert(fmt):
     for E, k in ((1, 1), (4, 1)):
         M, H, I = 260, 512, 256
@@ -151,7 +156,8 @@ def test_all_tokens_one_expert_and_single_expert(fmt):
 
 
 @pytest.mark.parametrize("name,ntok", [("tiny_bf16", 16), ("fp8_block", 96), ("nvfp4_decode", 24),
-                                       ("nvfp4_prefill", 24), ("fp8_prefill_routed", 48)])
+                                       ("nvfp4_prefill", 24), ("fp8_prefill_routed", 48),
+                                       ("mxfp8_prefill_routed", 48)])
 def test_full_size_workloads_sampled(name, ntok):
     """The full-size workloads through moe_fused, the launch the benchmark
     times: routing (in-kernel for the logits workload) and the whole layout
