@@ -107,11 +107,9 @@ def stored_traffic(workload, kernel):
             rec = json.load(f)[workload]
     except Exception:
         return None
-    # sources_sha: the kernel sources the counters were taken on; later
-    # sources whose diff against them touches comments only are listed in
-    # sources_sha_same_code
-    shas = [rec.get("sources_sha")] + list(rec.get("sources_sha_same_code", []))
-    if rec.get("kernel") != kernel or kernel_sources_sha() not in shas:
+    # sources_sha: the kernel sources the counters were taken on; any later
+    # change to them drops the figure
+    if rec.get("kernel") != kernel or kernel_sources_sha() != rec.get("sources_sha"):
         return None
     return float(rec["dram_bytes_per_launch"])
 
