@@ -367,12 +367,28 @@ def _expert_scale(inputs, name, e):
     return None if arr is None else np.asarray(arr, np.float32)[e]
 
 
+def shared_expert_slots(topk_idx, topk_weights, num_experts):
+    """EPConfig fused_shared_expert / DistributedEPCombine fused_shared_expert:
+    the shared expert's computation is fused with the routed experts'.  Read
+    as one more expert, index num_experts (after the routed ones, same shapes),
+    that every token goes through with router weight 1: each token's slot list
+    gains a last column (num_experts, 1.0) after its k routed slots."""
+    idx = np.asarray(topk_idx, np.int64)
+    w = np.asarray(topk_weights, np.float32)
+    M = idx.shape[0]
+    return (np.concatenate([idx, np.full((M, 1), num_experts, np.int64)], axis=1),
+            np.concatenate([w, np.ones((M, 1), np.float32)], axis=1))
+
+
 def moe_forward(problem, inputs, topk_idx, topk_weights, tokens=None,
                 keep_intermediate=False, hhat_override=None):
     """The routed MoE FFN by its per-token definition.
 
     problem: dict(hidden, intermediate_hidden, num_experts, num_topk,
-                  activation_clamp, format)
+                  activation_clamp, format, optional shared_expert)
+             With shared_expert = 1 the weights hold num_experts + 1 experts
+             (the last one shared) and topk_idx / topk_weights carry the
+             shared slot (shared_expert_slots).
     inputs:  dict(x, x_scale, w13, w13_scale, w2, w2_scale,
                   gate_up_expert_scales, down_expert_scales, c_input_scales,
                   and for NVFP4 quantised per token, x_row_scale: BF16 [M])
@@ -388,7 +404,7 @@ def moe_forward(problem, inputs, topk_idx, topk_weights, tokens=None,
     fmt = problem["format"]
     H = problem["hidden"]
     I = problem["intermediate_hidden"]
-    E = problem["num_experts"]
+    E = problem["num_experts"] + int(problem.get("shared_expert", 0))
     clamp = problem.get("activation_clamp", 10.0)
     idx = np.asarray(topk_idx, np.int64)
     w = np.asarray(topk_weights, np.float32).astype(np.float64)
