@@ -100,7 +100,22 @@ typedef enum {
 
 /* The problem statement, after flashinfer.megamoe.MegaMoESymmBuffer
  * (num_experts, num_topk, hidden, intermediate_hidden, activation_clamp,
- * fast_math), plus the GEMM tile regime. */
+ * fast_math), plus the GEMM tile regime and the shared expert.
+ *
+ * shared_expert = 1 (EPConfig fused_shared_expert; DistributedEPCombine
+ * fused_shared_expert): the shared expert's computation is fused with the
+ * routed experts'.  It is expert index num_experts, after the routed ones,
+ * with their shapes and formats, and every token goes through it with
+ * router weight 1 in the same grouped GEMMs.  Then:
+ *   - every weight array and per-expert array holds num_experts + 1
+ *     experts, the shared one last;
+ *   - every per-token slot array (topk_idx, topk_weights, and the rows of
+ *     the layout) has num_topk + 1 columns, the last being (num_experts,
+ *     1.0): moe_route and moe_fused's in-kernel routing choose num_topk of
+ *     the num_experts routed experts and write that column themselves;
+ *     callers passing precomputed routing pass it too;
+ *   - sizes, layouts and the tile regime are those of the problem with
+ *     num_experts + 1 experts and num_topk + 1 slots. */
 typedef struct {
   int64_t num_tokens;           /* M >= 0 */
   int32_t hidden;               /* H, multiple of 256 */
@@ -111,6 +126,7 @@ typedef struct {
   int32_t format;               /* moe_format_t */
   int32_t fast_math;            /* nonzero: the SiLU uses the fast exponential */
   int32_t tile_regime;          /* moe_tile_regime_t: the grouped GEMMs' tile shape */
+  int32_t shared_expert;        /* 0, or 1: a fused shared expert (above) */
 } moe_problem_t;
 
 /* Tile shape of the grouped GEMMs (the tile-regime choice the pages make

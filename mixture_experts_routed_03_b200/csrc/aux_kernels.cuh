@@ -25,8 +25,10 @@ struct RouteArgs {
   const float* bias;     // [E] or null
   int64_t M;
   int E, k;
-  int64_t* idx_out;      // [M][k]
-  float* w_out;          // [M][k]
+  int64_t* idx_out;      // [M][out_k]
+  float* w_out;          // [M][out_k]
+  int out_k;             // k, or k + 1 with a shared expert
+  int shared;            // 1: column k is the shared expert (index E, weight 1)
 };
 
 __device__ __forceinline__ uint64_t route_key(float s, int e) {
@@ -86,8 +88,12 @@ __device__ __forceinline__ void route_token(const RouteArgs& a, int64_t t, const
 #pragma unroll
   for (int off = 16; off; off >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, off);
   if (mine) {
-    a.idx_out[t * a.k + lane] = my_e;
-    a.w_out[t * a.k + lane] = __fdiv_rn(ex, sum);
+    a.idx_out[t * a.out_k + lane] = my_e;
+    a.w_out[t * a.out_k + lane] = __fdiv_rn(ex, sum);
+  }
+  if (a.shared && lane == 0) {
+    a.idx_out[t * a.out_k + a.k] = a.E;
+    a.w_out[t * a.out_k + a.k] = 1.0f;
   }
 }
 

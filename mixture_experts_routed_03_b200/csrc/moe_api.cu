@@ -39,19 +39,35 @@ moe_status_t check_problem(const moe_problem_t* p) {
   if (p->hidden <= 0 || p->hidden % 256 != 0) return MOE_ERR_INVALID_ARG;
   if (p->intermediate_hidden <= 0 || p->intermediate_hidden % 128 != 0) return MOE_ERR_INVALID_ARG;
   if (p->num_experts < 1 || p->num_topk < 1 || p->num_topk > p->num_experts) return MOE_ERR_INVALID_ARG;
-  if (p->num_experts > 1024) return MOE_ERR_UNSUPPORTED;
+  if (p->shared_expert != 0 && p->shared_expert != 1) return MOE_ERR_INVALID_ARG;
+  // with a shared expert: num_experts + 1 experts, num_topk + 1 slots per token
+  const int E_all = p->num_experts + p->shared_expert;
+  const int k_all = p->num_topk + p->shared_expert;
+  if (E_all > 1024) return MOE_ERR_UNSUPPORTED;
   if (std::isnan(p->activation_clamp) || !(p->activation_clamp > 0.0f)) return MOE_ERR_INVALID_ARG;
   if (p->tile_regime < MOE_TILE_AUTO || p->tile_regime > MOE_TILE_SMALL_M) return MOE_ERR_INVALID_ARG;
   if (p->tile_regime == MOE_TILE_SMALL_M && (p->format == MOE_FMT_NVFP4 || p->format == MOE_FMT_MXFP8))
     return MOE_ERR_UNSUPPORTED;
   if (p->format == MOE_FMT_NVFP4 && p->intermediate_hidden % 256 != 0) return MOE_ERR_UNSUPPORTED;
-  const int64_t R = p->num_tokens * p->num_topk;
+  const int64_t R = p->num_tokens * k_all;
   if (R > (int64_t(1) << 30)) return MOE_ERR_UNSUPPORTED;
   // expert weight row indices are 32-bit in the TMA coordinates
-  if (int64_t(p->num_experts) * 2 * p->intermediate_hidden >= (int64_t(1) << 31) ||
-      int64_t(p->num_experts) * p->hidden >= (int64_t(1) << 31))
+  if (int64_t(E_all) * 2 * p->intermediate_hidden >= (int64_t(1) << 31) ||
+      int64_t(E_all) * p->hidden >= (int64_t(1) << 31))
     return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
+}
+
+// The problem every step after the routing works on: a fused shared expert
+// (EPConfig fused_shared_expert) is one more expert, index num_experts, and
+// one more slot per token, its last column, so the permutation, the GEMMs
+// and the combine treat it as a routed expert that every token chose.
+moe_problem_t effective(const moe_problem_t* p) {
+  moe_problem_t q = *p;
+  q.num_experts += p->shared_expert;
+  q.num_topk += p->shared_expert;
+  q.shared_expert = 0;
+  return q;
 }
 
 // ---------------------------------------------------------------- workspace
@@ -307,6 +323,8 @@ RouteArgs route_args(const moe_problem_t* p, const float* logits, const float* b
   a.k = p->num_topk;
   a.idx_out = idx;
   a.w_out = w;
+  a.shared = p->shared_expert;
+  a.out_k = p->num_topk + p->shared_expert;
   return a;
 }
 
@@ -644,6 +662,8 @@ moe_status_t moe_init(int device) {
 moe_status_t moe_get_workspace_offsets(const moe_problem_t* p, moe_workspace_offsets_t* o) {
   moe_status_t s = check_problem(p);
   if (s != MOE_OK) return s;
+  const moe_problem_t pe = effective(p);
+  p = &pe;
   if (!o) return MOE_ERR_INVALID_ARG;
   const WsLayout L = make_layout(p);
   o->status = L.header;
@@ -667,6 +687,8 @@ moe_status_t moe_get_workspace_offsets(const moe_problem_t* p, moe_workspace_off
 moe_status_t moe_get_workspace_size(const moe_problem_t* p, size_t* bytes) {
   moe_status_t s = check_problem(p);
   if (s != MOE_OK) return s;
+  const moe_problem_t pe = effective(p);
+  p = &pe;
   if (!bytes) return MOE_ERR_INVALID_ARG;
   *bytes = make_layout(p).total;
   return MOE_OK;
@@ -675,6 +697,8 @@ moe_status_t moe_get_workspace_size(const moe_problem_t* p, size_t* bytes) {
 moe_status_t moe_get_tile_regime(const moe_problem_t* p, int32_t* regime) {
   moe_status_t s = check_problem(p);
   if (s != MOE_OK) return s;
+  const moe_problem_t pe = effective(p);
+  p = &pe;
   if (!regime) return MOE_ERR_INVALID_ARG;
   *regime = small_m_tiles(p) ? MOE_TILE_SMALL_M : MOE_TILE_LARGE_M;
   return MOE_OK;
@@ -683,6 +707,8 @@ moe_status_t moe_get_tile_regime(const moe_problem_t* p, int32_t* regime) {
 moe_status_t moe_get_intermediate_size(const moe_problem_t* p, size_t* bytes, size_t* scale_offset) {
   moe_status_t s = check_problem(p);
   if (s != MOE_OK) return s;
+  const moe_problem_t pe = effective(p);
+  p = &pe;
   if (!bytes || !scale_offset) return MOE_ERR_INVALID_ARG;
   const WsLayout L = make_layout(p);
   *scale_offset = align_up(std::max<size_t>(L.h_bytes, 1), kAlign);
@@ -709,6 +735,8 @@ moe_status_t moe_workspace_test_hooks(void* ws, size_t ws_bytes, int32_t wait_li
 moe_status_t moe_get_prepared_weights_size(const moe_problem_t* p, size_t* w13_bytes, size_t* w2_bytes) {
   moe_status_t s = check_problem(p);
   if (s != MOE_OK) return s;
+  const moe_problem_t pe = effective(p);
+  p = &pe;
   if (!w13_bytes || !w2_bytes) return MOE_ERR_INVALID_ARG;
   *w13_bytes = prepared_bytes(p, true);
   *w2_bytes = prepared_bytes(p, false);
@@ -719,6 +747,8 @@ moe_status_t moe_prepare_weights(const moe_problem_t* p, const moe_weights_t* lo
                                  void* out_w2, void* stream) {
   moe_status_t s = check_problem(p);
   if (s != MOE_OK) return s;
+  const moe_problem_t pe = effective(p);
+  p = &pe;
   if (!logical || !logical->w13 || !logical->w2 || !out_w13 || !out_w2) return MOE_ERR_INVALID_ARG;
   if (!aligned16(logical->w13) || !aligned16(logical->w2) || !aligned16(out_w13) || !aligned16(out_w2))
     return MOE_ERR_INVALID_ARG;
@@ -796,6 +826,8 @@ moe_status_t moe_permute(const moe_problem_t* p, const int64_t* topk_idx, const 
                          size_t ws_bytes, void* stream) {
   moe_status_t s = check_problem(p);
   if (s != MOE_OK) return s;
+  const moe_problem_t pe = effective(p);
+  p = &pe;
   if (p->num_tokens == 0) return MOE_OK;
   if (!topk_idx || !layout_ok(layout) || !ws) return MOE_ERR_INVALID_ARG;
   const WsLayout L = make_layout(p);
@@ -815,6 +847,8 @@ moe_status_t moe_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_wei
                      void* intermediate, void* ws, size_t ws_bytes, void* stream) {
   moe_status_t s = check_problem(p);
   if (s != MOE_OK) return s;
+  const moe_problem_t pe = effective(p);
+  p = &pe;
   if (out_mode != MOE_OUT_ACCUMULATE && out_mode != MOE_OUT_STAGED) return MOE_ERR_INVALID_ARG;
   if (p->num_tokens == 0) return MOE_OK;
   if ((s = check_act_weights(p, act, w)) != MOE_OK) return s;
@@ -850,6 +884,8 @@ moe_status_t moe_combine(const moe_problem_t* p, const moe_layout_t* layout, con
                          const void* in, int32_t in_mode, void* out_bf16, void* stream) {
   moe_status_t s = check_problem(p);
   if (s != MOE_OK) return s;
+  const moe_problem_t pe = effective(p);
+  p = &pe;
   if (in_mode != MOE_IN_ACCUMULATED && in_mode != MOE_IN_STAGED) return MOE_ERR_INVALID_ARG;
   if (p->num_tokens == 0) return MOE_OK;
   if (!in || !out_bf16 || !aligned16(in) || !aligned16(out_bf16)) return MOE_ERR_INVALID_ARG;
@@ -874,12 +910,17 @@ moe_status_t moe_fused(const moe_problem_t* p, const moe_act_t* act, const moe_w
                        const float* bias, void* out_bf16, void* ws, size_t ws_bytes, void* stream) {
   moe_status_t s = check_problem(p);
   if (s != MOE_OK) return s;
+  // the routing chooses among the routed experts; every later step works on
+  // the effective problem (a shared expert is one more expert and slot)
+  const moe_problem_t* p_route = p;
+  const moe_problem_t pe = effective(p);
+  p = &pe;
   if (p->num_tokens == 0) return MOE_OK;
   if ((s = check_act_weights(p, act, w)) != MOE_OK) return s;
   const bool pre = topk_idx != nullptr && topk_weights != nullptr;
   const bool from_logits = logits != nullptr;
   if (pre == from_logits || (!pre && (topk_idx || topk_weights))) return MOE_ERR_INVALID_ARG;
-  if (from_logits && p->num_topk > 32) return MOE_ERR_UNSUPPORTED;
+  if (from_logits && p_route->num_topk > 32) return MOE_ERR_UNSUPPORTED;
   if (!out_bf16 || !aligned16(out_bf16) || !ws) return MOE_ERR_INVALID_ARG;
   const WsLayout L = make_layout(p);
   if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
@@ -893,7 +934,7 @@ moe_status_t moe_fused(const moe_problem_t* p, const moe_act_t* act, const moe_w
   if (from_logits) {
     int64_t* ridx = reinterpret_cast<int64_t*>(base + L.route_idx);
     float* rw = reinterpret_cast<float*>(base + L.route_w);
-    f.route = route_args(p, logits, bias, ridx, rw);
+    f.route = route_args(p_route, logits, bias, ridx, rw);
     f.do_route = 1;
     idx = ridx;
     wts = rw;
@@ -961,6 +1002,8 @@ moe_status_t moe_permute_noalloc(const moe_problem_t* p, const int64_t* topk_idx
                                  int32_t* device_status, void* stream) {
   moe_status_t s = check_problem(p);
   if (s != MOE_OK) return s;
+  const moe_problem_t pe = effective(p);
+  p = &pe;
   if (p->num_tokens == 0) return MOE_OK;
   if (!topk_idx || !layout_ok(layout) || !device_status) return MOE_ERR_INVALID_ARG;
   const int64_t R = p->num_tokens * p->num_topk;

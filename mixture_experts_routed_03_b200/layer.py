@@ -55,6 +55,11 @@ class MoELayer:
         self.fast_math = fast_math
         api.init(self.device.index if self.device.index is not None else 0)
         self.max_tokens = int(p["num_tokens"])
+        # a fused shared expert (p["shared_expert"] = 1) is one more expert
+        # and one more slot per token after the routing
+        self.shared = int(p.get("shared_expert", 0))
+        self.k_all = int(p["num_topk"]) + self.shared
+        self.E_all = int(p["num_experts"]) + self.shared
         self.prob = api.problem_from_dict(self.p, fast_math=fast_math)
         w = weights
         self.alpha1 = w.get("gate_up_expert_scales")
@@ -100,9 +105,22 @@ class MoELayer:
         api.quantize_nvfp4_rowwise(self.problem(M), x_bf16, codes, scales, rowwise, stream=stream)
         return codes, scales, rowwise
 
+    def shared_slots(self, topk_idx, topk_weights):
+        """Precomputed routing [M, k] -> [M, k + 1]: the shared expert's slot
+        (index num_experts, weight 1) appended, as every call after the
+        routing expects when the layer has a shared expert."""
+        if not self.shared:
+            return topk_idx, topk_weights
+        M = topk_idx.shape[0]
+        idx = torch.cat([topk_idx, torch.full((M, 1), self.p["num_experts"], dtype=topk_idx.dtype,
+                                              device=topk_idx.device)], dim=1)
+        w = torch.cat([topk_weights, torch.ones((M, 1), dtype=topk_weights.dtype, device=topk_weights.device)],
+                      dim=1)
+        return idx.contiguous(), w.contiguous()
+
     def route(self, logits, bias=None, stream=None):
         M = logits.shape[0]
-        k = self.p["num_topk"]
+        k = self.k_all
         idx = torch.empty((M, k), dtype=torch.int64, device=self.device)
         w = torch.empty((M, k), dtype=torch.float32, device=self.device)
         api.route(self.problem(M), logits, bias, idx, w, stream=stream)
@@ -110,7 +128,7 @@ class MoELayer:
 
     def permute(self, topk_idx, stream=None):
         M = topk_idx.shape[0]
-        lay = LayoutBuffers(M, self.p["num_topk"], self.p["num_experts"], self.device)
+        lay = LayoutBuffers(M, self.k_all, self.E_all, self.device)
         api.permute(self.problem(M), topk_idx, lay.struct, self.ws, self.ws_bytes, stream=stream)
         return lay
 
@@ -120,7 +138,7 @@ class MoELayer:
         M = x.shape[0]
         prob = self.problem(M)
         H = self.p["hidden"]
-        rows = M if out_mode == api.MOE_OUT_ACCUMULATE else M * self.p["num_topk"]
+        rows = M if out_mode == api.MOE_OUT_ACCUMULATE else M * self.k_all
         out = torch.empty((rows, H), dtype=torch.float32, device=self.device)
         inter = None
         if keep_intermediate:
@@ -143,7 +161,7 @@ class MoELayer:
         Read them only after that call has completed."""
         prob = self.problem(M)
         off = api.workspace_offsets(prob)
-        k, E, H = self.p["num_topk"], self.p["num_experts"], self.p["hidden"]
+        k, E, H = self.k_all, self.E_all, self.p["hidden"]
         R = M * k
         n_int, so = api.intermediate_size(prob)
         ws = self.ws

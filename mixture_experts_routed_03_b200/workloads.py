@@ -143,40 +143,43 @@ def make_inputs(p, seed=0, device="cpu"):
     g = _gen(device, seed)
     fmt = p["format"]
     M, H, I, E = p["num_tokens"], p["hidden"], p["intermediate_hidden"], p["num_experts"]
+    # experts whose weights are drawn: the routed ones, then a shared expert
+    # (EPConfig fused_shared_expert) if the problem has one
+    Ew = E + int(p.get("shared_expert", 0))
     d = {}
     if fmt == "bf16":
         d["x"] = _bf16_codes((M, H), BF16_X_STD, g, device)
-        d["w13"] = _bf16_codes((E, 2 * I, H), W_STD, g, device)
-        d["w2"] = _bf16_codes((E, H, I), W_STD, g, device)
+        d["w13"] = _bf16_codes((Ew, 2 * I, H), W_STD, g, device)
+        d["w2"] = _bf16_codes((Ew, H, I), W_STD, g, device)
         d["x_scale"] = d["w13_scale"] = d["w2_scale"] = None
     elif fmt == "fp8":
         d["x"] = _e4m3_codes((M, H), g, device)
         d["x_scale"] = _uniform((M, H // 128), 0.5, 1.5, g, device) * (X_STD / FP8_CODE_STD)
-        d["w13"] = torch.empty((E, 2 * I, H), dtype=torch.uint8, device=device)
-        d["w2"] = torch.empty((E, H, I), dtype=torch.uint8, device=device)
-        for e in range(E):                       # per expert: bounded host memory
+        d["w13"] = torch.empty((Ew, 2 * I, H), dtype=torch.uint8, device=device)
+        d["w2"] = torch.empty((Ew, H, I), dtype=torch.uint8, device=device)
+        for e in range(Ew):                       # per expert: bounded host memory
             d["w13"][e] = _e4m3_codes((2 * I, H), g, device)
             d["w2"][e] = _e4m3_codes((H, I), g, device)
-        d["w13_scale"] = _uniform((E, 2 * I // 128, H // 128), 0.5, 1.5, g, device) * (W_STD / FP8_CODE_STD)
-        d["w2_scale"] = _uniform((E, H // 128, I // 128), 0.5, 1.5, g, device) * (W_STD / FP8_CODE_STD)
+        d["w13_scale"] = _uniform((Ew, 2 * I // 128, H // 128), 0.5, 1.5, g, device) * (W_STD / FP8_CODE_STD)
+        d["w2_scale"] = _uniform((Ew, H // 128, I // 128), 0.5, 1.5, g, device) * (W_STD / FP8_CODE_STD)
     elif fmt == "nvfp4":
         d["x"] = _fp4_bytes((M, H // 2), g, device)
         d["x_scale"] = _e4m3_positive((M, H // 16), 0.5, 1.5, g, device)
-        d["w13"] = _fp4_bytes((E, 2 * I, H // 2), g, device)
-        d["w13_scale"] = _e4m3_positive((E, 2 * I, H // 16), 0.5, 1.5, g, device)
-        d["w2"] = _fp4_bytes((E, H, I // 2), g, device)
-        d["w2_scale"] = _e4m3_positive((E, H, I // 16), 0.5, 1.5, g, device)
+        d["w13"] = _fp4_bytes((Ew, 2 * I, H // 2), g, device)
+        d["w13_scale"] = _e4m3_positive((Ew, 2 * I, H // 16), 0.5, 1.5, g, device)
+        d["w2"] = _fp4_bytes((Ew, H, I // 2), g, device)
+        d["w2_scale"] = _e4m3_positive((Ew, H, I // 16), 0.5, 1.5, g, device)
         # Per-tensor activation global and per-expert weight globals, as
         # dequant multipliers; the layer takes their products per expert.
         x_global = X_STD / FP4_CODE_RMS
-        w13_global = _uniform((E,), 0.8, 1.2, g, device) * (W_STD / FP4_CODE_RMS)
-        w2_global = _uniform((E,), 0.8, 1.2, g, device) * (W_STD / FP4_CODE_RMS)
+        w13_global = _uniform((Ew,), 0.8, 1.2, g, device) * (W_STD / FP4_CODE_RMS)
+        w2_global = _uniform((Ew,), 0.8, 1.2, g, device) * (W_STD / FP4_CODE_RMS)
         # Static per-expert re-quant scale (a checkpoint-style calibration):
         # with the clamp c, |h| < c*c, so 2688 * G >= c*c never saturates the
         # E4M3 block scale.  Without a clamp a fixed bound of 1000 stands in.
         c = float(p.get("activation_clamp", 10.0))
         bound = c * c if math.isfinite(c) else 1000.0
-        c_in = _uniform((E,), 1.0, 1.2, g, device) * (bound / 2688.0)
+        c_in = _uniform((Ew,), 1.0, 1.2, g, device) * (bound / 2688.0)
         d["gate_up_expert_scales"] = (w13_global * x_global).to(torch.float32)
         d["down_expert_scales"] = (w2_global * c_in).to(torch.float32)
         d["c_input_scales"] = c_in.to(torch.float32)
@@ -185,13 +188,13 @@ def make_inputs(p, seed=0, device="cpu"):
         # 120..122) and W_STD / FP8_CODE_STD ~ 2^-11.6 (codes 115..117)
         d["x"] = _e4m3_codes((M, H), g, device)
         d["x_scale"] = _ue8m0_codes((M, H // 32), 120, 122, g, device)
-        d["w13"] = torch.empty((E, 2 * I, H), dtype=torch.uint8, device=device)
-        d["w2"] = torch.empty((E, H, I), dtype=torch.uint8, device=device)
-        for e in range(E):
+        d["w13"] = torch.empty((Ew, 2 * I, H), dtype=torch.uint8, device=device)
+        d["w2"] = torch.empty((Ew, H, I), dtype=torch.uint8, device=device)
+        for e in range(Ew):
             d["w13"][e] = _e4m3_codes((2 * I, H), g, device)
             d["w2"][e] = _e4m3_codes((H, I), g, device)
-        d["w13_scale"] = _ue8m0_codes((E, 2 * I, H // 32), 115, 117, g, device)
-        d["w2_scale"] = _ue8m0_codes((E, H, I // 32), 115, 117, g, device)
+        d["w13_scale"] = _ue8m0_codes((Ew, 2 * I, H // 32), 115, 117, g, device)
+        d["w2_scale"] = _ue8m0_codes((Ew, H, I // 32), 115, 117, g, device)
     else:
         raise ValueError(fmt)
     if p.get("act") == "bf16":

@@ -30,6 +30,16 @@ FLIP_FACTOR = 3.0
 L2_REL = 1e-3
 
 
+def k_all(p):
+    """Slots per token after the routing (a shared expert adds one)."""
+    return p["num_topk"] + int(p.get("shared_expert", 0))
+
+
+def e_all(p):
+    """Experts after the routing (a shared expert adds one)."""
+    return p["num_experts"] + int(p.get("shared_expert", 0))
+
+
 def device():
     return torch.device("cuda", 0)
 
@@ -140,7 +150,7 @@ class GpuResult:
         NVFP4 E4M3 codes, MXFP8 UE8M0 codes), hhat = dequantised row (float64,
         the L2 input)."""
         fmt, I = p["format"], p["intermediate_hidden"]
-        R_total = p["num_tokens"] * p["num_topk"]
+        R_total = p["num_tokens"] * k_all(p)
         out = {}
         if fmt == "bf16":
             codes = self.codes[: R_total * I * 2].view(np.uint16).reshape(R_total, I)
@@ -351,7 +361,7 @@ def check_against_oracle(p, host, res, tokens, label="", ref=None):
           FLIP_FACTOR * TOL * rms of the pure oracle.
     Returns a dict of statistics (flip counts, errors relative to rms)."""
     fmt = p["format"]
-    k = p["num_topk"]
+    k = k_all(p)
     tokens = np.asarray(tokens)
     if ref is None:
         ref = oracle_reference(p, host, tokens)

@@ -58,6 +58,9 @@ def _prob(**kw):
     (dict(tile_regime=3), api.MOE_ERR_INVALID_ARG),
     (dict(format="nvfp4", tile_regime="small_m"), api.MOE_ERR_UNSUPPORTED),
     (dict(format="mxfp8", tile_regime="small_m"), api.MOE_ERR_UNSUPPORTED),
+    (dict(shared_expert=2), api.MOE_ERR_INVALID_ARG),
+    (dict(shared_expert=-1), api.MOE_ERR_INVALID_ARG),
+    (dict(num_experts=1024, num_topk=2, shared_expert=1), api.MOE_ERR_UNSUPPORTED),
     (dict(format=4), api.MOE_ERR_INVALID_ARG),
 ])
 def test_geometry_validation(lib, kw, code):
@@ -135,3 +138,18 @@ def test_tile_regime_resolution(lib):
     assert api.tile_regime(_prob(num_tokens=16, format="mxfp8", num_experts=8, num_topk=2)) == "large_m"
     assert api.tile_regime(_prob(num_tokens=16, tile_regime="large_m")) == "large_m"
     assert api.tile_regime(_prob(num_tokens=100000, tile_regime="small_m")) == "small_m"
+
+
+def test_shared_expert_sizes_are_those_of_one_more_expert_and_slot(lib):
+    """A fused shared expert is one more expert and one more slot per token
+    after the routing: every size equals the plain problem's with E + 1 and
+    k + 1."""
+    for fmt in ("bf16", "fp8", "nvfp4", "mxfp8"):
+        kw = dict(format=fmt, hidden=512, intermediate_hidden=256, num_tokens=300)
+        shared = _prob(num_experts=8, num_topk=2, shared_expert=1, **kw)
+        plain = _prob(num_experts=9, num_topk=3, **kw)
+        assert api.workspace_size(shared) == api.workspace_size(plain)
+        assert api.prepared_weights_size(shared) == api.prepared_weights_size(plain)
+        assert api.intermediate_size(shared) == api.intermediate_size(plain)
+        assert api.workspace_offsets(shared) == api.workspace_offsets(plain)
+        assert api.tile_regime(shared) == api.tile_regime(plain)
