@@ -327,7 +327,7 @@ def mma_probe(fmt, achieved_tflops):
     try:
         from mixture_experts_routed_03_b200 import peak
         out = {}
-        for pair in (False, True) if fmt != "nvfp4" else (False,):
+        for pair in (False, True) if fmt in ("bf16", "fp8") else (False,):
             tf, cyc = peak.mma_peak(fmt, 256, pair, iters=20000)
             out["cta_pair" if pair else "one_cta"] = {"tflops": tf, "cycles_per_mma": cyc}
         best = max(v["tflops"] for v in out.values())

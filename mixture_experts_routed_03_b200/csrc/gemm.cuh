@@ -31,8 +31,8 @@
 // Roles: warp 0 lane 0 issues the copies into a 4-stage ring guarded by
 // mbarriers; warp 1 lane 0 issues the MMAs (M = 128, N = 256, four 32-byte K
 // steps per stage) and commits them; for NVFP4 and MXFP8, warp 2 lane 0 moves each
-// stage's scale factors from shared memory into one of two TMEM scale
-// buffers (tcgen05.cp), so their issue cost overlaps the MMAs; the last 8
+// stage's scale factors from shared memory into the stage's own TMEM scale
+// buffer (tcgen05.cp), so their issue cost overlaps the MMAs; the last 8
 // warps are the epilogue, two per 32-lane TMEM quarter, one per 128-column
 // half, one row per thread.
 //
@@ -77,11 +77,13 @@ constexpr int kSFBStage = 2 * 4 * kSFTile;    // 2 row blocks x 4 K-steps
 constexpr int kMxSFAStage = kSFTile;          // MXFP8: 4 scales (128 E4M3) per row
 constexpr int kMxSFBStage = 2 * kSFTile;      // MXFP8: 2 row blocks
 constexpr int kTmemCols = 512;
-// NVFP4 scale factors in TMEM: two buffers of 48 columns after the
-// accumulator, A scales (16 columns) then B scales (32 columns).  MXFP8 uses
-// the same buffers: A in columns 0..3, B in columns 16..23 of each.  (A ring of
-// four was measured no faster: the stage's twelve tcgen05.cp take ~600
-// cycles of the tensor pipe per K step whatever the ring depth.)
+// Block-scale factors in TMEM: one buffer of 48 columns per shared-memory
+// stage after the accumulator (4 x 48 + 256 <= 512).  NVFP4: A scales (16
+// columns) then B scales (32 columns); MXFP8: A in columns 0..3, B in
+// columns 16..23.  Buffer s belongs to stage s, so the copier needs no
+// release barrier: stage s's data lands only after the producer refilled
+// it, which it did only after the MMAs of the stage's previous use -- the
+// last readers of buffer s -- completed.
 constexpr int kSFCol0 = 256;
 constexpr int kSFBufCols = 48;
 constexpr int kSFBOff = 16;
@@ -340,9 +342,8 @@ __device__ __forceinline__ void gemm_phase(const GemmArgs& p, const CUtensorMap*
   uint64_t* acc_empty = acc_full + NACC;
   uint64_t* final_bar = acc_empty + NACC;
   uint64_t* xbar = final_bar + 1;  // FP8 L1: one per TMEM lane quarter
-  uint64_t* sf_full = xbar + 4;    // NVFP4: scale buffer b holds the current stage's scales
-  uint64_t* sf_empty = sf_full + 2;   // NVFP4: the MMAs reading scale buffer b completed
-  uint64_t* sf_final = sf_empty + 2;  // NVFP4: the copier's last copies completed
+  uint64_t* sf_full = xbar + 4;    // NVFP4 / MXFP8: scale buffer s holds stage s's scales
+  uint64_t* sf_final = sf_full + 4;   // NVFP4 / MXFP8: the copier's last copies completed
   uint64_t* hbar = sf_final + 1;      // FP8 L1: one per TMEM lane quarter (h rows staged)
   float* xbuf = reinterpret_cast<float*>(smem + S * SB + 1024);  // FP8 L1: [2][2][128] amax
   float* xpose = reinterpret_cast<float*>(smem + S * SB + Cfg::kBarrierBytes);  // L2: per-warp 32 x 32
@@ -361,10 +362,7 @@ __device__ __forceinline__ void gemm_phase(const GemmArgs& p, const CUtensorMap*
     }
     mbar_init(final_bar, 1);
     for (int i = 0; i < 4; ++i) mbar_init(&xbar[i], 64);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&sf_full[i], 1);
-      mbar_init(&sf_empty[i], 1);
-    }
+    for (int i = 0; i < S; ++i) mbar_init(&sf_full[i], 1);
     mbar_init(sf_final, 1);
     for (int i = 0; i < 4; ++i) mbar_init(&hbar[i], 64);
     fence_mbar_init();
@@ -434,8 +432,6 @@ __device__ __forceinline__ void gemm_phase(const GemmArgs& p, const CUtensorMap*
       int ab = 0;
       uint32_t aphase = 0;
       bool ok = true;
-      int sb = 0;
-      uint32_t sphase = 0;
       for (int T = cta; T < total && ok; T += ncta) {
         if (FMT != FMT_FP8) {
           if (!mbar_wait(&acc_empty[ab], aphase ^ 1u, abort_flag, p.status, 2)) break;
@@ -459,9 +455,9 @@ __device__ __forceinline__ void gemm_phase(const GemmArgs& p, const CUtensorMap*
           uint8_t* sbp = sa + kAStage;
           const uint64_t adesc = sdesc_sw128(smem_u32(sa));
           const uint64_t bdesc = sdesc_sw128(smem_u32(sbp));
-          const uint32_t sfa_t = tmem + kSFCol0 + kSFBufCols * sb;
+          const uint32_t sfa_t = tmem + kSFCol0 + kSFBufCols * stage;
           if (hw_scaled(FMT)) {
-            if (!mbar_wait(&sf_full[sb], sphase, abort_flag, p.status, 8)) {
+            if (!mbar_wait(&sf_full[stage], phase, abort_flag, p.status, 8)) {
               ok = false;
               break;
             }
@@ -479,13 +475,6 @@ __device__ __forceinline__ void gemm_phase(const GemmArgs& p, const CUtensorMap*
             else mma_mxf8(d, a, b, idesc_mxf8(kBN, kc), sfa_t, sfa_t + kSFBOff, acc);
           }
           mma_commit(&empty[stage]);
-          if (hw_scaled(FMT)) {
-            mma_commit(&sf_empty[sb]);
-            if (++sb == 2) {
-              sb = 0;
-              sphase ^= 1u;
-            }
-          }
           if (++stage == S) {
             stage = 0;
             phase ^= 1u;
@@ -515,19 +504,19 @@ __device__ __forceinline__ void gemm_phase(const GemmArgs& p, const CUtensorMap*
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      int sb = 0;
-      uint32_t sphase = 0;
       for (int T = cta; T < total; T += ncta) {
         bool ok = true;
         for (int ks = 0; ks < p.k_stages; ++ks) {
-          if (!mbar_wait(&full[stage], phase, abort_flag, p.status, 9) ||
-              !mbar_wait(&sf_empty[sb], sphase ^ 1u, abort_flag, p.status, 10)) {
+          // The stage's data has landed, so the MMAs that last read its scale
+          // buffer (the stage's previous use) have completed: the producer
+          // refilled the stage only after they released it.
+          if (!mbar_wait(&full[stage], phase, abort_flag, p.status, 9)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint32_t sfb_s = smem_u32(smem + stage * SB + kAStage + kBStage);
-          const uint32_t dst = tmem + kSFCol0 + kSFBufCols * sb;
+          const uint32_t dst = tmem + kSFCol0 + kSFBufCols * stage;
           if (FMT == FMT_NVFP4) {
             const uint32_t sfa_s = sfb_s + kSFBStage;
 #pragma unroll
@@ -542,11 +531,7 @@ __device__ __forceinline__ void gemm_phase(const GemmArgs& p, const CUtensorMap*
             tmem_copy_sf(dst + kSFBOff, sdesc_sf_tile(sfb_s));
             tmem_copy_sf(dst + kSFBOff + 4, sdesc_sf_tile(sfb_s + kSFTile));
           }
-          mma_commit(&sf_full[sb]);
-          if (++sb == 2) {
-            sb = 0;
-            sphase ^= 1u;
-          }
+          mma_commit(&sf_full[stage]);
           if (++stage == S) {
             stage = 0;
             phase ^= 1u;

@@ -12,7 +12,8 @@
 //
 // extern "C" moe_peak_mma(kind, n, pair, iters, scratch, stream, *tflops, *cycles)
 //   kind   0 BF16 (kind::f16), 1 E4M3 (kind::f8f6f4), 2 NVFP4
-//          (kind::mxf4nvf4.block_scale.scale_vec::4X; cta_group::1 only)
+//          (kind::mxf4nvf4.block_scale.scale_vec::4X; cta_group::1 only),
+//          3 MXFP8 (kind::mxf8f6f4.block_scale.scale_vec::1X; cta_group::1 only)
 //   iters  K blocks of 4 instructions each CTA (or pair) issues
 //   scratch device buffer of at least 16 bytes x grid (status, cycles)
 // Returns 0 on success; *tflops = dense FLOPs / event time over the whole
@@ -101,12 +102,17 @@ __global__ void __launch_bounds__(kPeakThreads, 1) mma_peak_kernel(int iters, in
       // issued by this thread ahead of its MMAs
       for (int t = 0; t < 12; ++t)
         tmem_copy_sf(tmem + 256 + 4 * t, sdesc_sf_tile(smem_u32(base + kOffSF + 512 * t)));
+    } else if (KIND == 3) {
+      // one scale tile for A (4 columns) and two for B's 256 rows, which
+      // serve all four K steps (byte kc of each word)
+      for (int t = 0; t < 3; ++t)
+        tmem_copy_sf(tmem + 256 + (t ? 12 + 4 * t : 0), sdesc_sf_tile(smem_u32(base + kOffSF + 512 * t)));
     }
     constexpr uint32_t M = PAIR ? 256 : 128;
     constexpr uint32_t idesc_m = (M >> 4) << 24;
     const uint32_t idesc = (KIND == 0)   ? ((idesc_dense(1, 1, N) & ~(31u << 24)) | idesc_m)
                            : (KIND == 1) ? ((idesc_dense(0, 0, N) & ~(31u << 24)) | idesc_m)
-                                         : idesc_nvf4(N);
+                                         : idesc_nvf4(N);   // (KIND 3 builds its own per K step)
     const uint64_t adesc = sdesc_sw128(smem_u32(base + kOffA));
     const uint64_t bdesc = sdesc_sw128(smem_u32(base + kOffB));
     t0 = clock64();
@@ -119,8 +125,10 @@ __global__ void __launch_bounds__(kPeakThreads, 1) mma_peak_kernel(int iters, in
           if (PAIR) mma_f16_pair(tmem, a, b, idesc); else mma_f16(tmem, a, b, idesc, 1u);
         } else if (KIND == 1) {
           if (PAIR) mma_f8_pair(tmem, a, b, idesc); else mma_f8(tmem, a, b, idesc, 1u);
-        } else {
+        } else if (KIND == 2) {
           mma_nvf4(tmem, a, b, idesc, tmem + 256 + 4 * kc, tmem + 256 + 16 + 8 * kc, 1u);
+        } else {
+          mma_mxf8(tmem, a, b, idesc_mxf8(N, kc), tmem + 256, tmem + 256 + 16, 1u);
         }
       }
     }
@@ -216,7 +224,7 @@ int run_peak(int iters, int* scratch, cudaStream_t st, float* tflops, float* cyc
     }
   }
   delete[] host;
-  const double k = (KIND == 0) ? 16.0 : (KIND == 1 ? 32.0 : 64.0);
+  const double k = (KIND == 0) ? 16.0 : (KIND == 2 ? 64.0 : 32.0);
   const double m = PAIR ? 256.0 : 128.0;
   const double issuers = PAIR ? grid / 2 : grid;
   const double flops = 2.0 * m * N * k * 4.0 * iters * issuers;
@@ -643,6 +651,7 @@ extern "C" int moe_peak_mma(int kind, int n, int pair, int iters, void* scratch,
   if (kind == 1 && n == 128 && pair) return run_peak<1, 128, true>(iters, s, st, tflops, cycles);
   if (kind == 2 && n == 256 && !pair) return run_peak<2, 256, false>(iters, s, st, tflops, cycles);
   if (kind == 2 && n == 128 && !pair) return run_peak<2, 128, false>(iters, s, st, tflops, cycles);
+  if (kind == 3 && n == 256 && !pair) return run_peak<3, 256, false>(iters, s, st, tflops, cycles);
   return 2;
 }
 

@@ -8,7 +8,7 @@ import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmoe_peak.so")
-KINDS = {"bf16": 0, "fp8": 1, "nvfp4": 2}
+KINDS = {"bf16": 0, "fp8": 1, "nvfp4": 2, "mxfp8": 3}
 _lib = None
 
 
