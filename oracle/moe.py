@@ -259,6 +259,34 @@ def clamped_swiglu(g, u, clamp):
     return g / (1.0 + np.exp(-g)) * u
 
 
+def swigluoai(g, u, clamp, alpha):
+    """h = min(g, c) * sigmoid(alpha * min(g, c)) * (clamp(u, -c, c) + 1), in
+    float64.
+
+    Struct_mega_ffn_ep_combine_send, ``clamp_activation``: the clamped
+    ("swigluoai") L1 activation, whose constants the dispatch supplies.  Read
+    as the SwiGLU variant with a sigmoid slope alpha on the gate and a bias of
+    1 on the up branch (the pages print neither; alpha is an input), with the
+    same clamps as clamped_swiglu: the gate from above, the up branch on both
+    sides.
+    """
+    c = float(clamp)
+    a = float(alpha)
+    g = np.minimum(g, c)
+    u = np.clip(u, -c, c)
+    with np.errstate(over="ignore"):
+        return g / (1.0 + np.exp(-a * g)) * (u + 1.0)
+
+
+def activation(problem, g, u):
+    """The L1 activation the problem selects: "swiglu" (the default, the
+    clamped SwiGLU) or "swigluoai" with slope problem["activation_alpha"]."""
+    clamp = problem.get("activation_clamp", 10.0)
+    if problem.get("activation", "swiglu") == "swigluoai":
+        return swigluoai(g, u, clamp, problem["activation_alpha"])
+    return clamped_swiglu(g, u, clamp)
+
+
 def gate_up(fmt, xhat, w13hat, alpha1, I):
     """L1: g = x^ W1^T, u = x^ W3^T with W1 = W13[:I], W3 = W13[I:]; NVFP4 scaled by alpha1."""
     acc = xhat @ w13hat.T
@@ -385,7 +413,9 @@ def moe_forward(problem, inputs, topk_idx, topk_weights, tokens=None,
     """The routed MoE FFN by its per-token definition.
 
     problem: dict(hidden, intermediate_hidden, num_experts, num_topk,
-                  activation_clamp, format, optional shared_expert)
+                  activation_clamp, format, optional shared_expert,
+                  optional activation ("swiglu" | "swigluoai") and
+                  activation_alpha)
              With shared_expert = 1 the weights hold num_experts + 1 experts
              (the last one shared) and topk_idx / topk_weights carry the
              shared slot (shared_expert_slots).
@@ -405,7 +435,6 @@ def moe_forward(problem, inputs, topk_idx, topk_weights, tokens=None,
     H = problem["hidden"]
     I = problem["intermediate_hidden"]
     E = problem["num_experts"] + int(problem.get("shared_expert", 0))
-    clamp = problem.get("activation_clamp", 10.0)
     idx = np.asarray(topk_idx, np.int64)
     w = np.asarray(topk_weights, np.float32).astype(np.float64)
     check_indices(idx, E)
@@ -422,7 +451,7 @@ def moe_forward(problem, inputs, topk_idx, topk_weights, tokens=None,
         w13hat = decode_weight(fmt, inputs["w13"], inputs.get("w13_scale"), e, 2 * I, H)
         w2hat = decode_weight(fmt, inputs["w2"], inputs.get("w2_scale"), e, H, I)
         g, u = gate_up(fmt, xhat[ti], w13hat, _expert_scale(inputs, "gate_up_expert_scales", e), I)
-        h32 = clamped_swiglu(g, u, clamp).astype(np.float32)
+        h32 = activation(problem, g, u).astype(np.float32)
         rq = requant(fmt, h32, _expert_scale(inputs, "c_input_scales", e))
         hhat = rq["hhat"] if hhat_override is None else hhat_override(e, tok[ti], sj)
         y = down(fmt, hhat, w2hat, _expert_scale(inputs, "down_expert_scales", e))
