@@ -127,7 +127,23 @@ typedef struct {
   int32_t fast_math;            /* nonzero: the SiLU uses the fast exponential */
   int32_t tile_regime;          /* moe_tile_regime_t: the grouped GEMMs' tile shape */
   int32_t shared_expert;        /* 0, or 1: a fused shared expert (above) */
+  int32_t activation;           /* moe_activation_t: the L1 activation */
+  float activation_alpha;       /* swigluoai: the gate's sigmoid slope (finite, > 0); else ignored */
 } moe_problem_t;
+
+/* The L1 activation, on the gate g and up u of an intermediate column, with
+ * c = activation_clamp (the gate clamped from above, the up branch on both
+ * sides):
+ *   SWIGLU     h = min(g,c) * sigmoid(min(g,c)) * clamp(u,-c,c)
+ *              (MegaMoESymmBuffer activation_clamp, the SwiGLU clamp value)
+ *   SWIGLUOAI  h = min(g,c) * sigmoid(a * min(g,c)) * (clamp(u,-c,c) + 1),
+ *              a = activation_alpha (Struct_mega_ffn_ep_combine_send
+ *              clamp_activation: the clamped "swigluoai" activation, whose
+ *              constants the dispatch supplies). */
+typedef enum {
+  MOE_ACT_SWIGLU = 0,
+  MOE_ACT_SWIGLUOAI = 1
+} moe_activation_t;
 
 /* Tile shape of the grouped GEMMs (the tile-regime choice the pages make
  * between prefill and decode batches).  AUTO picks SMALL_M for BF16 and FP8

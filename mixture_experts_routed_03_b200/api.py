@@ -64,6 +64,8 @@ class Problem(ctypes.Structure):
         ("fast_math", ctypes.c_int32),
         ("tile_regime", ctypes.c_int32),
         ("shared_expert", ctypes.c_int32),
+        ("activation", ctypes.c_int32),
+        ("activation_alpha", ctypes.c_float),
     ]
 
 
@@ -171,23 +173,26 @@ def _check(fn, code):
 
 
 TILE_REGIMES = {"auto": 0, "large_m": 1, "small_m": 2}
+ACTIVATIONS = {"swiglu": 0, "swigluoai": 1}
 
 
 def problem(num_tokens, hidden, intermediate_hidden, num_experts, num_topk,
-            activation_clamp=10.0, format="bf16", fast_math=1, tile_regime="auto", shared_expert=0):
+            activation_clamp=10.0, format="bf16", fast_math=1, tile_regime="auto", shared_expert=0,
+            activation="swiglu", activation_alpha=1.702):
     fmt = FORMATS[format] if isinstance(format, str) else int(format)
     clamp = float(activation_clamp)
     regime = TILE_REGIMES[tile_regime] if isinstance(tile_regime, str) else int(tile_regime)
+    act = ACTIVATIONS[activation] if isinstance(activation, str) else int(activation)
     return Problem(int(num_tokens), int(hidden), int(intermediate_hidden), int(num_experts),
                    int(num_topk), math.inf if math.isinf(clamp) else clamp, fmt, int(fast_math), regime,
-                   int(shared_expert))
+                   int(shared_expert), act, float(activation_alpha))
 
 
 def problem_from_dict(d, num_tokens=None, fast_math=1):
     return problem(d["num_tokens"] if num_tokens is None else num_tokens, d["hidden"],
                    d["intermediate_hidden"], d["num_experts"], d["num_topk"],
                    d.get("activation_clamp", 10.0), d["format"], fast_math, d.get("tile_regime", "auto"),
-                   d.get("shared_expert", 0))
+                   d.get("shared_expert", 0), d.get("activation", "swiglu"), d.get("activation_alpha", 1.702))
 
 
 def act(x, x_scale=None, x_rowwise_scale=None):

@@ -155,6 +155,9 @@ struct GemmArgs {
   int I, H, topk;
   float clamp;
   int fast_math;
+  // the L1 activation min(g,c) * sigmoid(act_a*min(g,c)) * (clamp(u,-c,c) + act_b):
+  // act_a = 1, act_b = 0 (clamped SwiGLU) or the slope and 1 (swigluoai)
+  float act_a, act_b;
   // layout (device, from the permute step)
   const int* expert_ids;
   const int* num_active;
@@ -285,24 +288,29 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// The L1 activation of gate g and up u with clamp c, slope a and up bias b:
+// min(g,c) * sigmoid(a*min(g,c)) * (clamp(u,-c,c) + b).  a = 1, b = 0 is the
+// clamped SwiGLU (both exact no-ops); b = 1 with the caller's slope is the
+// clamped "swigluoai" of Struct_mega_ffn_ep_combine_send clamp_activation.
 template <bool FAST>
-__device__ __forceinline__ float clamped_swiglu(float g, float u, float c) {
+__device__ __forceinline__ float l1_act(float g, float u, float c, float a, float b) {
   const float gc = fminf(g, c);
   const float uc = fminf(fmaxf(u, -c), c);
-  if (FAST) return __fmul_rn(__fdividef(gc, 1.0f + __expf(-gc)), uc);
-  return __fmul_rn(__fdiv_rn(gc, 1.0f + expf(-gc)), uc);
+  const float z = __fmul_rn(a, gc);
+  const float s = FAST ? __fdividef(gc, 1.0f + __expf(-z)) : __fdiv_rn(gc, 1.0f + expf(-z));
+  return __fmul_rn(s, __fadd_rn(uc, b));
 }
 
-// h[i] = clamped SwiGLU of (gate acc[i], up acc[64 + i]), i < 64.  The
+// h[i] = the activation of (gate acc[i], up acc[64 + i]), i < 64.  The
 // precision switch is taken once, outside the unrolled loop, so only one of
 // the two sequences runs.
-__device__ __forceinline__ void swiglu_row(const float (&acc)[128], float (&h)[64], float c, int fast) {
-  if (fast) {
+__device__ __forceinline__ void swiglu_row(const float (&acc)[128], float (&h)[64], const GemmArgs& p) {
+  if (p.fast_math) {
 #pragma unroll
-    for (int i = 0; i < 64; ++i) h[i] = clamped_swiglu<true>(acc[i], acc[64 + i], c);
+    for (int i = 0; i < 64; ++i) h[i] = l1_act<true>(acc[i], acc[64 + i], p.clamp, p.act_a, p.act_b);
   } else {
 #pragma unroll
-    for (int i = 0; i < 64; ++i) h[i] = clamped_swiglu<false>(acc[i], acc[64 + i], c);
+    for (int i = 0; i < 64; ++i) h[i] = l1_act<false>(acc[i], acc[64 + i], p.clamp, p.act_a, p.act_b);
   }
 }
 
@@ -663,7 +671,7 @@ __device__ __forceinline__ void gemm_phase(const GemmArgs& p, const CUtensorMap*
         // h for intermediate columns j0 + 64*half + i, i < 64
         const int hcol0 = t.n_tile * 128 + half * 64;
         float h[64];
-        swiglu_row(acc, h, p.clamp, p.fast_math);
+        swiglu_row(acc, h, p);
         uint8_t* hrow = p.h_out + static_cast<size_t>(r) * p.h_row_bytes;
         if constexpr (FMT == FMT_FP8) {
           float amax = 0.0f;

@@ -319,16 +319,18 @@ __device__ __forceinline__ void gemm_phase_swap(const GemmArgs& p, const CUtenso
         for (int j = 0; j < 4; ++j) {
           const int tr = ew * 4 + j;                    // routed row of the tile (warp-uniform)
           float h[4];
+          float gv[4], uv[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            gv[i] = stage_rows[(gate_row0 + i) * Cfg::kSStride + tr];
+            uv[i] = stage_rows[(gate_row0 + G + i) * Cfg::kSStride + tr];
+          }
           if (p.fast_math) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              h[i] = clamped_swiglu<true>(stage_rows[(gate_row0 + i) * Cfg::kSStride + tr],
-                                          stage_rows[(gate_row0 + G + i) * Cfg::kSStride + tr], p.clamp);
+            for (int i = 0; i < 4; ++i) h[i] = l1_act<true>(gv[i], uv[i], p.clamp, p.act_a, p.act_b);
           } else {
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              h[i] = clamped_swiglu<false>(stage_rows[(gate_row0 + i) * Cfg::kSStride + tr],
-                                           stage_rows[(gate_row0 + G + i) * Cfg::kSStride + tr], p.clamp);
+            for (int i = 0; i < 4; ++i) h[i] = l1_act<false>(gv[i], uv[i], p.clamp, p.act_a, p.act_b);
           }
           const bool row_ok = tr < t.rows;
           uint8_t* hrow = p.h_out + static_cast<size_t>(t.row0 + tr) * p.h_row_bytes;

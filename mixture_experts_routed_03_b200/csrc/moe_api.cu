@@ -40,6 +40,9 @@ moe_status_t check_problem(const moe_problem_t* p) {
   if (p->intermediate_hidden <= 0 || p->intermediate_hidden % 128 != 0) return MOE_ERR_INVALID_ARG;
   if (p->num_experts < 1 || p->num_topk < 1 || p->num_topk > p->num_experts) return MOE_ERR_INVALID_ARG;
   if (p->shared_expert != 0 && p->shared_expert != 1) return MOE_ERR_INVALID_ARG;
+  if (p->activation != MOE_ACT_SWIGLU && p->activation != MOE_ACT_SWIGLUOAI) return MOE_ERR_INVALID_ARG;
+  if (p->activation == MOE_ACT_SWIGLUOAI && !(std::isfinite(p->activation_alpha) && p->activation_alpha > 0.0f))
+    return MOE_ERR_INVALID_ARG;
   // with a shared expert: num_experts + 1 experts, num_topk + 1 slots per token
   const int E_all = p->num_experts + p->shared_expert;
   const int k_all = p->num_topk + p->shared_expert;
@@ -437,6 +440,9 @@ moe_status_t plan_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_we
   a.topk = k;
   a.clamp = p->activation_clamp;
   a.fast_math = p->fast_math;
+  const bool oai = p->activation == MOE_ACT_SWIGLUOAI;
+  a.act_a = oai ? p->activation_alpha : 1.0f;
+  a.act_b = oai ? 1.0f : 0.0f;
   a.expert_ids = b.expert_ids;
   a.num_active = b.num_active;
   a.starts = b.starts;

@@ -178,7 +178,8 @@ def make_inputs(p, seed=0, device="cpu"):
         # with the clamp c, |h| < c*c, so 2688 * G >= c*c never saturates the
         # E4M3 block scale.  Without a clamp a fixed bound of 1000 stands in.
         c = float(p.get("activation_clamp", 10.0))
-        bound = c * c if math.isfinite(c) else 1000.0
+        # |h| < c*c for the clamped SwiGLU, < c*(c+1) for swigluoai
+        bound = (c * (c + 1.0) if p.get("activation") == "swigluoai" else c * c) if math.isfinite(c) else 1000.0
         c_in = _uniform((Ew,), 1.0, 1.2, g, device) * (bound / 2688.0)
         d["gate_up_expert_scales"] = (w13_global * x_global).to(torch.float32)
         d["down_expert_scales"] = (w2_global * c_in).to(torch.float32)

@@ -59,6 +59,10 @@ def _prob(**kw):
     (dict(format="nvfp4", tile_regime="small_m"), api.MOE_ERR_UNSUPPORTED),
     (dict(format="mxfp8", tile_regime="small_m"), api.MOE_ERR_UNSUPPORTED),
     (dict(shared_expert=2), api.MOE_ERR_INVALID_ARG),
+    (dict(activation=2), api.MOE_ERR_INVALID_ARG),
+    (dict(activation="swigluoai", activation_alpha=0.0), api.MOE_ERR_INVALID_ARG),
+    (dict(activation="swigluoai", activation_alpha=float("nan")), api.MOE_ERR_INVALID_ARG),
+    (dict(activation="swigluoai", activation_alpha=float("inf")), api.MOE_ERR_INVALID_ARG),
     (dict(shared_expert=-1), api.MOE_ERR_INVALID_ARG),
     (dict(num_experts=1024, num_topk=2, shared_expert=1), api.MOE_ERR_UNSUPPORTED),
     (dict(format=4), api.MOE_ERR_INVALID_ARG),

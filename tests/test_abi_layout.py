@@ -20,7 +20,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 STRUCTS = {
     "moe_problem_t": (api.Problem, ["num_tokens", "hidden", "intermediate_hidden", "num_experts", "num_topk",
                                      "activation_clamp", "format", "fast_math", "tile_regime",
-                                     "shared_expert"]),
+                                     "shared_expert", "activation", "activation_alpha"]),
     "moe_act_t": (api.Act, ["x", "x_scale", "x_rowwise_scale"]),
     "moe_weights_t": (api.Weights, [f[0] for f in api.Weights._fields_]),
     "moe_layout_t": (api.Layout, [f[0] for f in api.Layout._fields_]),

@@ -191,3 +191,30 @@ def test_full_size_workloads_sampled(name, ntok):
     # and at rounding midpoints of the intermediate)
     a, b = chain.out, fused.out
     assert np.mean(~S.close_bf16(a, b, S.TOL[p["format"]] * S.rms(a))) < 1e-3
+
+
+@pytest.mark.parametrize("fmt,regime", [("bf16", "large_m"), ("bf16", "small_m"), ("fp8", "large_m"),
+                                        ("fp8", "small_m"), ("nvfp4", "large_m"), ("mxfp8", "large_m")])
+def test_swigluoai_activation(fmt, regime):
+    """The clamped swigluoai activation (Struct_mega_ffn_ep_combine_send,
+    clamp_activation) with slope 1.702 and clamp 7, weights scaled so that
+    the clamp is active: chain and single launch against the oracle."""
+    M, H, I, E, k = 150, 512, 256, 4, 2
+    p = dict(_small(fmt, M, H, I, E, k, clamp=7.0, regime=regime), activation="swigluoai",
+             activation_alpha=1.702)
+    d, host = S.make(p, seed=21)
+    if fmt == "bf16":
+        d["w13"] = (d["w13"].view(torch.bfloat16).float() * 40).to(torch.bfloat16).view(torch.int16)
+        host["w13"] = d["w13"].cpu().view(torch.int16).numpy().view(np.uint16)
+    elif fmt == "fp8":
+        d["w13_scale"] = d["w13_scale"] * 40
+        host["w13_scale"] = d["w13_scale"].cpu().numpy()
+    elif fmt == "mxfp8":
+        d["w13_scale"] = d["w13_scale"] + 5        # x 32
+        host["w13_scale"] = d["w13_scale"].cpu().numpy()
+    else:
+        d["gate_up_expert_scales"] = d["gate_up_expert_scales"] * 40
+        host["gate_up_expert_scales"] = d["gate_up_expert_scales"].cpu().numpy()
+    L = layer.MoELayer(p, S.weights_of(d), device=S.device())
+    assert api.tile_regime(L.problem(M)) == regime
+    _check_both_paths(p, d, host, L, np.arange(M), f"swigluoai/{fmt}/{regime}")
