@@ -45,17 +45,20 @@ reasoning in the design notes of the repository):
 * ``topk_idx == -1`` is a skipped slot (the masked-id convention of
   ``expert_ids``); duplicates within a token are independent slots.
 * Activation: h = min(g,c) * sigmoid(min(g,c)) * clamp(u,-c,c); c = +inf is
-  the textbook SwiGLU.  Gate rows are W13[e, :I], up rows are W13[e, I:].
+  the textbook SwiGLU (or the clamped swigluoai, see ``swigluoai``).  Gate
+  rows are W13[e, :I], up rows are W13[e, I:].
 * Re-quant of h (computed in float64, then held in float32 as the kernel
   holds it): NVFP4 per 16 values along I with an E4M3 block scale and the
   per-expert FP32 ``c_input_scales`` G as the dequant multiplier; FP8 per 128
-  values with an FP32 scale amax/448; BF16 by round-to-nearest-even.  The
+  values with an FP32 scale amax/448; MXFP8 per 32 values with a power-of-two
+  scale; FP8 per-tensor against the per-expert G; BF16 by
+  round-to-nearest-even.  The
   FP32 steps of the quantisers are fixed (see ``requant``) so that a code is
   decided in the same precision on both sides.
 * NVFP4 GEMMs: the MMA sums products of (e2m1 x e4m3 block scale) operands,
   then the per-expert scale (``gate_up_expert_scales`` or
-  ``down_expert_scales``) multiplies the sum.  FP8 GEMMs: every operand is
-  its E4M3 code times its FP32 block scale.
+  ``down_expert_scales``) multiplies the sum.  FP8, FP8 per-tensor and MXFP8
+  GEMMs: every operand is its E4M3 code times its scale.
 * The output is BF16, rounded once from the float64 sum (via float32).
 """
 
@@ -63,7 +66,7 @@ import numpy as np
 
 from . import formats as F
 
-FORMATS = ("bf16", "fp8", "nvfp4", "mxfp8")
+FORMATS = ("bf16", "fp8", "nvfp4", "mxfp8", "fp8_tensor")
 
 
 # ----------------------------------------------------------------------------
@@ -155,6 +158,8 @@ def decode_x(fmt, x, x_scale, H, rows=None, row_scale=None):
     """Activations [M, H] -> float64.
 
     fp8: E4M3 codes times the FP32 per-128 block scale of the token.
+    fp8_tensor: E4M3 codes times the one FP32 dequantisation scale of the
+    whole activation tensor (x_scale of shape [1]).
     mxfp8: E4M3 codes times the UE8M0 per-32 block scale of the token.
     nvfp4: e2m1 codes times the E4M3 per-16 block scale, times the token's
     BF16 rowwise scale when the activations were quantised per token
@@ -162,6 +167,9 @@ def decode_x(fmt, x, x_scale, H, rows=None, row_scale=None):
     carried by the per-expert L1 output scaling instead.
     """
     x = np.asarray(x)
+    if fmt == "fp8_tensor":
+        x = x if rows is None else x[rows]
+        return F.e4m3_decode(x) * float(np.asarray(x_scale, np.float32).reshape(-1)[0])
     if rows is not None:
         x = x[rows]
         x_scale = None if x_scale is None else np.asarray(x_scale)[rows]
@@ -224,8 +232,9 @@ def quantize_nvfp4_rowwise(x):
 def decode_weight(fmt, w, w_scale, e, n_rows, k_cols):
     """Expert e's weight [n_rows, k_cols] (K-major, as stored) -> float64.
 
-    fp8 scales are per 128 x 128 block; mxfp8 (UE8M0) scales per 1 x 32
-    block; nvfp4 scales per 1 x 16 block.
+    fp8 scales are per 128 x 128 block; fp8_tensor has one FP32 scale per
+    expert's matrix (w_scale [E]); mxfp8 (UE8M0) scales per 1 x 32 block;
+    nvfp4 scales per 1 x 16 block.
     """
     if fmt == "bf16":
         return F.bf16_decode(np.asarray(w)[e])
@@ -233,6 +242,8 @@ def decode_weight(fmt, w, w_scale, e, n_rows, k_cols):
         s = np.asarray(w_scale, np.float32)[e].astype(np.float64)
         full = np.repeat(np.repeat(s, 128, axis=0), 128, axis=1)
         return F.e4m3_decode(np.asarray(w)[e]) * full
+    if fmt == "fp8_tensor":
+        return F.e4m3_decode(np.asarray(w)[e]) * float(np.asarray(w_scale, np.float32)[e])
     if fmt == "mxfp8":
         return F.e4m3_decode(np.asarray(w)[e]) * np.repeat(F.ue8m0_decode(np.asarray(w_scale)[e]), 32, axis=1)
     if fmt == "nvfp4":
@@ -318,6 +329,12 @@ def requant(fmt, h32, G=None):
                E4M3 exponent; X = -127 where amax == 0)
         q    = e4m3_satfinite(h * 2**-X)      (exact power-of-two scaling)
         scale code = X + 127
+    fp8_tensor, one static scale per expert (the per-tensor FP8 encoding of
+    MoEActivationPack read with the static re-quant scale of
+    Struct_mega_ffn_ep_combine_send, c_input_scales = G, a dequant
+    multiplier):
+        q    = e4m3_satfinite(h * (1 / G))     (FP32 steps)
+        hhat = q * G                           (scales = G per row)
     """
     h32 = np.asarray(h32, np.float32)
     rows, I = h32.shape
@@ -335,6 +352,13 @@ def requant(fmt, h32, G=None):
         codes = np.where((s == 0)[:, :, None], np.uint8(0), codes).reshape(rows, I)
         hhat = F.e4m3_decode(codes).reshape(rows, I // 128, 128) * s[:, :, None].astype(np.float64)
         return dict(codes=codes, scales=s, hhat=hhat.reshape(rows, I), pre=v.reshape(rows, I), pre_scale=None)
+    if fmt == "fp8_tensor":
+        G32 = np.float32(G)
+        inv = np.float32(np.float32(1.0) / G32)
+        v = (h32 * inv).astype(np.float32)
+        codes = F.e4m3_encode(v)
+        hhat = F.e4m3_decode(codes) * float(G32)
+        return dict(codes=codes, scales=np.full(rows, G32, np.float32), hhat=hhat, pre=v, pre_scale=None)
     if fmt == "mxfp8":
         blk = h32.reshape(rows, I // 32, 32)
         amax = np.max(np.abs(blk), axis=2).astype(np.float64)
@@ -374,6 +398,8 @@ def dequant_intermediate(fmt, codes, scales, I):
     if fmt == "fp8":
         s = np.asarray(scales, np.float32).astype(np.float64)
         return F.e4m3_decode(codes) * np.repeat(s, 128, axis=1)
+    if fmt == "fp8_tensor":
+        return F.e4m3_decode(codes) * np.asarray(scales, np.float32).astype(np.float64).reshape(-1, 1)
     if fmt == "mxfp8":
         return F.e4m3_decode(codes) * np.repeat(F.ue8m0_decode(scales), 32, axis=1)
     if fmt == "nvfp4":
