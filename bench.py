@@ -38,16 +38,16 @@ DEFAULT_WORKLOAD = "fp8_prefill_routed"
 METRIC = "routed tokens/sec and achieved TFLOPS (% of roofline) per MoE layer, 1 B200"
 FLUSH_BYTES = 512 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-FMT_TENSOR_RATIO = {"bf16": 1.0, "fp8": 2.0, "nvfp4": 4.0, "mxfp8": 2.0}   # nominal dense ratio to bf16
+FMT_TENSOR_RATIO = {"bf16": 1.0, "fp8": 2.0, "nvfp4": 4.0, "mxfp8": 2.0, "fp8_tensor": 2.0}   # nominal dense ratio to bf16
 # B200 datasheet dense peaks (the sparse figures halved) and the ~8 TB/s of
 # HBM the layer's roofline is stated against: time = max(FLOPs / tensor peak,
 # bytes / HBM bandwidth)
-SPEC_TFLOPS = {"bf16": 2250.0, "fp8": 4500.0, "nvfp4": 9000.0, "mxfp8": 4500.0}
+SPEC_TFLOPS = {"bf16": 2250.0, "fp8": 4500.0, "nvfp4": 9000.0, "mxfp8": 4500.0, "fp8_tensor": 4500.0}
 SPEC_HBM_GBS = 8000.0
-ELEM_BYTES = {"bf16": 2.0, "fp8": 1.0, "nvfp4": 0.5, "mxfp8": 1.0}
+ELEM_BYTES = {"bf16": 2.0, "fp8": 1.0, "nvfp4": 0.5, "mxfp8": 1.0, "fp8_tensor": 1.0}
 BOUND = {"tiny_bf16": "hbm", "fp8_block": "hbm", "nvfp4_decode": "hbm",
          "nvfp4_prefill": "tensor", "fp8_prefill_routed": "tensor", "nvfp4_prefill_rowwise": "tensor",
-         "mxfp8_prefill_routed": "tensor"}
+         "mxfp8_prefill_routed": "tensor", "fp8_tensor_prefill_routed": "tensor"}
 
 
 def parse():
@@ -63,7 +63,8 @@ def parse():
     ap.add_argument("--no-mma-peak", action="store_true",
                     help="skip the tensor-core peak probe (run after the timed steps)")
     ap.add_argument("--side-workloads",
-                    default="fp8_block,nvfp4_prefill,nvfp4_decode,nvfp4_prefill_rowwise,mxfp8_prefill_routed",
+                    default="fp8_block,nvfp4_prefill,nvfp4_decode,nvfp4_prefill_rowwise,mxfp8_prefill_routed,"
+                            "fp8_tensor_prefill_routed",
                     help="other configurations timed after the main one (one GPU, rank 0), reported "
                          "under 'workloads'; empty for none")
     ap.add_argument("--chain", action="store_true",
@@ -236,6 +237,9 @@ def work_model(p, num_active):
     elif fmt == "mxfp8":
         w13_sc, w2_sc = 2 * I * H // 32, H * I // 32
         x_sc, h_sc = H // 32, I // 32
+    elif fmt == "fp8_tensor":
+        w13_sc = w2_sc = 4
+        x_sc = h_sc = 0
     else:
         w13_sc = w2_sc = x_sc = h_sc = 0
     w13 = num_active * (2 * I * H * eb + w13_sc)
@@ -327,8 +331,9 @@ def mma_probe(fmt, achieved_tflops):
     try:
         from mixture_experts_routed_03_b200 import peak
         out = {}
-        for pair in (False, True) if fmt in ("bf16", "fp8") else (False,):
-            tf, cyc = peak.mma_peak(fmt, 256, pair, iters=20000)
+        kind = "fp8" if fmt == "fp8_tensor" else fmt   # the same E4M3 MMAs
+        for pair in (False, True) if kind in ("bf16", "fp8") else (False,):
+            tf, cyc = peak.mma_peak(kind, 256, pair, iters=20000)
             out["cta_pair" if pair else "one_cta"] = {"tflops": tf, "cycles_per_mma": cyc}
         best = max(v["tflops"] for v in out.values())
         out["frac_of_best"] = achieved_tflops / best
@@ -596,7 +601,8 @@ def main_ours(args):
         "vs_baseline": None,
         "dtype": {"bf16": "bf16", "fp8": "e4m3+f32 scales (f32 accumulate)",
                   "nvfp4": "e2m1+e4m3 scales (f32 accumulate)",
-                  "mxfp8": "e4m3+ue8m0 scales per 32 (f32 accumulate)"}[p["format"]],
+                  "mxfp8": "e4m3+ue8m0 scales per 32 (f32 accumulate)",
+                  "fp8_tensor": "e4m3+f32 per-tensor scales (f32 accumulate)"}[p["format"]],
         "data": "synthetic (seeded torch generators; random-init experts of the workload's shapes)",
         "config": {"workload": args.workload + ("" if not args.set else " (" + ",".join(args.set) + ")"),
                    "path": "multi-launch chain" if args.chain else "moe_fused (one launch)",

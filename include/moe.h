@@ -64,6 +64,14 @@
  *                   w2  e4m3 [E, H, I],  w2_scale  ue8m0 [E, H, I/32]
  *                   the intermediate is re-quantised per 32 columns with
  *                   scale 2^(floor(log2 amax) - 8), clamped to 2^[-127, 127]
+ *  format FP8 per-tensor (MoEActivationPack, FP8 per-tensor: E4M3 values
+ *                   with a scalar FP32 dequantisation scale)
+ *                   x  e4m3 [M, H], x_scale fp32 [1]
+ *                   w13 e4m3 [E, 2I, H], w13_scale fp32 [E] (one per matrix)
+ *                   w2  e4m3 [E, H, I],  w2_scale  fp32 [E]
+ *                   c_input_scales fp32 [E]: the intermediate's static
+ *                   re-quant scale G, q = e4m3(h * (1/G)), a dequant
+ *                   multiplier of the down GEMM
  *  topk_idx int64 [M, k]; topk_weights fp32 [M, k]; output bf16 [M, H].
  *
  *  Geometry (flashinfer.megamoe.MegaMoESymmBuffer, Parameters): hidden is a
@@ -95,7 +103,8 @@ typedef enum {
   MOE_FMT_BF16 = 0,
   MOE_FMT_FP8_E4M3_B128 = 1,  /* E4M3 with FP32 per-128 block scales */
   MOE_FMT_NVFP4 = 2,          /* e2m1 with E4M3 per-16 block scales + per-expert FP32 */
-  MOE_FMT_MXFP8 = 3           /* E4M3 with UE8M0 (power-of-two) per-32 block scales */
+  MOE_FMT_MXFP8 = 3,          /* E4M3 with UE8M0 (power-of-two) per-32 block scales */
+  MOE_FMT_FP8_PER_TENSOR = 4  /* E4M3 with one FP32 scale per tensor / expert matrix */
 } moe_format_t;
 
 /* The problem statement, after flashinfer.megamoe.MegaMoESymmBuffer
@@ -151,7 +160,7 @@ typedef enum {
  * 64*num_experts), else LARGE_M.  LARGE_M: 128 routed rows x 256 weight rows
  * per tile.  SMALL_M: the operands swapped, 256 weight rows x 32 routed rows
  * per tile, so the tensor work follows the routed rows that exist; BF16 and
- * FP8 only (MOE_ERR_UNSUPPORTED for NVFP4 and MXFP8).  Results agree between regimes
+ * FP8 only (MOE_ERR_UNSUPPORTED for NVFP4, MXFP8 and FP8 per-tensor).  Results agree between regimes
  * up to FP32 summation order. */
 typedef enum {
   MOE_TILE_AUTO = 0,
@@ -175,9 +184,10 @@ typedef struct {
  * blobs that moe_prepare_weights wrote (Struct_mega_ffn_ep_combine_send:
  * "pre-permuted gate/up weights", "pre-permuted W13 scale tile"); for NVFP4
  * and MXFP8 the block scales are inside those blobs and w13_scale / w2_scale
- * are ignored; for FP8 w13_scale / w2_scale are the logical FP32 block scales.
- * The three per-expert FP32 arrays are used by NVFP4 only and may be NULL
- * otherwise. */
+ * are ignored; for FP8 w13_scale / w2_scale are the logical FP32 block scales,
+ * for FP8 per-tensor the FP32 [E] per-matrix scales.  gate_up_expert_scales
+ * and down_expert_scales are used by NVFP4 only, c_input_scales by NVFP4 and
+ * FP8 per-tensor; they may be NULL otherwise. */
 typedef struct {
   const void* w13;
   const void* w13_scale;

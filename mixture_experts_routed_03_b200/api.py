@@ -26,7 +26,7 @@ MOE_ERR_CUDA = 4
 MOE_ERR_BAD_INDEX = 5
 MOE_ERR_TIMEOUT = 6
 
-FORMATS = {"bf16": 0, "fp8": 1, "nvfp4": 2, "mxfp8": 3}
+FORMATS = {"bf16": 0, "fp8": 1, "nvfp4": 2, "mxfp8": 3, "fp8_tensor": 4}
 
 MOE_OUT_ACCUMULATE = 0
 MOE_OUT_STAGED = 1

@@ -716,7 +716,7 @@ __device__ __forceinline__ void gather_scales(const GatherArgs& g, int64_t t, in
   if (g.fmt == 1) {
     const float* xs = static_cast<const float*>(g.x_scale) + t * (g.H / 128);
     for (int kb = lane; kb < g.H / 128; kb += 32) g.sa_t[static_cast<size_t>(kb) * g.ld + pr] = xs[kb];
-  } else if (g.fmt >= 2) {
+  } else if (g.fmt == 2 || g.fmt == 3) {
     // one byte per 16 (NVFP4) or 32 (MXFP8) elements, four per tile row
     const int cols = g.fmt == 2 ? g.H / 16 : g.H / 32;
     const uint8_t* xs = static_cast<const uint8_t*>(g.x_scale) + t * cols;
@@ -762,7 +762,7 @@ __device__ __forceinline__ void gather_rows(const GatherArgs& g, int64_t warp_id
     const int64_t t0 = g.src_info[r0] / g.topk;
     const int64_t t1 = (r1 >= 0) ? g.src_info[r1] / g.topk : 0;
     gather_copy2(g, r0, t0, r1, t1, lane);
-    if (g.fmt >= 2) {
+    if (g.fmt == 2 || g.fmt == 3) {
       gather_scales(g, t0, p0, lane);
       if (r1 >= 0) gather_scales(g, t1, p1, lane);
     }

@@ -12,6 +12,9 @@
 //          128-wide K block into a TMEM partial; the epilogue warps promote
 //          it, partial * (a_scale[row, kb] * b_scale[n_blk, kb]), into FP32
 //          registers (the per-128 FP32 block scales have no hardware form)
+//   FP8T   (per-tensor scales) tcgen05.mma kind::f8f6f4, FP32 accumulation
+//          over all of K in TMEM; the epilogue applies the per-tensor and
+//          per-expert scales to the sum
 //   MXFP8  tcgen05.mma kind::mxf8f6f4 block_scale scale_vec::1X: E4M3
 //          operands, UE8M0 scale per 32 elements (one per MMA instruction,
 //          picked by the descriptor's scale-factor id), copied to TMEM with
@@ -46,8 +49,8 @@
 // registers, the accumulator is released, then h is re-quantised (BF16 by
 // rounding; FP8 per 128 columns with scale amax/448; NVFP4 per 16 columns
 // with an E4M3 scale against the per-expert c_input_scales; MXFP8 per 32
-// columns with the power-of-two scale 2^(floor(log2 amax) - 8)) and stored
-// in expert order for L2.
+// columns with the power-of-two scale 2^(floor(log2 amax) - 8); FP8T
+// against the per-expert c_input_scales) and stored in expert order for L2.
 // L2 epilogue: the row is read into registers, the accumulator released, and
 // the row, times its router weight, added into the token-ordered FP32
 // accumulator -- float4 atomics through a 32 x 32 transpose (BF16, FP8, MXFP8) or
@@ -63,7 +66,7 @@
 
 namespace moe {
 
-enum { FMT_BF16 = 0, FMT_FP8 = 1, FMT_NVFP4 = 2, FMT_MXFP8 = 3 };
+enum { FMT_BF16 = 0, FMT_FP8 = 1, FMT_NVFP4 = 2, FMT_MXFP8 = 3, FMT_FP8T = 4 };
 enum { EPI_L1 = 0, EPI_L2_ACC = 1, EPI_L2_STAGED = 2 };
 
 constexpr int kBM = 128;          // MMA M: rows of A (routed rows) per tile
@@ -177,8 +180,13 @@ struct GemmArgs {
   int sa_ld;
   const float* sb;
   int sb_nb, sb_kb;
-  // NVFP4 per-expert scalars
-  const float* alpha;   // gate_up_expert_scales (L1) or down_expert_scales (L2)
+  // NVFP4 per-expert scalars: gate_up_expert_scales (L1) or
+  // down_expert_scales (L2); FP8T: the experts' weight scales, times
+  // alpha_scalar[0] (L1: the activation scale) or alpha_e2[e] (L2:
+  // c_input_scales) when those are set
+  const float* alpha;
+  const float* alpha_scalar;
+  const float* alpha_e2;
   const uint16_t* x_row_scale;   // NVFP4 L1: BF16 per-token rowwise scales of x, or null
   const float* c_in;    // c_input_scales (L1 re-quant)
   // L1 output: the re-quantised intermediate, expert order
@@ -432,7 +440,7 @@ __device__ __forceinline__ void gemm_phase(const GemmArgs& p, const CUtensorMap*
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t kIdesc = (FMT == FMT_BF16)    ? idesc_dense(1, 1, kBN)
-                                  : (FMT == FMT_FP8)   ? idesc_dense(0, 0, kBN)
+                                  : (FMT == FMT_FP8 || FMT == FMT_FP8T) ? idesc_dense(0, 0, kBN)
                                   : (FMT == FMT_NVFP4) ? idesc_nvf4(kBN)
                                                        : idesc_mxf8(kBN, 0);
       int stage = 0;
@@ -477,7 +485,7 @@ __device__ __forceinline__ void gemm_phase(const GemmArgs& p, const CUtensorMap*
             const uint64_t a = adesc + static_cast<uint64_t>(2 * kc);
             const uint64_t b = bdesc + static_cast<uint64_t>(2 * kc);
             if (FMT == FMT_BF16) mma_f16(d, a, b, kIdesc, acc);
-            else if (FMT == FMT_FP8) mma_f8(d, a, b, kIdesc, acc);
+            else if (FMT == FMT_FP8 || FMT == FMT_FP8T) mma_f8(d, a, b, kIdesc, acc);
             else if (FMT == FMT_NVFP4) mma_nvf4(d, a, b, kIdesc, sfa_t + 4 * kc, sfa_t + kSFBOff + 8 * kc, acc);
             // one UE8M0 scale per 32-wide K step: byte kc of the stage's scale words
             else mma_mxf8(d, a, b, idesc_mxf8(kBN, kc), sfa_t, sfa_t + kSFBOff, acc);
@@ -626,7 +634,7 @@ __device__ __forceinline__ void gemm_phase(const GemmArgs& p, const CUtensorMap*
         }
         if (!ok) break;
       } else {
-        // BF16 / NVFP4 / MXFP8: the whole K sum is in TMEM; read it, release it.
+        // BF16 / NVFP4 / MXFP8 / FP8T: the whole K sum is in TMEM; read it, release it.
         if (!mbar_wait(&acc_full[ab], aphase, abort_flag, p.status, 6)) break;
         tc_fence_after();
         if (gather_wgt) wgt = __ldg(p.topk_weights + s_flat);
@@ -657,6 +665,14 @@ __device__ __forceinline__ void gemm_phase(const GemmArgs& p, const CUtensorMap*
         if (++ab == NACC) {
           ab = 0;
           aphase ^= 1u;
+        }
+        if (FMT == FMT_FP8T) {
+          // (activation scale x weight scale) or (re-quant scale x weight scale)
+          float alpha = __ldg(p.alpha + t.e);
+          if (p.alpha_scalar) alpha = __fmul_rn(__ldg(p.alpha_scalar), alpha);
+          if (p.alpha_e2) alpha = __fmul_rn(__ldg(p.alpha_e2 + t.e), alpha);
+#pragma unroll
+          for (int i = 0; i < 128; ++i) acc[i] = __fmul_rn(acc[i], alpha);
         }
         if (FMT == FMT_NVFP4) {
           float alpha = __ldg(p.alpha + t.e);
@@ -714,6 +730,21 @@ __device__ __forceinline__ void gemm_phase(const GemmArgs& p, const CUtensorMap*
             const uint4 v = *reinterpret_cast<const uint4*>(stg + row * Cfg::kHStageStride + c16 * 16);
             if (row < rows_here)
               *reinterpret_cast<uint4*>(hbase + static_cast<size_t>(row) * p.h_row_bytes + c16 * 16) = v;
+          }
+        } else if constexpr (FMT == FMT_FP8T) {
+          // one static scale per expert: codes e4m3(h * (1 / G)), saturating
+          const float inv = __frcp_rn(__ldg(p.c_in + t.e));
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const uint32_t lo = cvt_e4m3x2(__fmul_rn(h[4 * i], inv), __fmul_rn(h[4 * i + 1], inv));
+            const uint32_t hi = cvt_e4m3x2(__fmul_rn(h[4 * i + 2], inv), __fmul_rn(h[4 * i + 3], inv));
+            w[i] = lo | (hi << 16);
+          }
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(hrow + hcol0);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
           }
         } else if constexpr (FMT == FMT_MXFP8) {
           // two 32-column blocks: scale 2^X, X = floor(log2 amax) - 8 clamped

@@ -35,7 +35,7 @@ size_t scale_row_bytes(int fmt, int K) {
 moe_status_t check_problem(const moe_problem_t* p) {
   if (!p) return MOE_ERR_INVALID_ARG;
   if (p->num_tokens < 0) return MOE_ERR_INVALID_ARG;
-  if (p->format < MOE_FMT_BF16 || p->format > MOE_FMT_MXFP8) return MOE_ERR_INVALID_ARG;
+  if (p->format < MOE_FMT_BF16 || p->format > MOE_FMT_FP8_PER_TENSOR) return MOE_ERR_INVALID_ARG;
   if (p->hidden <= 0 || p->hidden % 256 != 0) return MOE_ERR_INVALID_ARG;
   if (p->intermediate_hidden <= 0 || p->intermediate_hidden % 128 != 0) return MOE_ERR_INVALID_ARG;
   if (p->num_experts < 1 || p->num_topk < 1 || p->num_topk > p->num_experts) return MOE_ERR_INVALID_ARG;
@@ -49,7 +49,7 @@ moe_status_t check_problem(const moe_problem_t* p) {
   if (E_all > 1024) return MOE_ERR_UNSUPPORTED;
   if (std::isnan(p->activation_clamp) || !(p->activation_clamp > 0.0f)) return MOE_ERR_INVALID_ARG;
   if (p->tile_regime < MOE_TILE_AUTO || p->tile_regime > MOE_TILE_SMALL_M) return MOE_ERR_INVALID_ARG;
-  if (p->tile_regime == MOE_TILE_SMALL_M && (p->format == MOE_FMT_NVFP4 || p->format == MOE_FMT_MXFP8))
+  if (p->tile_regime == MOE_TILE_SMALL_M && p->format != MOE_FMT_BF16 && p->format != MOE_FMT_FP8_E4M3_B128)
     return MOE_ERR_UNSUPPORTED;
   if (p->format == MOE_FMT_NVFP4 && p->intermediate_hidden % 256 != 0) return MOE_ERR_UNSUPPORTED;
   const int64_t R = p->num_tokens * k_all;
@@ -258,10 +258,12 @@ cudaError_t set_all_attrs() {
   if ((e = set_fused_attr<FMT_FP8>()) != cudaSuccess) return e;
   if ((e = set_fused_attr<FMT_NVFP4>()) != cudaSuccess) return e;
   if ((e = set_fused_attr<FMT_MXFP8>()) != cudaSuccess) return e;
+  if ((e = set_fused_attr<FMT_FP8T>()) != cudaSuccess) return e;
   if ((e = set_attrs_fmt<FMT_BF16>()) != cudaSuccess) return e;
   if ((e = set_attrs_fmt<FMT_FP8>()) != cudaSuccess) return e;
   if ((e = set_attrs_fmt<FMT_NVFP4>()) != cudaSuccess) return e;
   if ((e = set_attrs_fmt<FMT_MXFP8>()) != cudaSuccess) return e;
+  if ((e = set_attrs_fmt<FMT_FP8T>()) != cudaSuccess) return e;
   if ((e = set_swap_attrs_fmt<FMT_BF16>()) != cudaSuccess) return e;
   return set_swap_attrs_fmt<FMT_FP8>();
 }
@@ -297,6 +299,7 @@ cudaError_t launch_gemm_fmt(int fmt, bool swap, const GemmArgs& a, const CUtenso
     case FMT_BF16: return launch_gemm<FMT_BF16, EPI>(a, ta, grid, st);
     case FMT_FP8: return launch_gemm<FMT_FP8, EPI>(a, ta, grid, st);
     case FMT_MXFP8: return launch_gemm<FMT_MXFP8, EPI>(a, ta, grid, st);
+    case FMT_FP8T: return launch_gemm<FMT_FP8T, EPI>(a, ta, grid, st);
     default: return launch_gemm<FMT_NVFP4, EPI>(a, ta, grid, st);
   }
 }
@@ -388,7 +391,7 @@ struct FfnPlan {
 // The GEMMs' tile regime for this problem (MOE_TILE_AUTO resolved).
 bool small_m_tiles(const moe_problem_t* p) {
   if (p->tile_regime == MOE_TILE_SMALL_M) return true;
-  if (p->tile_regime == MOE_TILE_LARGE_M || p->format == FMT_NVFP4 || p->format == FMT_MXFP8) return false;
+  if (p->tile_regime == MOE_TILE_LARGE_M || (p->format != FMT_BF16 && p->format != FMT_FP8)) return false;
   return p->num_tokens * p->num_topk <= int64_t(64) * p->num_experts;
 }
 
@@ -464,7 +467,12 @@ moe_status_t plan_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_we
   a.sb = static_cast<const float*>(w->w13_scale);
   a.sb_nb = 2 * I / 128;
   a.sb_kb = H / 128;
-  a.alpha = w->gate_up_expert_scales;
+  // per-expert output scaling: NVFP4's products, or FP8 per-tensor's weight
+  // scales times the activation scale (L1) / the re-quant scale (L2)
+  const bool per_tensor = fmt == FMT_FP8T;
+  a.alpha = per_tensor ? static_cast<const float*>(w->w13_scale) : w->gate_up_expert_scales;
+  a.alpha_scalar = per_tensor ? static_cast<const float*>(act->x_scale) : nullptr;
+  a.alpha_e2 = nullptr;
   a.x_row_scale = static_cast<const uint16_t*>(act->x_rowwise_scale);
   a.c_in = w->c_input_scales;
   a.h_out = b.h;
@@ -505,7 +513,9 @@ moe_status_t plan_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_we
   a2.sb = static_cast<const float*>(w->w2_scale);
   a2.sb_nb = H / 128;
   a2.sb_kb = I / 128;
-  a2.alpha = w->down_expert_scales;
+  a2.alpha = per_tensor ? static_cast<const float*>(w->w2_scale) : w->down_expert_scales;
+  a2.alpha_scalar = nullptr;
+  a2.alpha_e2 = per_tensor ? w->c_input_scales : nullptr;
   a2.out = out;
   pl.grid2 = std::max(1, int(std::min<int64_t>(nsm, mtiles_bound * a2.n_tiles)));
   return MOE_OK;
@@ -567,6 +577,8 @@ moe_status_t check_act_weights(const moe_problem_t* p, const moe_act_t* act, con
   if (p->format == MOE_FMT_FP8_E4M3_B128 && (!w->w13_scale || !w->w2_scale)) return MOE_ERR_INVALID_ARG;
   if (p->format == MOE_FMT_NVFP4 &&
       (!w->gate_up_expert_scales || !w->down_expert_scales || !w->c_input_scales))
+    return MOE_ERR_INVALID_ARG;
+  if (p->format == MOE_FMT_FP8_PER_TENSOR && (!w->w13_scale || !w->w2_scale || !w->c_input_scales))
     return MOE_ERR_INVALID_ARG;
   // rowwise activation scales exist for NVFP4 only
   if (act->x_rowwise_scale && p->format != MOE_FMT_NVFP4) return MOE_ERR_INVALID_ARG;
@@ -999,6 +1011,7 @@ moe_status_t moe_fused(const moe_problem_t* p, const moe_act_t* act, const moe_w
       e = pl.swap ? launch_fused_fmt<FMT_FP8, true>(f, pl, grid, st) : launch_fused_fmt<FMT_FP8, false>(f, pl, grid, st);
       break;
     case FMT_MXFP8: e = launch_fused_fmt<FMT_MXFP8, false>(f, pl, grid, st); break;
+    case FMT_FP8T: e = launch_fused_fmt<FMT_FP8T, false>(f, pl, grid, st); break;
     default: e = launch_fused_fmt<FMT_NVFP4, false>(f, pl, grid, st); break;
   }
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;

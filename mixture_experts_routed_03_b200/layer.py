@@ -65,9 +65,11 @@ class MoELayer:
         self.alpha1 = w.get("gate_up_expert_scales")
         self.alpha2 = w.get("down_expert_scales")
         self.c_in = w.get("c_input_scales")
-        # FP8 block scales stay logical; NVFP4 and MXFP8 scales go into the prepared blobs
-        self.w13_scale = w.get("w13_scale") if self.p["format"] == "fp8" else None
-        self.w2_scale = w.get("w2_scale") if self.p["format"] == "fp8" else None
+        # FP8 block and per-tensor scales stay logical; NVFP4 and MXFP8 scales
+        # go into the prepared blobs
+        keep = self.p["format"] in ("fp8", "fp8_tensor")
+        self.w13_scale = w.get("w13_scale") if keep else None
+        self.w2_scale = w.get("w2_scale") if keep else None
         n13, n2 = api.prepared_weights_size(self.prob)
         self.w13 = torch.empty(n13, dtype=torch.uint8, device=self.device)
         self.w2 = torch.empty(n2, dtype=torch.uint8, device=self.device)

@@ -22,6 +22,9 @@ activation encodings and FromLogits routing):
                      (x_bf16) for the per-token quantiser
   mxfp8_prefill_routed   the fp8_prefill_routed shapes in MXFP8: E4M3 with
                      UE8M0 scales per 32 (MoEActivationPack MXFP8)
+  fp8_tensor_prefill_routed  the same shapes in FP8 per-tensor: E4M3 with
+                     one FP32 scale per tensor (MoEActivationPack FP8
+                     per-tensor)
 """
 
 import math
@@ -48,6 +51,10 @@ WORKLOADS = {
     # scales per 32 elements, which the tensor cores apply themselves
     "mxfp8_prefill_routed": dict(num_tokens=16384, hidden=4096, intermediate_hidden=1536,
                                  num_experts=128, num_topk=8, format="mxfp8", routing="logits"),
+    # the same shapes with one FP32 scale per tensor: the tensor cores sum all
+    # of K and the epilogue applies the scales once
+    "fp8_tensor_prefill_routed": dict(num_tokens=16384, hidden=4096, intermediate_hidden=1536,
+                                      num_experts=128, num_topk=8, format="fp8_tensor", routing="logits"),
 }
 
 # Typical magnitudes of the drawn values.
@@ -184,6 +191,21 @@ def make_inputs(p, seed=0, device="cpu"):
         d["gate_up_expert_scales"] = (w13_global * x_global).to(torch.float32)
         d["down_expert_scales"] = (w2_global * c_in).to(torch.float32)
         d["c_input_scales"] = c_in.to(torch.float32)
+    elif fmt == "fp8_tensor":
+        # one FP32 scale for the activations and one per expert matrix; the
+        # intermediate's static re-quant scale G with 448 * G above |h|
+        d["x"] = _e4m3_codes((M, H), g, device)
+        d["x_scale"] = _uniform((1,), 0.5, 1.5, g, device) * (X_STD / FP8_CODE_STD)
+        d["w13"] = torch.empty((Ew, 2 * I, H), dtype=torch.uint8, device=device)
+        d["w2"] = torch.empty((Ew, H, I), dtype=torch.uint8, device=device)
+        for e in range(Ew):
+            d["w13"][e] = _e4m3_codes((2 * I, H), g, device)
+            d["w2"][e] = _e4m3_codes((H, I), g, device)
+        d["w13_scale"] = _uniform((Ew,), 0.5, 1.5, g, device) * (W_STD / FP8_CODE_STD)
+        d["w2_scale"] = _uniform((Ew,), 0.5, 1.5, g, device) * (W_STD / FP8_CODE_STD)
+        c = float(p.get("activation_clamp", 10.0))
+        bound = (c * (c + 1.0) if p.get("activation") == "swigluoai" else c * c) if math.isfinite(c) else 1000.0
+        d["c_input_scales"] = (_uniform((Ew,), 1.0, 1.2, g, device) * (bound / 448.0)).to(torch.float32)
     elif fmt == "mxfp8":
         # power-of-two scales around X_STD / FP8_CODE_STD = 2^-6 (codes
         # 120..122) and W_STD / FP8_CODE_STD ~ 2^-11.6 (codes 115..117)

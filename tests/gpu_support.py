@@ -10,7 +10,7 @@ from oracle import formats as F
 from oracle import moe as O
 
 # max|err| bounds of the FFN output, relative to rms(oracle output)
-TOL = {"bf16": 5e-3, "fp8": 2e-2, "nvfp4": 2e-2, "mxfp8": 2e-2}
+TOL = {"bf16": 5e-3, "fp8": 2e-2, "nvfp4": 2e-2, "mxfp8": 2e-2, "fp8_tensor": 2e-2}
 # An intermediate code may differ from the oracle's only if it is the correct
 # rounding of a value within this distance of the oracle's pre-rounding FP32
 # value, relative to that value (the kernel's FP32 h differs from the
@@ -144,7 +144,7 @@ class GpuResult:
         self.out = bf16_to_np(out)
         self.route = route
 
-    def rows(self, p, rows):
+    def rows(self, p, rows, host=None):
         """GPU intermediate rows -> {row: dict(values, scales, hhat)}: values =
         decoded element codes (unscaled), scales = block scales (FP8 float32,
         NVFP4 E4M3 codes, MXFP8 UE8M0 codes), hhat = dequantised row (float64,
@@ -167,6 +167,15 @@ class GpuResult:
                 s = sc[:, pr].copy()
                 out[r] = dict(codes=codes[r], values=F.e4m3_decode(codes[r]), scales=s,
                               hhat=O.dequant_intermediate("fp8", codes[r][None], s[None], I)[0])
+            return out
+        if fmt == "fp8_tensor":
+            # one static scale per expert (an input, not in the workspace)
+            codes = self.codes[: R_total * I].reshape(R_total, I)
+            for r in rows:
+                e, _ = row_scale_positions(self.lay_h, r)
+                G = np.float32(host["c_input_scales"][e])
+                out[r] = dict(codes=codes[r], values=F.e4m3_decode(codes[r]), scales=np.array([G]),
+                              hhat=O.dequant_intermediate("fp8_tensor", codes[r][None], np.array([G]), I)[0])
             return out
         if fmt == "mxfp8":
             codes = self.codes[: R_total * I].reshape(R_total, I)
@@ -270,6 +279,9 @@ def _compare_codes(p, host, e, it, g, stats):
         assert np.all(np.abs(s_g - s_o) <= SCALE_REL * np.abs(s_o)), \
             f"FP8 block scales differ: {s_g} vs {s_o}"
         ref_vals = F.e4m3_decode(it["codes"])
+    elif fmt == "fp8_tensor":
+        table = "e4m3"
+        ref_vals = F.e4m3_decode(it["codes"]).astype(np.float64)
     elif fmt == "mxfp8":
         table = "e4m3"
         ref_vals = F.e4m3_decode(it["codes"]).astype(np.float64)
@@ -331,7 +343,7 @@ def _compare_codes(p, host, e, it, g, stats):
     stats["code_vals"] += diff.size
     if diff.any():
         # quantisation blocks: the whole row (BF16), 128 (FP8), 16 (NVFP4) or 32 (MXFP8) values
-        scale = block_max(pre, {"bf16": I, "fp8": 128, "nvfp4": 16, "mxfp8": 32}[fmt])
+        scale = block_max(pre, {"bf16": I, "fp8": 128, "nvfp4": 16, "mxfp8": 32, "fp8_tensor": I}[fmt])
         ok = rounding_of_nearby(table, got_vals[diff], pre[diff], scale[diff])
         assert ok.all(), (f"{fmt} intermediate codes are not a rounding of the oracle's value: GPU "
                           f"{got_vals[diff][~ok][:8]} oracle {ref_vals[diff][~ok][:8]} "
@@ -367,7 +379,7 @@ def check_against_oracle(p, host, res, tokens, label="", ref=None):
         ref = oracle_reference(p, host, tokens)
     slot_to_row = res.lay_h["slot_to_row"]
     rows = [int(slot_to_row[t * k + j]) for t in tokens for j in range(k) if slot_to_row[t * k + j] >= 0]
-    gi = res.rows(p, rows)
+    gi = res.rows(p, rows, host)
 
     # (a) codes
     stats = dict(code_flips=0, scale_flips=0, code_vals=0)

@@ -65,7 +65,8 @@ def _prob(**kw):
     (dict(activation="swigluoai", activation_alpha=float("inf")), api.MOE_ERR_INVALID_ARG),
     (dict(shared_expert=-1), api.MOE_ERR_INVALID_ARG),
     (dict(num_experts=1024, num_topk=2, shared_expert=1), api.MOE_ERR_UNSUPPORTED),
-    (dict(format=4), api.MOE_ERR_INVALID_ARG),
+    (dict(format=5), api.MOE_ERR_INVALID_ARG),
+    (dict(format="fp8_tensor", tile_regime="small_m"), api.MOE_ERR_UNSUPPORTED),
 ])
 def test_geometry_validation(lib, kw, code):
     n = ctypes.c_size_t(0)
@@ -74,7 +75,7 @@ def test_geometry_validation(lib, kw, code):
 
 
 def test_valid_geometry_and_sizes(lib):
-    for fmt, eb in (("bf16", 2.0), ("fp8", 1.0), ("nvfp4", 0.5), ("mxfp8", 1.0)):
+    for fmt, eb in (("bf16", 2.0), ("fp8", 1.0), ("nvfp4", 0.5), ("mxfp8", 1.0), ("fp8_tensor", 1.0)):
         p = _prob(format=fmt, hidden=512, intermediate_hidden=256)
         assert api.workspace_size(p) > 0
         a, b = api.prepared_weights_size(p)

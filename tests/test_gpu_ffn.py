@@ -50,6 +50,8 @@ SMALL = [
     ("nvfp4", 333, 1024, 512, 5, 2),
     ("mxfp8", 200, 512, 256, 6, 3),
     ("mxfp8", 700, 1024, 384, 3, 2),   # several m and n tiles, ragged
+    ("fp8_tensor", 200, 512, 256, 6, 3),
+    ("fp8_tensor", 700, 1024, 384, 3, 2),
 ]
 
 
@@ -75,7 +77,8 @@ def test_ffn_parity_both_tile_regimes(fmt, M, H, I, E, k, regime):
 
 
 @pytest.mark.parametrize("fmt,regime", [("bf16", "large_m"), ("fp8", "large_m"), ("nvfp4", "large_m"),
-                                        ("mxfp8", "large_m"), ("bf16", "small_m"), ("fp8", "small_m")])
+                                        ("mxfp8", "large_m"), ("fp8_tensor", "large_m"), ("bf16", "small_m"),
+                                        ("fp8", "small_m")])
 def test_staged_mode_and_deterministic_combine(fmt, regime):
     """Staged rows + the deterministic gather-combine meet the format's own
     tolerance; the combine gives the same bytes twice."""
@@ -95,7 +98,7 @@ def test_staged_mode_and_deterministic_combine(fmt, regime):
     assert torch.equal(o1, o2)
 
 
-@pytest.mark.parametrize("fmt", ["bf16", "fp8", "nvfp4", "mxfp8"])
+@pytest.mark.parametrize("fmt", ["bf16", "fp8", "nvfp4", "mxfp8", "fp8_tensor"])
 def test_clamp_active(fmt):
     """Weights scaled up so that more than 20% of g and u pass +-c: the clamp
     is exercised in every format, chain and single launch."""
@@ -106,7 +109,7 @@ def test_clamp_active(fmt):
     if fmt == "bf16":
         d["w13"] = (d["w13"].view(torch.bfloat16).float() * 60).to(torch.bfloat16).view(torch.int16)
         host["w13"] = d["w13"].cpu().view(torch.int16).numpy().view(np.uint16)
-    elif fmt == "fp8":
+    elif fmt in ("fp8", "fp8_tensor"):
         d["w13_scale"] = d["w13_scale"] * 60
         host["w13_scale"] = d["w13_scale"].cpu().numpy()
     elif fmt == "mxfp8":
@@ -126,7 +129,7 @@ def test_clamp_active(fmt):
     _check_both_paths(p, d, host, L, np.arange(M), f"clamp/{fmt}")
 
 
-@pytest.mark.parametrize("fmt", ["bf16", "fp8", "nvfp4", "mxfp8"])
+@pytest.mark.parametrize("fmt", ["bf16", "fp8", "nvfp4", "mxfp8", "fp8_tensor"])
 def test_skipped_and_duplicate_slots(fmt):
     M, H, I, E, k = 40, 512, 256, 3, 3
     p = _small(fmt, M, H, I, E, k)
@@ -140,7 +143,7 @@ def test_skipped_and_duplicate_slots(fmt):
     _check_both_paths(p, d, host, L, np.arange(M), f"skip/dup/{fmt}")
 
 
-@pytest.mark.parametrize("fmt", ["bf16", "fp8", "nvfp4", "mxfp8"])
+@pytest.mark.parametrize("fmt", ["bf16", "fp8", "nvfp4", "mxfp8", "fp8_tensor"])
 def test_all_tokens_one_expert_and_single_expert(fmt):
     for E, k in ((1, 1), (4, 1)):
         M, H, I = 260, 512, 256
@@ -157,7 +160,7 @@ def test_all_tokens_one_expert_and_single_expert(fmt):
 
 @pytest.mark.parametrize("name,ntok", [("tiny_bf16", 16), ("fp8_block", 96), ("nvfp4_decode", 24),
                                        ("nvfp4_prefill", 24), ("fp8_prefill_routed", 48),
-                                       ("mxfp8_prefill_routed", 48)])
+                                       ("mxfp8_prefill_routed", 48), ("fp8_tensor_prefill_routed", 48)])
 def test_full_size_workloads_sampled(name, ntok):
     """The full-size workloads through moe_fused, the launch the benchmark
     times: routing (in-kernel for the logits workload) and the whole layout
@@ -194,7 +197,8 @@ def test_full_size_workloads_sampled(name, ntok):
 
 
 @pytest.mark.parametrize("fmt,regime", [("bf16", "large_m"), ("bf16", "small_m"), ("fp8", "large_m"),
-                                        ("fp8", "small_m"), ("nvfp4", "large_m"), ("mxfp8", "large_m")])
+                                        ("fp8", "small_m"), ("nvfp4", "large_m"), ("mxfp8", "large_m"),
+                                        ("fp8_tensor", "large_m")])
 def test_swigluoai_activation(fmt, regime):
     """The clamped swigluoai activation (Struct_mega_ffn_ep_combine_send,
     clamp_activation) with slope 1.702 and clamp 7, weights scaled so that
@@ -206,7 +210,7 @@ def test_swigluoai_activation(fmt, regime):
     if fmt == "bf16":
         d["w13"] = (d["w13"].view(torch.bfloat16).float() * 40).to(torch.bfloat16).view(torch.int16)
         host["w13"] = d["w13"].cpu().view(torch.int16).numpy().view(np.uint16)
-    elif fmt == "fp8":
+    elif fmt in ("fp8", "fp8_tensor"):
         d["w13_scale"] = d["w13_scale"] * 40
         host["w13_scale"] = d["w13_scale"].cpu().numpy()
     elif fmt == "mxfp8":
