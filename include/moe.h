@@ -148,7 +148,7 @@ typedef struct {
  *   SWIGLUOAI  h = min(g,c) * sigmoid(a * min(g,c)) * (clamp(u,-c,c) + 1),
  *              a = activation_alpha (Struct_mega_ffn_ep_combine_send
  *              clamp_activation: the clamped "swigluoai" activation, whose
- *              constants the dispatch supplies). */
+ *              constants come from the dispatch code). */
 typedef enum {
   MOE_ACT_SWIGLU = 0,
   MOE_ACT_SWIGLUOAI = 1

@@ -275,7 +275,7 @@ def swigluoai(g, u, clamp, alpha):
     float64.
 
     Struct_mega_ffn_ep_combine_send, ``clamp_activation``: the clamped
-    ("swigluoai") L1 activation, whose constants the dispatch supplies.  Read
+    ("swigluoai") L1 activation; its constants come from the dispatch code.  Read
     as the SwiGLU variant with a sigmoid slope alpha on the gate and a bias of
     1 on the up branch (the pages print neither; alpha is an input), with the
     same clamps as clamped_swiglu: the gate from above, the up branch on both
