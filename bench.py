@@ -86,17 +86,27 @@ def workload(args):
     return workloads.problem(args.workload, **over)
 
 
+def _code_only(text):
+    """C/C++/CUDA source without its comments and blank lines (a comment edit
+    leaves the compiled kernels, and so a measured traffic figure, unchanged)."""
+    import re
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+
+
 def kernel_sources_sha():
-    """SHA-256 over the CUDA sources and the C header (identifies the kernels
-    a stored ncu traffic figure was measured on)."""
+    """SHA-256 over the code (comments removed) of the CUDA sources and the C
+    header: identifies the kernels a stored ncu traffic figure was measured
+    on; any code change drops the figure."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "mixture_experts_routed_03_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
         if name.endswith((".cu", ".cuh", ".h")):
             h.update(name.encode())
-            h.update(open(os.path.join(csrc, name), "rb").read())
-    h.update(open(os.path.join(ROOT, "include", "moe.h"), "rb").read())
+            h.update(_code_only(open(os.path.join(csrc, name)).read()).encode())
+    h.update(_code_only(open(os.path.join(ROOT, "include", "moe.h")).read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -2,7 +2,7 @@
 //
 // One persistent, warp-specialised kernel template serves both legs of the
 // expert FFN (Struct_mega_ffn_ep_combine_send: "L1" gate_up and "L2" down,
-// walking one shared active-expert list) in three element formats:
+// walking one shared active-expert list) in five element formats:
 //
 //   BF16   tcgen05.mma kind::f16, FP32 accumulation over all of K in TMEM
 //   NVFP4  tcgen05.mma kind::mxf4nvf4 block_scale scale_vec::4X: e2m1
