@@ -322,10 +322,11 @@ moe_status_t moe_permute(const moe_problem_t* problem, const int64_t* topk_idx,
  * scatter-reduces w * y into `out` (MOE_OUT_ACCUMULATE) or stores y per row
  * (MOE_OUT_STAGED).  topk_weights fp32 [M, k] (read in accumulate mode).
  * If `intermediate` is not NULL the re-quantised intermediate is ALSO kept
- * there for inspection: codes [R, I] (BF16: 2 bytes, FP8 and MXFP8: 1,
- * NVFP4: 1/2 byte per element) at byte 0, followed at the byte offset
- * `scale_offset` of moe_get_intermediate_size by its scales (FP8: fp32 [I/128][P];
- * NVFP4: 512-byte tiles [P/128][I/64]; MXFP8: 512-byte tiles [P/128][I/128];
+ * there for inspection: codes [R, I] (BF16: 2 bytes, FP8, FP8 per-tensor and
+ * MXFP8: 1, NVFP4: 1/2 byte per element) at byte 0, followed at the byte
+ * offset `scale_offset` of moe_get_intermediate_size by its scales (FP8:
+ * fp32 [I/128][P]; NVFP4: 512-byte tiles [P/128][I/64]; MXFP8: 512-byte
+ * tiles [P/128][I/128]; FP8 per-tensor: none, its scale is c_input_scales;
  * P = padded rows, a_scale_offsets[E]).
  * Size it with moe_get_intermediate_size. */
 moe_status_t moe_ffn(const moe_problem_t* problem, const moe_act_t* act,

@@ -45,7 +45,10 @@ class MoELayer:
              activation_clamp, format, num_tokens = the largest batch served)
     weights: dict of device tensors w13, w13_scale, w2, w2_scale and, for
              NVFP4, gate_up_expert_scales, down_expert_scales, c_input_scales
-             (logical layouts of include/moe.h; the weights are prepared here)
+             (FP8 per-tensor: c_input_scales) in the logical layouts of
+             include/moe.h; the weights are prepared here
+    p may also carry "shared_expert" (0/1), "activation" ("swiglu" |
+    "swigluoai") and "activation_alpha"
     p may also carry "tile_regime" ("auto", "large_m", "small_m")
     """
 
