@@ -82,7 +82,13 @@ def workload(args):
     over = {}
     for kv in args.set:
         k, v = kv.split("=", 1)
-        over[k] = type(workloads.WORKLOADS[args.workload].get(k, 0))(v) if k in workloads.WORKLOADS[args.workload] else float(v)
+        if k in workloads.WORKLOADS[args.workload]:
+            over[k] = type(workloads.WORKLOADS[args.workload][k])(v)
+        else:
+            try:
+                over[k] = float(v)
+            except ValueError:       # a named option, e.g. tile_regime=pair
+                over[k] = v
     return workloads.problem(args.workload, **over)
 
 
