@@ -179,6 +179,11 @@ ACTIVATIONS = {"swiglu": 0, "swigluoai": 1}
 def problem(num_tokens, hidden, intermediate_hidden, num_experts, num_topk,
             activation_clamp=10.0, format="bf16", fast_math=1, tile_regime="auto", shared_expert=0,
             activation="swiglu", activation_alpha=1.702):
+    """A moe_problem_t.  format: a FORMATS name or code; tile_regime: a
+    TILE_REGIMES name or code; shared_expert: 0 or 1 (a fused shared expert,
+    one more expert and slot after the routing); activation: "swiglu" or
+    "swigluoai", whose gate slope is activation_alpha (1.702 by default, one
+    public model's value; the pages leave it to the caller)."""
     fmt = FORMATS[format] if isinstance(format, str) else int(format)
     clamp = float(activation_clamp)
     regime = TILE_REGIMES[tile_regime] if isinstance(tile_regime, str) else int(tile_regime)
