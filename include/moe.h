@@ -159,9 +159,10 @@ typedef enum {
  * when the routed rows average at most 64 per expert (num_tokens*num_topk <=
  * 64*num_experts), else LARGE_M.  LARGE_M: 128 routed rows x 256 weight rows
  * per tile.  SMALL_M: the operands swapped, 256 weight rows x 32 routed rows
- * per tile, so the tensor work follows the routed rows that exist; BF16 and
- * FP8 only (MOE_ERR_UNSUPPORTED for NVFP4, MXFP8 and FP8 per-tensor).  Results agree between regimes
- * up to FP32 summation order. */
+ * per tile, so the tensor work follows the routed rows that exist; every
+ * format (NVFP4 and MXFP8 with the routed rows' block scales as the MMA's
+ * N-side scale factors).  Results agree between regimes up to FP32
+ * summation order. */
 typedef enum {
   MOE_TILE_AUTO = 0,
   MOE_TILE_LARGE_M = 1,

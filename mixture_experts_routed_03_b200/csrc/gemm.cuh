@@ -205,6 +205,9 @@ struct GemmArgs {
   int x_row_bytes;
   const float* x_sc;
   int x_sc_ld;
+  // ... and (NVFP4, MXFP8) the byte scales of x, [M][x_sf_ld]
+  const uint8_t* x_sf_rows;
+  int x_sf_ld;
 };
 
 struct TileInfo {

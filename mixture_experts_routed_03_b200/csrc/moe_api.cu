@@ -49,8 +49,6 @@ moe_status_t check_problem(const moe_problem_t* p) {
   if (E_all > 1024) return MOE_ERR_UNSUPPORTED;
   if (std::isnan(p->activation_clamp) || !(p->activation_clamp > 0.0f)) return MOE_ERR_INVALID_ARG;
   if (p->tile_regime < MOE_TILE_AUTO || p->tile_regime > MOE_TILE_SMALL_M) return MOE_ERR_INVALID_ARG;
-  if (p->tile_regime == MOE_TILE_SMALL_M && p->format != MOE_FMT_BF16 && p->format != MOE_FMT_FP8_E4M3_B128)
-    return MOE_ERR_UNSUPPORTED;
   if (p->format == MOE_FMT_NVFP4 && p->intermediate_hidden % 256 != 0) return MOE_ERR_UNSUPPORTED;
   const int64_t R = p->num_tokens * k_all;
   if (R > (int64_t(1) << 30)) return MOE_ERR_UNSUPPORTED;
@@ -265,7 +263,10 @@ cudaError_t set_all_attrs() {
   if ((e = set_attrs_fmt<FMT_MXFP8>()) != cudaSuccess) return e;
   if ((e = set_attrs_fmt<FMT_FP8T>()) != cudaSuccess) return e;
   if ((e = set_swap_attrs_fmt<FMT_BF16>()) != cudaSuccess) return e;
-  return set_swap_attrs_fmt<FMT_FP8>();
+  if ((e = set_swap_attrs_fmt<FMT_FP8>()) != cudaSuccess) return e;
+  if ((e = set_swap_attrs_fmt<FMT_NVFP4>()) != cudaSuccess) return e;
+  if ((e = set_swap_attrs_fmt<FMT_MXFP8>()) != cudaSuccess) return e;
+  return set_swap_attrs_fmt<FMT_FP8T>();
 }
 
 bool ensure_init() {
@@ -293,8 +294,15 @@ cudaError_t launch_swap(const GemmArgs& a, const CUtensorMap& ta, int grid, cuda
 template <int EPI>
 cudaError_t launch_gemm_fmt(int fmt, bool swap, const GemmArgs& a, const CUtensorMap& ta, int grid,
                             cudaStream_t st) {
-  if (swap) return fmt == FMT_BF16 ? launch_swap<FMT_BF16, EPI>(a, ta, grid, st)
-                                   : launch_swap<FMT_FP8, EPI>(a, ta, grid, st);
+  if (swap) {
+    switch (fmt) {
+      case FMT_BF16: return launch_swap<FMT_BF16, EPI>(a, ta, grid, st);
+      case FMT_FP8: return launch_swap<FMT_FP8, EPI>(a, ta, grid, st);
+      case FMT_MXFP8: return launch_swap<FMT_MXFP8, EPI>(a, ta, grid, st);
+      case FMT_FP8T: return launch_swap<FMT_FP8T, EPI>(a, ta, grid, st);
+      default: return launch_swap<FMT_NVFP4, EPI>(a, ta, grid, st);
+    }
+  }
   switch (fmt) {
     case FMT_BF16: return launch_gemm<FMT_BF16, EPI>(a, ta, grid, st);
     case FMT_FP8: return launch_gemm<FMT_FP8, EPI>(a, ta, grid, st);
@@ -457,6 +465,10 @@ moe_status_t plan_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_we
     a.x_row_bytes = x_row_bytes(fmt, H);
     a.x_sc = static_cast<const float*>(act->x_scale);   // FP8; null for BF16
     a.x_sc_ld = H / 128;
+    if (fmt == FMT_NVFP4 || fmt == FMT_MXFP8) {
+      a.x_sf_rows = static_cast<const uint8_t*>(act->x_scale);
+      a.x_sf_ld = fmt == FMT_NVFP4 ? H / 16 : H / 32;
+    }
   }
   a.src_info = b.src_info;
   a.topk_weights = topk_weights;
@@ -491,6 +503,7 @@ moe_status_t plan_ffn(const moe_problem_t* p, const moe_act_t* act, const moe_we
   a2 = a;
   a2.x_rows = nullptr;   // the down leg reads the intermediate through its TMA map
   a2.x_sc = nullptr;
+  a2.x_sf_rows = nullptr;
   a2.x_row_scale = nullptr;
   a2.k_stages = h_row_bytes(fmt, I) / 128;
   a2.n_tiles = H / 256;
@@ -1010,9 +1023,15 @@ moe_status_t moe_fused(const moe_problem_t* p, const moe_act_t* act, const moe_w
     case FMT_FP8:
       e = pl.swap ? launch_fused_fmt<FMT_FP8, true>(f, pl, grid, st) : launch_fused_fmt<FMT_FP8, false>(f, pl, grid, st);
       break;
-    case FMT_MXFP8: e = launch_fused_fmt<FMT_MXFP8, false>(f, pl, grid, st); break;
-    case FMT_FP8T: e = launch_fused_fmt<FMT_FP8T, false>(f, pl, grid, st); break;
-    default: e = launch_fused_fmt<FMT_NVFP4, false>(f, pl, grid, st); break;
+    case FMT_MXFP8:
+      e = pl.swap ? launch_fused_fmt<FMT_MXFP8, true>(f, pl, grid, st) : launch_fused_fmt<FMT_MXFP8, false>(f, pl, grid, st);
+      break;
+    case FMT_FP8T:
+      e = pl.swap ? launch_fused_fmt<FMT_FP8T, true>(f, pl, grid, st) : launch_fused_fmt<FMT_FP8T, false>(f, pl, grid, st);
+      break;
+    default:
+      e = pl.swap ? launch_fused_fmt<FMT_NVFP4, true>(f, pl, grid, st) : launch_fused_fmt<FMT_NVFP4, false>(f, pl, grid, st);
+      break;
   }
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

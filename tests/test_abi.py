@@ -56,8 +56,6 @@ def _prob(**kw):
     (dict(format=7), api.MOE_ERR_INVALID_ARG),
     (dict(format="nvfp4", intermediate_hidden=384), api.MOE_ERR_UNSUPPORTED),
     (dict(tile_regime=3), api.MOE_ERR_INVALID_ARG),
-    (dict(format="nvfp4", tile_regime="small_m"), api.MOE_ERR_UNSUPPORTED),
-    (dict(format="mxfp8", tile_regime="small_m"), api.MOE_ERR_UNSUPPORTED),
     (dict(shared_expert=2), api.MOE_ERR_INVALID_ARG),
     (dict(activation=2), api.MOE_ERR_INVALID_ARG),
     (dict(activation="swigluoai", activation_alpha=0.0), api.MOE_ERR_INVALID_ARG),
@@ -66,7 +64,6 @@ def _prob(**kw):
     (dict(shared_expert=-1), api.MOE_ERR_INVALID_ARG),
     (dict(num_experts=1024, num_topk=2, shared_expert=1), api.MOE_ERR_UNSUPPORTED),
     (dict(format=5), api.MOE_ERR_INVALID_ARG),
-    (dict(format="fp8_tensor", tile_regime="small_m"), api.MOE_ERR_UNSUPPORTED),
 ])
 def test_geometry_validation(lib, kw, code):
     n = ctypes.c_size_t(0)
@@ -142,6 +139,11 @@ def test_tile_regime_resolution(lib):
                                  num_topk=2)) == "large_m"
     assert api.tile_regime(_prob(num_tokens=16, format="mxfp8", num_experts=8, num_topk=2)) == "large_m"
     assert api.tile_regime(_prob(num_tokens=16, tile_regime="large_m")) == "large_m"
+    # every format has both regimes when forced
+    for fmt in ("bf16", "fp8", "nvfp4", "mxfp8", "fp8_tensor"):
+        kw = dict(num_tokens=16, format=fmt, intermediate_hidden=256)
+        assert api.tile_regime(_prob(tile_regime="small_m", **kw)) == "small_m"
+        assert api.tile_regime(_prob(tile_regime="large_m", **kw)) == "large_m"
     assert api.tile_regime(_prob(num_tokens=100000, tile_regime="small_m")) == "small_m"
 
 

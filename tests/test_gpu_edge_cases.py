@@ -57,7 +57,8 @@ def test_one_workspace_for_several_token_counts(fmt):
 
 
 @pytest.mark.parametrize("fmt,regime", [("bf16", "small_m"), ("fp8", "large_m"), ("nvfp4", "large_m"),
-                                        ("mxfp8", "large_m")])
+                                        ("mxfp8", "large_m"), ("nvfp4", "small_m"), ("mxfp8", "small_m"),
+                                        ("fp8_tensor", "small_m")])
 def test_tokens_with_every_slot_skipped_are_zero(fmt, regime):
     M, H, I, E, k = 96, 512, 256, 4, 3
     p = _problem(fmt, M, H, I, E, k, tile_regime=regime)

@@ -64,11 +64,11 @@ def test_ffn_parity_small(fmt, M, H, I, E, k):
 
 
 @pytest.mark.parametrize("regime", ["large_m", "small_m"])
-@pytest.mark.parametrize("fmt,M,H,I,E,k", [c for c in SMALL if c[0] in ("bf16", "fp8")])
+@pytest.mark.parametrize("fmt,M,H,I,E,k", SMALL)
 def test_ffn_parity_both_tile_regimes(fmt, M, H, I, E, k, regime):
     """Both GEMM tile regimes (128 routed rows x 256 weight rows, and the
-    swapped operands with 32 routed rows) on every BF16 / FP8 case, through
-    the chain and the single launch."""
+    swapped operands with 32 routed rows) on every case of every format,
+    through the chain and the single launch."""
     p = _small(fmt, M, H, I, E, k, regime=regime)
     d, host = S.make(p, seed=3)
     L = layer.MoELayer(p, S.weights_of(d), device=S.device())
@@ -76,9 +76,10 @@ def test_ffn_parity_both_tile_regimes(fmt, M, H, I, E, k, regime):
     _check_both_paths(p, d, host, L, np.arange(M), f"{fmt}/{regime}")
 
 
-@pytest.mark.parametrize("fmt,regime", [("bf16", "large_m"), ("fp8", "large_m"), ("nvfp4", "large_m"),
-                                        ("mxfp8", "large_m"), ("fp8_tensor", "large_m"), ("bf16", "small_m"),
-                                        ("fp8", "small_m")])
+ALL_FMT_REGIMES = [(f, r) for r in ("large_m", "small_m") for f in ("bf16", "fp8", "nvfp4", "mxfp8", "fp8_tensor")]
+
+
+@pytest.mark.parametrize("fmt,regime", ALL_FMT_REGIMES)
 def test_staged_mode_and_deterministic_combine(fmt, regime):
     """Staged rows + the deterministic gather-combine meet the format's own
     tolerance; the combine gives the same bytes twice."""
@@ -98,13 +99,13 @@ def test_staged_mode_and_deterministic_combine(fmt, regime):
     assert torch.equal(o1, o2)
 
 
-@pytest.mark.parametrize("fmt", ["bf16", "fp8", "nvfp4", "mxfp8", "fp8_tensor"])
-def test_clamp_active(fmt):
+@pytest.mark.parametrize("fmt,regime", ALL_FMT_REGIMES)
+def test_clamp_active(fmt, regime):
     """Weights scaled up so that more than 20% of g and u pass +-c: the clamp
-    is exercised in every format, chain and single launch."""
+    is exercised in every format and tile regime, chain and single launch."""
     M, H, I, E, k = 160, 512, 256, 3, 2
     clamp = 0.5
-    p = _small(fmt, M, H, I, E, k, clamp=clamp)
+    p = _small(fmt, M, H, I, E, k, clamp=clamp, regime=regime)
     d, host = S.make(p, seed=3)
     if fmt == "bf16":
         d["w13"] = (d["w13"].view(torch.bfloat16).float() * 60).to(torch.bfloat16).view(torch.int16)
@@ -126,7 +127,7 @@ def test_clamp_active(fmt):
     if fmt == "nvfp4":
         gu = gu * float(host["gate_up_expert_scales"][0])
     assert np.mean(np.abs(gu[:, :I]) > clamp) > 0.2 and np.mean(np.abs(gu[:, I:]) > clamp) > 0.2
-    _check_both_paths(p, d, host, L, np.arange(M), f"clamp/{fmt}")
+    _check_both_paths(p, d, host, L, np.arange(M), f"clamp/{fmt}/{regime}")
 
 
 @pytest.mark.parametrize("fmt", ["bf16", "fp8", "nvfp4", "mxfp8", "fp8_tensor"])
@@ -196,9 +197,7 @@ def test_full_size_workloads_sampled(name, ntok):
     assert np.mean(~S.close_bf16(a, b, S.TOL[p["format"]] * S.rms(a))) < 1e-3
 
 
-@pytest.mark.parametrize("fmt,regime", [("bf16", "large_m"), ("bf16", "small_m"), ("fp8", "large_m"),
-                                        ("fp8", "small_m"), ("nvfp4", "large_m"), ("mxfp8", "large_m"),
-                                        ("fp8_tensor", "large_m")])
+@pytest.mark.parametrize("fmt,regime", ALL_FMT_REGIMES)
 def test_swigluoai_activation(fmt, regime):
     """The clamped swigluoai activation (Struct_mega_ffn_ep_combine_send,
     clamp_activation) with slope 1.702 and clamp 7, weights scaled so that

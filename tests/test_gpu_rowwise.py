@@ -49,11 +49,12 @@ def test_quantizer_matches_oracle_bit_for_bit(M, H):
         assert np.all(F.e2m1_decode(g4[diff]) == 0) and np.all(F.e2m1_decode(r4[diff]) == 0)
 
 
-@pytest.mark.parametrize("name,M", [("small", 200), ("nvfp4_prefill", 512)])
-def test_layer_with_rowwise_scales_matches_oracle(name, M):
+@pytest.mark.parametrize("name,M,regime", [("small", 200, "large_m"), ("small", 200, "small_m"),
+                                           ("nvfp4_prefill", 512, "auto")])
+def test_layer_with_rowwise_scales_matches_oracle(name, M, regime):
     if name == "small":
         p = dict(num_tokens=M, hidden=1024, intermediate_hidden=512, num_experts=6, num_topk=3, format="nvfp4",
-                 routing="softmax", activation_clamp=10.0)
+                 routing="softmax", activation_clamp=10.0, tile_regime=regime)
     else:
         p = workloads.problem("nvfp4_prefill", num_tokens=M)
     d, host = S.make(p, seed=11)

@@ -27,7 +27,11 @@ def _problem(fmt, M, H, I, E, k, routing="softmax", regime="auto"):
     ("fp8", 300, 1024, 384, 8, 3, "large_m"),
     ("fp8", 64, 1024, 384, 16, 4, "small_m"),
     ("nvfp4", 200, 512, 256, 6, 3, "large_m"),
+    ("nvfp4", 48, 512, 256, 12, 3, "small_m"),
     ("mxfp8", 260, 1024, 384, 5, 2, "large_m"),
+    ("mxfp8", 64, 1024, 384, 16, 2, "small_m"),
+    ("fp8_tensor", 200, 512, 256, 6, 2, "large_m"),
+    ("fp8_tensor", 40, 512, 256, 8, 2, "small_m"),
 ])
 def test_shared_expert_parity(fmt, M, H, I, E, k, regime):
     p = _problem(fmt, M, H, I, E, k, regime=regime)
