@@ -155,8 +155,8 @@ typedef enum {
 } moe_activation_t;
 
 /* Tile shape of the grouped GEMMs (the tile-regime choice the pages make
- * between prefill and decode batches).  AUTO picks SMALL_M for BF16 and FP8
- * when the routed rows average at most 64 per expert (num_tokens*num_topk <=
+ * between prefill and decode batches).  AUTO picks SMALL_M when the routed
+ * rows average at most 64 per expert (num_tokens*num_topk <=
  * 64*num_experts), else LARGE_M.  LARGE_M: 128 routed rows x 256 weight rows
  * per tile.  SMALL_M: the operands swapped, 256 weight rows x 32 routed rows
  * per tile, so the tensor work follows the routed rows that exist; every

@@ -399,7 +399,7 @@ struct FfnPlan {
 // The GEMMs' tile regime for this problem (MOE_TILE_AUTO resolved).
 bool small_m_tiles(const moe_problem_t* p) {
   if (p->tile_regime == MOE_TILE_SMALL_M) return true;
-  if (p->tile_regime == MOE_TILE_LARGE_M || (p->format != FMT_BF16 && p->format != FMT_FP8)) return false;
+  if (p->tile_regime == MOE_TILE_LARGE_M) return false;
   return p->num_tokens * p->num_topk <= int64_t(64) * p->num_experts;
 }
 

@@ -131,13 +131,14 @@ def test_status_strings(lib):
 
 
 def test_tile_regime_resolution(lib):
-    # AUTO: swapped-operand tiles while routed rows average <= 64 per expert (BF16 / FP8)
+    # AUTO: swapped-operand tiles while routed rows average <= 64 per expert (every format)
     assert api.tile_regime(_prob(num_tokens=256, num_experts=8, num_topk=2)) == "small_m"     # 512 <= 512
     assert api.tile_regime(_prob(num_tokens=257, num_experts=8, num_topk=2)) == "large_m"
     assert api.tile_regime(_prob(num_tokens=256, format="fp8", num_experts=8, num_topk=2)) == "small_m"
     assert api.tile_regime(_prob(num_tokens=16, format="nvfp4", intermediate_hidden=256, num_experts=8,
-                                 num_topk=2)) == "large_m"
-    assert api.tile_regime(_prob(num_tokens=16, format="mxfp8", num_experts=8, num_topk=2)) == "large_m"
+                                 num_topk=2)) == "small_m"
+    assert api.tile_regime(_prob(num_tokens=16, format="mxfp8", num_experts=8, num_topk=2)) == "small_m"
+    assert api.tile_regime(_prob(num_tokens=257, format="mxfp8", num_experts=8, num_topk=2)) == "large_m"
     assert api.tile_regime(_prob(num_tokens=16, tile_regime="large_m")) == "large_m"
     # every format has both regimes when forced
     for fmt in ("bf16", "fp8", "nvfp4", "mxfp8", "fp8_tensor"):
