@@ -161,3 +161,18 @@ def test_shared_expert_sizes_are_those_of_one_more_expert_and_slot(lib):
         assert api.intermediate_size(shared) == api.intermediate_size(plain)
         assert api.workspace_offsets(shared) == api.workspace_offsets(plain)
         assert api.tile_regime(shared) == api.tile_regime(plain)
+
+
+@pytest.mark.parametrize("fmt", ["bf16", "fp8", "nvfp4", "mxfp8", "fp8_tensor"])
+def test_workspace_size_does_not_depend_on_the_tile_regime(lib, fmt):
+    """One workspace serves both tile regimes: a layer sized for its largest
+    batch (large-M tiles) also runs its small batches, which auto sends to the
+    small-M tiles."""
+    for M in (16, 5000):
+        sizes = set()
+        for regime in ("auto", "large_m", "small_m"):
+            n = ctypes.c_size_t(0)
+            p = _prob(num_tokens=M, hidden=512, intermediate_hidden=256, format=fmt, tile_regime=regime)
+            assert lib.moe_get_workspace_size(ctypes.byref(p), ctypes.byref(n)) == api.MOE_OK
+            sizes.add(n.value)
+        assert len(sizes) == 1, (fmt, M, sizes)
