@@ -169,7 +169,8 @@ typedef enum {
   MOE_TILE_SMALL_M = 2
 } moe_tile_regime_t;
 
-/* Activations (device).  x_scale is NULL for BF16.  x_rowwise_scale is
+/* Activations (device).  x is 16-byte aligned and x_scale 4-byte aligned
+ * (MOE_ERR_INVALID_ARG otherwise).  x_scale is NULL for BF16.  x_rowwise_scale is
  * NULL, or for NVFP4 activations quantised per token (EPConfig,
  * nvfp4_dyn_global_scales; moe_quantize_nvfp4_rowwise) the BF16 [M] rowwise
  * scales: row t dequantises as e2m1 * block scale * x_rowwise_scale[t], and

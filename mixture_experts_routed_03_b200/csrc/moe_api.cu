@@ -587,6 +587,9 @@ moe_status_t check_act_weights(const moe_problem_t* p, const moe_act_t* act, con
   if (!act || !w || !act->x || !w->w13 || !w->w2) return MOE_ERR_INVALID_ARG;
   if (!aligned16(act->x) || !aligned16(w->w13) || !aligned16(w->w2)) return MOE_ERR_INVALID_ARG;
   if (p->format != MOE_FMT_BF16 && !act->x_scale) return MOE_ERR_INVALID_ARG;
+  // the scales are read a 4-byte word at a time (the small-M gate_up copies
+  // a row's NVFP4 / MXFP8 scale words straight from x_scale)
+  if ((reinterpret_cast<uintptr_t>(act->x_scale) & 3) != 0) return MOE_ERR_INVALID_ARG;
   if (p->format == MOE_FMT_FP8_E4M3_B128 && (!w->w13_scale || !w->w2_scale)) return MOE_ERR_INVALID_ARG;
   if (p->format == MOE_FMT_NVFP4 &&
       (!w->gate_up_expert_scales || !w->down_expert_scales || !w->c_input_scales))

@@ -176,3 +176,20 @@ def test_workspace_size_does_not_depend_on_the_tile_regime(lib, fmt):
             assert lib.moe_get_workspace_size(ctypes.byref(p), ctypes.byref(n)) == api.MOE_OK
             sizes.add(n.value)
         assert len(sizes) == 1, (fmt, M, sizes)
+
+
+@pytest.mark.parametrize("fmt", ["fp8", "nvfp4", "mxfp8"])
+def test_misaligned_activations_rejected_before_launch(lib, fmt):
+    """x must be 16-byte aligned and x_scale 4-byte aligned; both are checked
+    before anything touches the device (the pointers are never dereferenced)."""
+    p = _prob(format=fmt, intermediate_hidden=256)
+    base = 1 << 20
+    w = api.weights(base, base, base, base, base, base, base)
+    for x, xs in ((base + 8, base), (base, base + 2), (base, base + 1)):
+        a = api.act(x, xs)
+        assert lib.moe_fused(ctypes.byref(p), ctypes.byref(a), ctypes.byref(w), base, base, None, None,
+                             base, base, 1 << 40, None) == api.MOE_ERR_INVALID_ARG, (x - base, xs - base)
+    # aligned pointers get past the checks to the workspace-size test
+    a = api.act(base, base + 4)
+    assert lib.moe_fused(ctypes.byref(p), ctypes.byref(a), ctypes.byref(w), base, base, None, None,
+                         base, base, 16, None) == api.MOE_ERR_WORKSPACE
